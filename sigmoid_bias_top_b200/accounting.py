@@ -1,0 +1,53 @@
+"""Algorithmic work of one MoE-block forward: the byte and FLOP counts that
+throughput and roofline fractions are computed from.
+
+Counts follow "LFM2.5-24B-A2B: Biased Routing, Short Convolutions and Ten KV
+Caches" (flozi.net, English page): section "The router has two different
+scores" (an expert is three matrices, 3 x 2048 x 1536 = 9,437,184 weights) and
+section "Active weights do not define resident memory" (a multiply-add counts
+as two FLOPs; the selected experts cost 2 x 38 x 4 x 3 x 2048 x 1536 FLOPs per
+token over 38 MoE layers).
+"""
+from __future__ import annotations
+
+
+def expert_weights(d: int, d_ff: int) -> int:
+    """Weights of one gated-SiLU expert: gate, up and down matrices."""
+    return 3 * d * d_ff
+
+
+def expert_flops_per_token(d: int, d_ff: int, top_k: int, n_layers: int = 1) -> int:
+    """Selected-expert matrix FLOPs per token (multiply-add = 2)."""
+    return 2 * n_layers * top_k * expert_weights(d, d_ff)
+
+
+def router_flops_per_token(d: int, n_experts: int) -> int:
+    return 2 * d * n_experts
+
+
+def decode_bytes(active_experts: int, n_tokens: int, d: int, d_ff: int, n_experts: int,
+                 w_bytes: int = 2, x_bytes: int = 2) -> int:
+    """HBM bytes a weight-streaming forward must move: the active experts'
+    weights, the fp32 router matrix, gain and bias, x read and out written.
+    Intermediates and unselected experts are not counted."""
+    return (active_experts * expert_weights(d, d_ff) * w_bytes
+            + n_experts * d * 4 + d * 4 + n_experts * 4
+            + 2 * n_tokens * d * x_bytes)
+
+
+def gate_up_bytes(active_experts: int, d: int, d_ff: int, w_bytes: int = 2) -> int:
+    """Weight bytes the packed gate/up grouped GEMM must stream."""
+    return active_experts * 2 * d_ff * d * w_bytes
+
+
+def down_bytes(active_experts: int, d: int, d_ff: int, w_bytes: int = 2) -> int:
+    return active_experts * d * d_ff * w_bytes
+
+
+def gate_up_flops(n_assign: int, d: int, d_ff: int) -> int:
+    """Tensor FLOPs of the gate/up contraction over all token-expert pairs."""
+    return 2 * n_assign * 2 * d_ff * d
+
+
+def down_flops(n_assign: int, d: int, d_ff: int) -> int:
+    return 2 * n_assign * d * d_ff

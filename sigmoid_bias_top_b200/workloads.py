@@ -1,0 +1,168 @@
+"""Seeded synthetic inputs for the sigmoid-bias top-k MoE feed-forward block.
+
+This module only draws random tensors of the shapes and distributions of the
+five workloads; it contains none of the layer's arithmetic (no norm, no
+routing, no expert math), so that the CUDA path and the CPU oracle can both be
+fed from it without sharing any computation.
+
+Shapes follow "LFM2.5-24B-A2B: Biased Routing, Short Convolutions and Ten KV
+Caches" (flozi.net, English page), section "The router has two different
+scores": hidden width 2048, 64 experts, top-4, expert intermediate 1536, a
+fp32 router matrix W_r[E x d] and a stored 64-element expert bias.
+
+Tensor layout (what the C ABI consumes):
+  x          [N, d]        f32 or bf16   residual stream (the block input)
+  norm_gain  [d]           f32           RMSNorm gain, multiplied as stored
+  router_w   [E, d]        f32           router matrix, row-major
+  bias       [E]           f32           expert bias (selection only)
+  w_gate_up  [E, 2I, d]    f32 or bf16   rows 0..I-1 = gate, rows I..2I-1 = up
+  w_down     [E, d, I]     f32 or bf16   down projection
+Distribution parameters written "N(0, v)" with v a fraction of the width
+(1/256, 1/192) are variances; "N(0, 0.02)" is a standard deviation, the usual
+initializer-range convention.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field, replace
+from typing import Dict, List, Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    n_tokens: int
+    d: int
+    n_experts: int
+    top_k: int
+    d_ff: int
+    dtype: str                      # "f32" or "bf16": x, out and expert weights
+    eps: float = 1e-6
+    routed_scale: float = 1.0
+    n_layers: int = 1
+    seed: int = 0
+    x_std: float = 1.0
+    gain_jitter: float = 0.0        # gain = 1 + N(0, jitter^2)
+    router_std: float = 0.02
+    bias_kind: str = "uniform"      # "uniform", "zero", "zipf"
+    bias_halfwidth: float = 0.05    # uniform bias in (-h, h)
+    gate_up_std: float = 0.02
+    down_std: float = 0.02
+    # skewed-load bias: b_e = zipf_scale * log p_rank(e) - zipf_tail_drop on the
+    # zipf_tail lowest ranks, with p_r proportional to r^-zipf_s
+    zipf_s: float = 1.2
+    zipf_scale: float = 0.08
+    zipf_tail: int = 4
+    zipf_tail_drop: float = 0.15
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def scaled(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+TINY_F32 = Workload(
+    name="tiny_f32_N64_d256_E16_k4_I192", n_tokens=64, d=256, n_experts=16, top_k=4,
+    d_ff=192, dtype="f32", seed=1, x_std=1.0, gain_jitter=0.0,
+    router_std=1.0 / 16.0, bias_kind="uniform", bias_halfwidth=0.5,
+    gate_up_std=1.0 / 16.0, down_std=1.0 / math.sqrt(192.0))
+
+DECODE = Workload(
+    name="decode_N32_d2048_E64_k4_I1536", n_tokens=32, d=2048, n_experts=64, top_k=4,
+    d_ff=1536, dtype="bf16", seed=2, gain_jitter=0.02, router_std=0.02,
+    bias_kind="uniform", bias_halfwidth=0.05)
+
+PREFILL = Workload(
+    name="prefill_N8192_d2048_E64_k4_I1536", n_tokens=8192, d=2048, n_experts=64,
+    top_k=4, d_ff=1536, dtype="bf16", seed=3, gain_jitter=0.02, router_std=0.02,
+    bias_kind="zero")
+
+SKEWED = Workload(
+    name="skewed_prefill_N16384_d2048_E64_k4_I1536", n_tokens=16384, d=2048,
+    n_experts=64, top_k=4, d_ff=1536, dtype="bf16", seed=4, gain_jitter=0.02,
+    router_std=0.02, bias_kind="zipf")
+
+STACKED = Workload(
+    name="stacked_decode_L38_N256_d2048_E64_k4_I1536", n_tokens=256, d=2048,
+    n_experts=64, top_k=4, d_ff=1536, dtype="bf16", seed=5, n_layers=38,
+    gain_jitter=0.02, router_std=0.02, bias_kind="uniform", bias_halfwidth=0.05)
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny": TINY_F32, "decode": DECODE, "prefill": PREFILL, "skewed": SKEWED,
+    "stacked": STACKED,
+}
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _normal(shape, std, g, device, dtype):
+    # drawn in f32 then stored in the target dtype; the stored values are the truth
+    return (torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std).to(dtype)
+
+
+def zipf_bias(w: Workload, g: torch.Generator, device) -> torch.Tensor:
+    """Expert bias for the skewed-load workload: a log-Zipf profile over ranks,
+    ranks assigned to experts by a seeded permutation."""
+    E = w.n_experts
+    r = torch.arange(1, E + 1, dtype=torch.float64)
+    p = r.pow(-w.zipf_s)
+    p = p / p.sum()
+    b_rank = w.zipf_scale * torch.log(p)
+    b_rank[E - w.zipf_tail:] -= w.zipf_tail_drop
+    perm = torch.randperm(E, generator=g, device=device).cpu()
+    b = torch.empty(E, dtype=torch.float64)
+    b[perm] = b_rank            # expert perm[r] gets rank r
+    return b.to(torch.float32).to(device)
+
+
+def make_layer(w: Workload, layer: int = 0, device="cpu",
+               seed: Optional[int] = None, with_experts: bool = True) -> Dict[str, torch.Tensor]:
+    """Weights of one MoE block (layer index selects an independent stream).
+
+    with_experts=False stops after the router tensors (same values as a full
+    draw, since the expert matrices are drawn last)."""
+    base = w.seed if seed is None else seed
+    g = _gen(device, 1_000_003 * (base + 1) + 7919 * (layer + 1))
+    E, d, I = w.n_experts, w.d, w.d_ff
+    dt = w.torch_dtype
+    gain = torch.ones(d, device=device, dtype=torch.float32)
+    if w.gain_jitter:
+        gain = gain + _normal((d,), w.gain_jitter, g, device, torch.float32)
+    router_w = _normal((E, d), w.router_std, g, device, torch.float32)
+    if w.bias_kind == "uniform":
+        bias = ((torch.rand(E, generator=g, device=device, dtype=torch.float32) * 2 - 1)
+                * w.bias_halfwidth)
+    elif w.bias_kind == "zero":
+        bias = torch.zeros(E, device=device, dtype=torch.float32)
+    elif w.bias_kind == "zipf":
+        bias = zipf_bias(w, g, device)
+    else:
+        raise ValueError(w.bias_kind)
+    out = {"norm_gain": gain.contiguous(), "router_w": router_w.contiguous(),
+           "bias": bias.contiguous()}
+    if with_experts:
+        out["w_gate_up"] = _normal((E, 2 * I, d), w.gate_up_std, g, device, dt).contiguous()
+        out["w_down"] = _normal((E, d, I), w.down_std, g, device, dt).contiguous()
+    return out
+
+
+def make_x(w: Workload, device="cpu", seed: Optional[int] = None,
+           n_tokens: Optional[int] = None) -> torch.Tensor:
+    base = w.seed if seed is None else seed
+    g = _gen(device, 7 * (base + 1) + 3)
+    n = w.n_tokens if n_tokens is None else n_tokens
+    return _normal((n, w.d), w.x_std, g, device, w.torch_dtype).contiguous()
+
+
+def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
+    """x plus the weights of every layer of the workload."""
+    layers = [make_layer(w, l, device, seed) for l in range(w.n_layers)]
+    return make_x(w, device, seed), layers

@@ -1,0 +1,36 @@
+"""Shape and FLOP accounting against the numbers the page prints."""
+from sigmoid_bias_top_b200 import accounting as A
+
+
+def test_expert_weights_per_expert():
+    # section "The router has two different scores": 3 x 2048 x 1536 = 9,437,184
+    assert A.expert_weights(2048, 1536) == 9_437_184
+
+
+def test_expert_parameter_totals():
+    # section "Active weights do not define resident memory": experts hold about
+    # 22.951 B over 38 layers; keeping 4 of 64 experts gives about 2.455 B active
+    # out of 23,971,585,280 total.
+    total_expert = 38 * 64 * A.expert_weights(2048, 1536)
+    assert total_expert == 22_951_231_488
+    assert round(total_expert / 1e9, 3) == 22.951
+    active = 23_971_585_280 - 38 * 60 * A.expert_weights(2048, 1536)
+    assert active == 2_454_805_760
+    assert round(active / 1e9, 3) == 2.455
+
+
+def test_expert_flops_per_token():
+    # 2 x 38 x 4 x 3 x 2048 x 1536 ~ 2.869 GFLOP per token
+    f = A.expert_flops_per_token(2048, 1536, top_k=4, n_layers=38)
+    assert f == 2_868_903_936
+    assert round(f / 1e9, 3) == 2.869
+    # all 64 experts would cost 16 times as much for that term
+    assert A.expert_flops_per_token(2048, 1536, 64, 38) == 16 * f
+
+
+def test_split_counts_add_up():
+    n = 8192 * 4
+    assert A.gate_up_flops(n, 2048, 1536) + A.down_flops(n, 2048, 1536) == \
+        8192 * A.expert_flops_per_token(2048, 1536, 4)
+    assert A.gate_up_bytes(56, 2048, 1536) + A.down_bytes(56, 2048, 1536) == \
+        56 * A.expert_weights(2048, 1536) * 2
