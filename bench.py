@@ -1,0 +1,406 @@
+"""Throughput of the sigmoid-bias top-k MoE feed-forward block on B200.
+
+One step = one forward of the whole block (RMSNorm, router, sigmoid, biased
+top-k, dispatch, gate/up + SiLU, down, combine + residual; all 38 blocks for
+the stacked workload) over one batch of synthetic tokens already resident in
+HBM. Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs an independent
+replica on its own batch (tokens are independent rows; no collective on the
+data path), so per-GPU work is fixed and scaling is weak; the timed region is
+bracketed by barriers and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sigmoid_bias_top_b200 import accounting as A  # noqa: E402
+from sigmoid_bias_top_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (d2048,E64,top4,I1536) + % of HBM / bf16 TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_STEPS = {"decode": 2000, "prefill": 200, "skewed": 100, "stacked": 20, "tiny": 2000}
+ROTATE = 4  # distinct weight copies cycled through (each step reads >= 1 GB > L2)
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def reduce_max(v: float, world: int, device=None) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(v: float, world: int, device=None) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_throughput(local_units: float, local_seconds: float, world: int, device=None):
+    """Whole-job units/s: units of all ranks over the slowest rank's time."""
+    units = reduce_sum(local_units, world, device)
+    secs = reduce_max(local_seconds, world, device)
+    return units / secs, secs
+
+
+# ----------------------------------------------------------------------------- peaks
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_from_profiles(kernel: str, workload: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the kernel source as it is now (source hash recorded in the summary)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"source_sha256:\s*([0-9a-f]+)", txt)
+    if not m or not h or h.group(1) != kernel_source_hash():
+        return None
+    return float(m.group(1))
+
+
+def kernel_source_hash() -> str:
+    hs = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sigmoid_bias_top_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            hs.update(open(os.path.join(csrc, f), "rb").read())
+    return hs.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def make_layers(w, device, n_copies):
+    n = w.n_layers if w.n_layers > 1 else n_copies
+    return [W.make_layer(w, l, device) for l in range(n)]
+
+
+def run_ours(args, w, world, rank, local):
+    from sigmoid_bias_top_b200 import MoeLayer
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    N = w.n_tokens
+    layers = make_layers(w, dev, ROTATE)
+    mods = [MoeLayer(l, w.top_k, w.eps, w.routed_scale, max_tokens=N) for l in layers]
+    n_rot = len(mods) if w.n_layers == 1 else 1
+    xs = [W.make_x(w, dev, seed=w.seed + 17 * rank + i) for i in range(max(n_rot, 2))]
+    outs = [torch.empty_like(xs[0]) for _ in range(2)]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        if w.n_layers > 1:  # chained blocks: h = x + MoE(RMSNorm(x))
+            h = xs[i % len(xs)]
+            for l, m in enumerate(mods):
+                dst = outs[l & 1]
+                m.forward(h, dst, stream)
+                h = dst
+        else:
+            r = i % n_rot
+            mods[r].forward(xs[r % len(xs)], outs[i & 1], stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    for m in mods:
+        assert m.status() == 0, m.status()
+
+    # routing statistics of the timed batches (distinct active experts per layer)
+    active = []
+    for r in range(min(n_rot, len(mods)) if w.n_layers == 1 else 1):
+        mods[r].forward(xs[r % len(xs)], outs[0], stream)
+        off = mods[r].debug_routing(N)["offsets"].cpu().numpy()
+        active.append(int((np.diff(off) > 0).sum()))
+    torch.cuda.synchronize()
+
+    for m in mods:
+        m.profile(True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.15)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    local_s = e0.elapsed_time(e1) / 1e3
+    ktimes = {}
+    for m in mods:
+        for name, ms in m.kernel_times().items():
+            ktimes.setdefault(name, []).append(ms)
+        m.profile(False)
+        assert m.status() == 0
+    value, secs = job_throughput(N * args.steps, local_s, world, dev)
+    ms_per_step = secs / args.steps * 1e3
+
+    # end to end through the C ABI with host buffers (H2D + forward + D2H per step)
+    xh = xs[0].cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    e2e_steps = max(10, min(args.steps, 500))
+    for _ in range(3):
+        mods[0].forward_host(xh, oh)
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        if w.n_layers > 1:
+            # first block from host, the chain on device, last block back to host
+            xd = xh.to(dev, non_blocking=True)
+            h = xd
+            for l, m in enumerate(mods):
+                dst = outs[l & 1]
+                m.forward(h, dst, stream)
+                h = dst
+            oh.copy_(h, non_blocking=True)
+            torch.cuda.synchronize()
+        else:
+            mods[0].forward_host(xh, oh)
+    e2e_local = time.perf_counter() - t0
+    e2e_value, _ = job_throughput(N * e2e_steps, e2e_local, world, dev)
+    nbytes = xh.numel() * xh.element_size()
+
+    # roofline of the dominant kernel
+    peaks, src = load_peaks()
+    mean_ms = {k: float(np.mean(v)) for k, v in ktimes.items()}   # per launch
+    per_layer = mean_ms
+    dom = max(mean_ms, key=mean_ms.get)
+    U = float(np.mean(active))
+    n_assign = N * w.top_k
+    bpe = 2 if w.dtype == "bf16" else 4
+    if N * w.top_k / max(U, 1) < 64:  # weight-streaming regime: HBM-bound
+        bound = "hbm"
+        if dom == "gate_up":
+            work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe)
+        elif dom == "down":
+            work = A.down_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe
+        else:
+            work = A.decode_bytes(U, N, w.d, w.d_ff, w.n_experts, bpe, bpe)
+        achieved = work / (mean_ms[dom] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        bound = "tensor"
+        work = (A.gate_up_flops(n_assign, w.d, w.d_ff) if dom == "gate_up"
+                else A.down_flops(n_assign, w.d, w.d_ff))
+        achieved = work / (mean_ms[dom] / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        unit = "TFLOP/s"
+    traffic = traffic_from_profiles(dom, args.workload)
+    launches = mods[0].launches_per_forward(N) * args.steps * (len(mods) if w.n_layers > 1 else 1)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded; random-init weights of the layer's shapes)",
+        "config": {"workload": w.name, "tokens_per_gpu": N, "layers": w.n_layers,
+                   "d": w.d, "experts": w.n_experts, "top_k": w.top_k, "d_ff": w.d_ff,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": (f"weights rotate over {n_rot} copies, >= 1 GB read per step (> 126 MB L2)"
+                          if w.n_layers == 1 else "38 distinct layers, 45.9 GB per step (> L2)"),
+                   "active_experts_per_layer": U},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+                "d2h_bytes_per_step": nbytes},
+        "gpu_launches": launches,
+        "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+                     "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
+                     "work_per_launch": work},
+        "kernel_ms": per_layer,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, xs[0], layers[0], budget_s=args.cpu_budget)
+    for m in mods:
+        m.close()
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def cpu_baseline(w, x, layer, budget_s=15.0, tokens_per_call=None):
+    """The fp64 oracle as it stands, timed on this host's cores over a bounded
+    sample of the workload (whole tokens through the whole layer)."""
+    import oracle
+    cores = oracle.set_threads(0)
+    x_cpu = x.detach().cpu()
+    l_cpu = {k: v.detach().cpu() for k, v in layer.items()}
+    n = tokens_per_call or min(w.n_tokens, max(1, cores))
+    done, t_total, calls = 0, 0.0, 0
+    while t_total < budget_s and calls < 1000:
+        toks = np.arange(done, done + n) % w.n_tokens
+        t0 = time.perf_counter()
+        oracle.forward(x_cpu, l_cpu, w.top_k, w.eps, w.routed_scale, tokens=toks)
+        t_total += time.perf_counter() - t0
+        done += n
+        calls += 1
+    tps = done / t_total / max(w.n_layers, 1)
+    return {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{done} tokens of {w.name} through one full block (fp64, "
+                       f"{calls} calls of {n} tokens, {t_total:.1f} s)"
+                       + ("; per-token cost of one block divided by 38 blocks"
+                          if w.n_layers > 1 else ""))}
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    cores = oracle.set_threads(0)
+    layer = W.make_layer(w, 0, "cpu")
+    x = W.make_x(w, "cpu")
+    # each step: a bounded sample (whole tokens through one block), sized so
+    # that warm-up + steps stay within about a minute
+    probe_t0 = time.perf_counter()
+    oracle.forward(x, layer, w.top_k, w.eps, w.routed_scale, tokens=np.arange(min(cores, w.n_tokens)))
+    t_tok = (time.perf_counter() - probe_t0) / min(cores, w.n_tokens)
+    per_step = max(1, int(60.0 / max(args.steps + args.warmup, 1) / max(t_tok, 1e-9)))
+    per_step = min(per_step, w.n_tokens)
+    done = 0
+    for i in range(args.warmup):
+        oracle.forward(x, layer, w.top_k, w.eps, w.routed_scale,
+                       tokens=(np.arange(per_step) + i * per_step) % w.n_tokens)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.forward(x, layer, w.top_k, w.eps, w.routed_scale,
+                       tokens=(np.arange(per_step) + i * per_step) % w.n_tokens)
+        done += per_step
+    secs = time.perf_counter() - t0
+    value = done / secs / max(w.n_layers, 1)
+    unit = "tokens/s"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "tokens_per_gpu": w.n_tokens, "layers": w.n_layers,
+                   "parallelism": "cpu", "sample_tokens_per_step": per_step},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} tokens per step through one block, fp64"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS[args.workload]
+    w = W.WORKLOADS[args.workload]
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args, w, world, rank)
+    else:
+        line = run_ours(args, w, world, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1 and torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,136 @@
+/*
+ * moe.h -- C ABI of the sigmoid-bias top-k mixture-of-experts feed-forward
+ * block, B200 (sm_100a) implementation.
+ *
+ * The layer is the sparse feed-forward half of a pre-norm block as stated in
+ * "LFM2.5-24B-A2B: Biased Routing, Short Convolutions and Ten KV Caches"
+ * (flozi.net, English page):
+ *   section "The exact checkpoint": out = x + FFN(RMSNorm(x)), shape-preserving;
+ *   section "The router has two different scores": tokens are rows of
+ *     X in R^{N x d}; a router matrix W_r in R^{E x d} gives E logits per token;
+ *     sigmoid is applied to each logit independently; a stored E-element bias
+ *     takes part in the top-k selection but not in the mixture weights, which
+ *     are the selected unbiased scores normalised by their sum plus an epsilon
+ *     and multiplied by the routed scaling factor (1 for that checkpoint); each
+ *     selected expert is a gated SiLU MLP whose gate and up matrices are packed
+ *     together;
+ *   section "What to verify in a deployment": tokens are grouped by expert and
+ *     the weighted expert outputs accumulated.
+ * Per token t:  xn = x_t / sqrt(mean(x_t^2) + eps) * gain
+ *               s_e = sigmoid(W_r[e] . xn),  c_e = s_e + bias_e
+ *               S = top-k of c (slots by descending c, ties to the lower index)
+ *               w_j = routed_scale * s_{S_j} / (sum_j s_{S_j} + eps)
+ *               out_t = x_t + sum_j w_j * Wd_e (silu(Wg_e xn) * (Wu_e xn)), e = S_j
+ *
+ * All pointers passed to these functions are DEVICE pointers unless the name
+ * says host. Every function returns 0 (MOE_OK) or a negative moe_err code.
+ * A context is not thread-safe: one forward at a time per context.
+ */
+#ifndef SIGMOID_BIAS_TOP_MOE_H
+#define SIGMOID_BIAS_TOP_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Storage type of x, out and the expert matrices. The RMSNorm gain, router
+ * matrix and expert bias are always fp32 (the router stays unquantised). */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,       /* null pointer, bad enum, n_tokens < 0        */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2, /* sizes outside the supported ranges below    */
+    MOE_ERR_ALIGNMENT = -3,         /* a pointer is not 16-byte aligned            */
+    MOE_ERR_TOO_MANY_TOKENS = -4,   /* n_tokens > max_tokens given at create       */
+    MOE_ERR_OOM = -5,               /* workspace allocation failed                 */
+    MOE_ERR_CUDA = -6,              /* a CUDA runtime call or launch failed        */
+    MOE_ERR_DEVICE_TIMEOUT = -7,    /* a bounded device-side wait ran out          */
+    MOE_ERR_DEVICE_BOUNDS = -8,     /* a device-side index check failed            */
+    MOE_ERR_NO_DEVICE = -9          /* no CUDA device, or not an sm_100 device     */
+} moe_err;
+
+/* Layer parameters: BORROWED device pointers, row-major, caller-owned; they
+ * must stay valid and unchanged until moe_destroy. 16-byte aligned. */
+typedef struct {
+    int dtype;                 /* moe_dtype of w_gate_up, w_down, x and out           */
+    const float *norm_gain;    /* [d]        RMSNorm gain, multiplied as stored       */
+    const float *router_w;     /* [E][d]     router matrix W_r                        */
+    const float *expert_bias;  /* [E]        selection-only expert bias               */
+    const void  *w_gate_up;    /* [E][2I][d] rows 0..I-1 gate, rows I..2I-1 up        */
+    const void  *w_down;       /* [E][d][I]  down projection                          */
+    float        routed_scale; /* multiplies the normalised weights (1 in the page)   */
+} moe_weights;
+
+typedef struct moe_ctx moe_ctx;
+
+/* Validates the shapes, allocates the workspace for up to max_tokens tokens on
+ * the current CUDA device and builds the TMA descriptors of the weights.
+ * d = hidden width, n_experts = E, d_ff = expert intermediate width I,
+ * top_k = k, eps serves both the RMSNorm and the weight normalisation.
+ * Supported: 1 <= top_k <= min(n_experts, 8), n_experts <= 256,
+ *   MOE_F32: d % 4 == 0, any d_ff >= 1;
+ *   MOE_BF16: d % 64 == 0, d_ff % 64 == 0 (tensor-core tiles).
+ * On success *out receives the context; on failure *out is set to NULL and
+ * nothing stays allocated. Synchronous. */
+int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
+               const moe_weights *w, int max_tokens, moe_ctx **out);
+
+/* out[N][d] = x + MoE(RMSNorm(x)) for x[N][d] (device, dtype of the weights).
+ * out == x (in place) is allowed; other overlap is not. Asynchronous on
+ * `stream` (a cudaStream_t, NULL = legacy default stream): no host sync, no
+ * allocation, a fixed sequence of kernel launches, so it can be captured in a
+ * CUDA graph. n_tokens == 0 is a no-op. Device-side failures are reported by
+ * moe_status. */
+int moe_forward(moe_ctx *h, const void *x, void *out, int n_tokens, void *stream);
+
+/* Same as moe_forward for HOST buffers: copies x_host into device staging,
+ * runs the forward and copies the result back into out_host, then waits for
+ * the stream. Pinned host memory gives asynchronous copies; pageable works. */
+int moe_forward_host(moe_ctx *h, const void *x_host, void *out_host, int n_tokens,
+                     void *stream);
+
+/* Frees the workspace (not the weights). Waits for the device. NULL is a no-op. */
+int moe_destroy(moe_ctx *h);
+
+/* Reads and clears the device status word after waiting for the device:
+ * MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BOUNDS. */
+int moe_status(moe_ctx *h);
+
+/* Device-to-device copy of the last forward's routing into caller buffers
+ * (any may be NULL): idx[N][k] int32 expert per slot, w[N][k] fp32 weights,
+ * perm[N*k] int32 assignment ids t*k+j grouped by expert (ascending expert,
+ * then ascending token), offsets[E+1] int32 exclusive prefix of the per-expert
+ * counts. Asynchronous on stream. */
+int moe_debug_routing(moe_ctx *h, int32_t *idx, float *w, int32_t *perm,
+                      int32_t *offsets, void *stream);
+
+/* Per-kernel timing. moe_profile(h, 1) starts (or restarts) profiling: each
+ * forward then records CUDA events between its launches on its stream (a ring
+ * of 1024 forwards; older entries are folded into running sums as it wraps).
+ * moe_kernel_times waits for the recorded forwards and writes up to n MEAN
+ * durations in milliseconds per kernel (launch order) over every forward since
+ * profiling started, returning the number of kernels per forward, 0 if none
+ * was recorded, or a negative moe_err. moe_profile(h, 0) stops recording. */
+int moe_profile(moe_ctx *h, int enable);
+int moe_kernel_times(moe_ctx *h, float *ms, int n);
+/* Name of kernel i of the forward's launch sequence (static string), or NULL. */
+const char *moe_kernel_name(moe_ctx *h, int i);
+
+/* Number of kernel launches one forward makes for n_tokens tokens. */
+int moe_launches_per_forward(moe_ctx *h, int n_tokens);
+
+/* Test hook of the bounded device waits: launches one kernel that waits on a
+ * barrier that nothing signals, with a limit of timeout_us microseconds, and
+ * records MOE_ERR_DEVICE_TIMEOUT in the status word. The context stays usable. */
+int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream);
+
+/* Static description of a moe_err code. */
+const char *moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SIGMOID_BIAS_TOP_MOE_H */

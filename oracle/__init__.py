@@ -16,7 +16,7 @@ import os
 import numpy as np
 import torch
 
-from .build import build
+from ._build import build
 
 F32, BF16, F64 = 0, 1, 2
 

@@ -1,0 +1,192 @@
+"""B200 (sm_100a) sigmoid-bias top-k mixture-of-experts feed-forward block.
+
+Thin ctypes binding of libmoe.so, the C ABI declared in include/moe.h. It only
+marshals torch tensors (device memory, streams) into the C calls: every step
+of the layer runs in the library's CUDA kernels. There is no CPU path; if the
+library is missing or no sm_100 GPU is present, the calls raise.
+
+Layer (see include/moe.h): out = x + sum_j w_j * Expert_{S_j}(RMSNorm(x)), with
+the top-k set S chosen on sigmoid(router logits) + expert bias and the weights
+w taken from the unbiased sigmoid scores normalised by (their sum + eps).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+ERRORS = {
+    0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
+    -3: "MOE_ERR_ALIGNMENT", -4: "MOE_ERR_TOO_MANY_TOKENS", -5: "MOE_ERR_OOM",
+    -6: "MOE_ERR_CUDA", -7: "MOE_ERR_DEVICE_TIMEOUT", -8: "MOE_ERR_DEVICE_BOUNDS",
+    -9: "MOE_ERR_NO_DEVICE",
+}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {ERRORS.get(code, code)} ({strerror(code)})")
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("norm_gain", ctypes.c_void_p),
+                ("router_w", ctypes.c_void_p), ("expert_bias", ctypes.c_void_p),
+                ("w_gate_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+                ("routed_scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m sigmoid_bias_top_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.moe_create.argtypes = [I, I, I, I, F, ctypes.POINTER(MoeWeights), I,
+                                 ctypes.POINTER(P)]
+        L.moe_forward.argtypes = [P, P, P, I, P]
+        L.moe_forward_host.argtypes = [P, P, P, I, P]
+        L.moe_destroy.argtypes = [P]
+        L.moe_status.argtypes = [P]
+        L.moe_debug_routing.argtypes = [P, P, P, P, P, P]
+        L.moe_profile.argtypes = [P, I]
+        L.moe_kernel_times.argtypes = [P, ctypes.POINTER(F), I]
+        L.moe_kernel_name.argtypes = [P, I]
+        L.moe_kernel_name.restype = ctypes.c_char_p
+        L.moe_launches_per_forward.argtypes = [P, I]
+        L.moe_selftest_timeout.argtypes = [P, I, P]
+        L.moe_strerror.argtypes = [I]
+        L.moe_strerror.restype = ctypes.c_char_p
+        for f in (L.moe_create, L.moe_forward, L.moe_forward_host, L.moe_destroy,
+                  L.moe_status, L.moe_debug_routing, L.moe_profile, L.moe_kernel_times,
+                  L.moe_launches_per_forward, L.moe_selftest_timeout):
+            f.restype = I
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().moe_strerror(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise MoeError(rc, what)
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+class MoeLayer:
+    """One MoE block bound to device weights (borrowed, kept alive here).
+
+    layer: dict with norm_gain [d] f32, router_w [E,d] f32, bias [E] f32,
+    w_gate_up [E,2I,d] and w_down [E,d,I] (both f32 or bf16), on one CUDA device.
+    """
+
+    def __init__(self, layer: Dict, top_k: int, eps: float = 1e-6,
+                 routed_scale: float = 1.0, max_tokens: int = 1024):
+        import torch
+        wgu, wd = layer["w_gate_up"], layer["w_down"]
+        E, twoI, d = wgu.shape
+        I = twoI // 2
+        if wgu.dtype == torch.bfloat16:
+            dt = MOE_BF16
+        elif wgu.dtype == torch.float32:
+            dt = MOE_F32
+        else:
+            raise TypeError(f"expert weights must be f32 or bf16, got {wgu.dtype}")
+        self._keep = {n: layer[n].contiguous() for n in
+                      ("norm_gain", "router_w", "bias", "w_gate_up", "w_down")}
+        for n, t in self._keep.items():
+            if not t.is_cuda:
+                raise ValueError(f"{n} must be a CUDA tensor")
+        self.d, self.E, self.I, self.k = d, E, I, top_k
+        self.dtype = wgu.dtype
+        self.max_tokens = max_tokens
+        k = self._keep
+        self._w = MoeWeights(dt, k["norm_gain"].data_ptr(), k["router_w"].data_ptr(),
+                             k["bias"].data_ptr(), k["w_gate_up"].data_ptr(),
+                             k["w_down"].data_ptr(), routed_scale)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(wgu.device):
+            _check(lib().moe_create(d, E, I, top_k, eps, ctypes.byref(self._w), max_tokens,
+                                    ctypes.byref(h)), "moe_create")
+        self._h = h
+        self.device = wgu.device
+
+    def forward(self, x, out=None, stream=None):
+        import torch
+        n = x.shape[0]
+        if out is None:
+            out = torch.empty_like(x)
+        _check(lib().moe_forward(self._h, x.data_ptr(), out.data_ptr(), n,
+                                 _stream_ptr(stream)), "moe_forward")
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, x_host, out_host, stream=None):
+        """x_host, out_host: CPU tensors (pinned for asynchronous copies)."""
+        _check(lib().moe_forward_host(self._h, x_host.data_ptr(), out_host.data_ptr(),
+                                      x_host.shape[0], _stream_ptr(stream)), "moe_forward_host")
+        return out_host
+
+    def debug_routing(self, n_tokens: int, stream=None):
+        """Routing of the last forward: dict(idx, w, perm, offsets) device tensors."""
+        import torch
+        dev = self.device
+        idx = torch.empty(n_tokens, self.k, dtype=torch.int32, device=dev)
+        w = torch.empty(n_tokens, self.k, dtype=torch.float32, device=dev)
+        perm = torch.empty(n_tokens * self.k, dtype=torch.int32, device=dev)
+        offsets = torch.empty(self.E + 1, dtype=torch.int32, device=dev)
+        _check(lib().moe_debug_routing(self._h, idx.data_ptr(), w.data_ptr(), perm.data_ptr(),
+                                       offsets.data_ptr(), _stream_ptr(stream)),
+               "moe_debug_routing")
+        return {"idx": idx, "w": w, "perm": perm, "offsets": offsets}
+
+    def status(self) -> int:
+        return lib().moe_status(self._h)
+
+    def profile(self, enable: bool = True):
+        _check(lib().moe_profile(self._h, int(enable)), "moe_profile")
+
+    def kernel_times(self) -> Dict[str, float]:
+        ms = (ctypes.c_float * 16)()
+        n = lib().moe_kernel_times(self._h, ms, 16)
+        if n < 0:
+            raise MoeError(n, "moe_kernel_times")
+        return {lib().moe_kernel_name(self._h, i).decode(): ms[i] for i in range(n)}
+
+    def launches_per_forward(self, n_tokens: int) -> int:
+        return lib().moe_launches_per_forward(self._h, n_tokens)
+
+    def selftest_timeout(self, timeout_us: int, stream=None):
+        _check(lib().moe_selftest_timeout(self._h, timeout_us, _stream_ptr(stream)),
+               "moe_selftest_timeout")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            rc = lib().moe_destroy(self._h)
+            self._h = None
+            _check(rc, "moe_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

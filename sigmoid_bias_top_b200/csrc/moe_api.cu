@@ -1,0 +1,402 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument validation,
+// workspace ownership, TMA descriptor set-up and the launch sequence of one
+// forward of the sigmoid-bias top-k MoE block.
+//
+// Launch sequence (all on the caller's stream, no host synchronisation):
+//   1 route            RMSNorm + fp32 router + sigmoid + biased top-k + weights
+//   2 dispatch_scan    per-expert counts, offsets, row-tile prefix, scatter bases
+//   3 dispatch_scatter perm / inv, rows copied into expert-grouped order
+//   4 gate_up          grouped GEMM + SiLU(gate)*up (tcgen05 for bf16, SIMT for fp32)
+//   5 down             grouped GEMM
+//   6 combine          out = x + sum_j w_j y_j in fixed slot order
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "moe_internal.cuh"
+
+using namespace moe;
+
+namespace {
+constexpr int kEvPerFwd = 8;     // event marks per forward (launches + 1, rounded up)
+constexpr int kRingForwards = 1024;
+}
+
+struct moe_ctx {
+    int d, E, I, k, dtype, max_tokens, device, n_sm;
+    float eps, scale;
+    moe_weights w;
+    size_t elem;  // bytes per element of x / experts
+
+    void *ws;  // one allocation, carved below
+    void *xn, *xp, *act, *y, *x_stage, *out_stage;
+    int32_t *idx, *hist, *base, *counts, *offsets, *mt_start, *perm, *inv;
+    float *wts;
+    int *status;
+    int rows_cap;
+
+    TcMaps maps;
+    bool use_tc;
+
+    int last_n;
+
+    // profiling: a ring of event sets, one set (kEvPerFwd events) per forward
+    bool profile;
+    std::vector<cudaEvent_t> ring;
+    long long head, pending_from;  // forwards recorded / first not yet accumulated
+    int n_kernels;
+    double sum_ms[kEvPerFwd];
+    long long n_fwd;
+};
+
+static const char *kKernelNames[6] = {"route", "dispatch_scan", "dispatch_scatter",
+                                      "gate_up", "down", "combine"};
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int toks_per_route_block(int N, int d, int E) {
+    // enough route CTAs to cover the SMs before packing tokens together, and
+    // the per-CTA rows (fp32 xn + scores) within 160 KB of shared memory
+    int tt = N >= 8 * 148 ? 8 : N >= 4 * 148 ? 4 : N >= 2 * 148 ? 2 : 1;
+    while (tt > 1 && static_cast<size_t>(tt) * (d + E) * 4 + E * 4 > 160 * 1024) tt /= 2;
+    return tt;
+}
+
+extern "C" const char *moe_strerror(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case MOE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case MOE_ERR_TOO_MANY_TOKENS: return "n_tokens exceeds max_tokens";
+        case MOE_ERR_OOM: return "device allocation failed";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case MOE_ERR_DEVICE_BOUNDS: return "device-side index out of bounds";
+        case MOE_ERR_NO_DEVICE: return "no sm_100 CUDA device";
+        default: return "unknown error";
+    }
+}
+
+static int check_shapes(int d, int E, int I, int k, int dtype, int max_tokens) {
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (d <= 0 || E <= 0 || I <= 0 || k <= 0 || max_tokens <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (E > kMaxExperts || k > kMaxTopK || k > E) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (d % 4 != 0 || d > 32768) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dtype == MOE_BF16 && (d % 64 != 0 || I % 64 != 0)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    // 32-bit row indices and TMA coordinates
+    if (static_cast<long long>(max_tokens) * k >= (1LL << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(E) * 2 * I >= (1LL << 30) ||
+        static_cast<long long>(E) * d >= (1LL << 30))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
+                          const moe_weights *w, int max_tokens, moe_ctx **out) {
+    if (!out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!w) return MOE_ERR_INVALID_ARG;
+    int rc = check_shapes(d, n_experts, d_ff, top_k, w->dtype, max_tokens);
+    if (rc != MOE_OK) return rc;
+    if (!w->norm_gain || !w->router_w || !w->expert_bias || !w->w_gate_up || !w->w_down)
+        return MOE_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !(w->routed_scale == w->routed_scale)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->norm_gain) || !aligned16(w->router_w) || !aligned16(w->w_gate_up) ||
+        !aligned16(w->w_down))
+        return MOE_ERR_ALIGNMENT;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_NO_DEVICE;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_NO_DEVICE;
+    if (prop.major != 10) return MOE_ERR_NO_DEVICE;
+
+    moe_ctx *h = new (std::nothrow) moe_ctx();
+    if (!h) return MOE_ERR_OOM;
+    h->d = d; h->E = n_experts; h->I = d_ff; h->k = top_k; h->dtype = w->dtype;
+    h->max_tokens = max_tokens; h->device = dev; h->n_sm = prop.multiProcessorCount;
+    h->eps = eps; h->scale = w->routed_scale; h->w = *w;
+    h->elem = (w->dtype == MOE_F32) ? 4 : 2;
+    h->use_tc = (w->dtype == MOE_BF16);
+    h->rows_cap = max_tokens * top_k;
+
+    // workspace layout (every block 256-byte aligned)
+    const size_t N = max_tokens, R = h->rows_cap, E = n_experts;
+    const size_t sizes[] = {
+        N * d * h->elem,            // xn
+        R * d * h->elem,            // xp
+        R * d_ff * h->elem,         // act
+        R * d * h->elem,            // y
+        N * d * h->elem,            // x_stage
+        N * d * h->elem,            // out_stage
+        N * top_k * 4,              // idx
+        N * E * 4,                  // hist (one row per route CTA; at most N CTAs)
+        N * E * 4,                  // base
+        E * 4,                      // counts
+        (E + 1) * 4,                // offsets
+        (E + 1) * 4,                // mt_start
+        R * 4,                      // perm
+        R * 4,                      // inv
+        N * top_k * 4,              // wts
+        256,                        // status
+    };
+    const int nblocks = sizeof(sizes) / sizeof(sizes[0]);
+    size_t total = 0, off[16];
+    for (int i = 0; i < nblocks; ++i) {
+        off[i] = total;
+        total += (sizes[i] + 255) & ~static_cast<size_t>(255);
+    }
+    if (getenv("MOE_TEST_FAIL_ALLOC") != nullptr ||
+        cudaMalloc(&h->ws, total) != cudaSuccess) {
+        cudaGetLastError();
+        delete h;
+        return MOE_ERR_OOM;
+    }
+    uint8_t *b = static_cast<uint8_t *>(h->ws);
+    h->xn = b + off[0]; h->xp = b + off[1]; h->act = b + off[2]; h->y = b + off[3];
+    h->x_stage = b + off[4]; h->out_stage = b + off[5];
+    h->idx = reinterpret_cast<int32_t *>(b + off[6]);
+    h->hist = reinterpret_cast<int32_t *>(b + off[7]);
+    h->base = reinterpret_cast<int32_t *>(b + off[8]);
+    h->counts = reinterpret_cast<int32_t *>(b + off[9]);
+    h->offsets = reinterpret_cast<int32_t *>(b + off[10]);
+    h->mt_start = reinterpret_cast<int32_t *>(b + off[11]);
+    h->perm = reinterpret_cast<int32_t *>(b + off[12]);
+    h->inv = reinterpret_cast<int32_t *>(b + off[13]);
+    h->wts = reinterpret_cast<float *>(b + off[14]);
+    h->status = reinterpret_cast<int *>(b + off[15]);
+    if (cudaMemset(h->ws, 0, total) != cudaSuccess) {
+        cudaFree(h->ws);
+        delete h;
+        return MOE_ERR_CUDA;
+    }
+    if (h->use_tc) {
+        rc = tc_build_maps(&h->maps, h->xp, h->act, w->w_gate_up, w->w_down, h->rows_cap,
+                           n_experts, d, d_ff);
+        if (rc != MOE_OK) {
+            cudaFree(h->ws);
+            delete h;
+            return rc;
+        }
+    }
+    *out = h;
+    return MOE_OK;
+}
+
+// Adds the durations of up to `count` (all if < 0) recorded forwards, oldest
+// first, to the per-kernel sums.
+static int accumulate(moe_ctx *h, long long count) {
+    while (h->pending_from < h->head && count-- != 0) {
+        cudaEvent_t *ev = &h->ring[static_cast<size_t>(h->pending_from % kRingForwards) * kEvPerFwd];
+        if (cudaEventSynchronize(ev[h->n_kernels]) != cudaSuccess) return MOE_ERR_CUDA;
+        for (int i = 0; i < h->n_kernels; ++i) {
+            float ms = 0.f;
+            if (cudaEventElapsedTime(&ms, ev[i], ev[i + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+            h->sum_ms[i] += ms;
+        }
+        h->n_fwd++;
+        h->pending_from++;
+    }
+    return MOE_OK;
+}
+
+static void free_ring(moe_ctx *h) {
+    for (cudaEvent_t e : h->ring) cudaEventDestroy(e);
+    h->ring.clear();
+}
+
+static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_t s) {
+    int rc;
+    const bool prof = h->profile;
+    int ne = 0;
+    cudaEvent_t *ev = nullptr;
+    if (prof) {
+        if (h->head - h->pending_from >= kRingForwards && (rc = accumulate(h, 1)) != MOE_OK)
+            return rc;
+        ev = &h->ring[static_cast<size_t>(h->head % kRingForwards) * kEvPerFwd];
+    }
+#define MOE_MARK()                                                          \
+    do {                                                                    \
+        if (prof && cudaEventRecord(ev[ne++], s) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+#define MOE_TRY(expr)                     \
+    do {                                  \
+        if ((rc = (expr)) != MOE_OK) return rc; \
+    } while (0)
+
+    const int tt = toks_per_route_block(N, h->d, h->E);
+    const int nblk = (N + tt - 1) / tt;
+    const int tile_m = h->use_tc ? kTcTileM : kSimtTileM;
+
+    MOE_MARK();
+    RouteParams rp;
+    rp.x = x; rp.gain = h->w.norm_gain; rp.router_w = h->w.router_w; rp.bias = h->w.expert_bias;
+    rp.xn = h->xn; rp.idx = h->idx; rp.wts = h->wts; rp.hist = h->hist;
+    rp.N = N; rp.d = h->d; rp.E = h->E; rp.k = h->k; rp.eps = h->eps; rp.scale = h->scale;
+    MOE_TRY(launch_route(rp, h->dtype, tt, s));
+    MOE_MARK();
+
+    DispatchParams dp;
+    dp.idx = h->idx; dp.hist = h->hist; dp.base = h->base; dp.counts = h->counts;
+    dp.offsets = h->offsets; dp.mt_start = h->mt_start; dp.perm = h->perm; dp.inv = h->inv;
+    dp.xn = h->xn; dp.xp = h->xp; dp.status = h->status;
+    dp.N = N; dp.d = h->d; dp.E = h->E; dp.k = h->k; dp.nblk = nblk; dp.toks_per_blk = tt;
+    dp.tile_m = tile_m; dp.elem_bytes = static_cast<int>(h->elem);
+    MOE_TRY(launch_dispatch_scan(dp, s));
+    MOE_MARK();
+    MOE_TRY(launch_dispatch_scatter(dp, s));
+    MOE_MARK();
+
+    GroupedParams gp;
+    gp.offsets = h->offsets; gp.mt_start = h->mt_start; gp.status = h->status;
+    gp.E = h->E; gp.d = h->d; gp.I = h->I; gp.rows_cap = h->rows_cap;
+    const int max_mtiles = (N * h->k + tile_m - 1) / tile_m + h->E;
+
+    gp.a = h->xp; gp.w = h->w.w_gate_up; gp.c = h->act;
+    if (h->use_tc)
+        MOE_TRY(launch_gemm_tc_gate_up(h->maps, gp, h->n_sm, s));
+    else
+        MOE_TRY(launch_gemm_simt_gate_up(gp, max_mtiles, s));
+    MOE_MARK();
+
+    gp.a = h->act; gp.w = h->w.w_down; gp.c = h->y;
+    if (h->use_tc)
+        MOE_TRY(launch_gemm_tc_down(h->maps, gp, h->n_sm, s));
+    else
+        MOE_TRY(launch_gemm_simt_down(gp, max_mtiles, s));
+    MOE_MARK();
+
+    CombineParams cp;
+    cp.x = x; cp.y = h->y; cp.wts = h->wts; cp.inv = h->inv; cp.out = out; cp.status = h->status;
+    cp.N = N; cp.d = h->d; cp.k = h->k;
+    MOE_TRY(launch_combine(cp, h->dtype, s));
+    MOE_MARK();
+#undef MOE_MARK
+#undef MOE_TRY
+    if (prof) {
+        h->n_kernels = ne - 1;
+        h->head++;
+    }
+    h->last_n = N;
+    return MOE_OK;
+}
+
+static int check_call(moe_ctx *h, int n_tokens) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (n_tokens < 0) return MOE_ERR_INVALID_ARG;
+    if (n_tokens > h->max_tokens) return MOE_ERR_TOO_MANY_TOKENS;
+    int dev;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+extern "C" int moe_forward(moe_ctx *h, const void *x, void *out, int n_tokens, void *stream) {
+    int rc = check_call(h, n_tokens);
+    if (rc != MOE_OK) return rc;
+    if (n_tokens == 0) return MOE_OK;
+    if (!x || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
+    return forward_impl(h, x, out, n_tokens, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int moe_forward_host(moe_ctx *h, const void *x_host, void *out_host, int n_tokens,
+                                void *stream) {
+    int rc = check_call(h, n_tokens);
+    if (rc != MOE_OK) return rc;
+    if (n_tokens == 0) return MOE_OK;
+    if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = static_cast<size_t>(n_tokens) * h->d * h->elem;
+    if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    rc = forward_impl(h, h->x_stage, h->out_stage, n_tokens, s);
+    if (rc != MOE_OK) return rc;
+    if (cudaMemcpyAsync(out_host, h->out_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_destroy(moe_ctx *h) {
+    if (!h) return MOE_OK;
+    int rc = MOE_OK;
+    if (cudaDeviceSynchronize() != cudaSuccess) rc = MOE_ERR_CUDA;
+    free_ring(h);
+    if (cudaFree(h->ws) != cudaSuccess) rc = MOE_ERR_CUDA;
+    delete h;
+    return rc;
+}
+
+extern "C" int moe_status(moe_ctx *h) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v & kStatusTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+    if (v & kStatusBounds) return MOE_ERR_DEVICE_BOUNDS;
+    return MOE_OK;
+}
+
+extern "C" int moe_debug_routing(moe_ctx *h, int32_t *idx, float *w, int32_t *perm,
+                                 int32_t *offsets, void *stream) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t N = h->last_n, k = h->k;
+    if (idx && N && cudaMemcpyAsync(idx, h->idx, N * k * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (w && N && cudaMemcpyAsync(w, h->wts, N * k * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (perm && N && cudaMemcpyAsync(perm, h->perm, N * k * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (offsets && cudaMemcpyAsync(offsets, h->offsets, (h->E + 1) * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+extern "C" int moe_profile(moe_ctx *h, int enable) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (enable && h->ring.empty()) {
+        h->ring.resize(static_cast<size_t>(kRingForwards) * kEvPerFwd);
+        for (size_t i = 0; i < h->ring.size(); ++i) {
+            if (cudaEventCreate(&h->ring[i]) != cudaSuccess) {
+                h->ring.resize(i);
+                free_ring(h);
+                return MOE_ERR_CUDA;
+            }
+        }
+    }
+    h->profile = enable != 0;
+    h->head = h->pending_from = h->n_fwd = 0;
+    for (int i = 0; i < kEvPerFwd; ++i) h->sum_ms[i] = 0.0;
+    return MOE_OK;
+}
+
+extern "C" int moe_kernel_times(moe_ctx *h, float *ms, int n) {
+    if (!h || (n > 0 && !ms)) return MOE_ERR_INVALID_ARG;
+    int rc = accumulate(h, -1);
+    if (rc != MOE_OK) return rc;
+    if (h->n_fwd == 0) return 0;
+    for (int i = 0; i < h->n_kernels && i < n; ++i)
+        ms[i] = static_cast<float>(h->sum_ms[i] / static_cast<double>(h->n_fwd));
+    return h->n_kernels;
+}
+
+extern "C" const char *moe_kernel_name(moe_ctx *h, int i) {
+    (void)h;
+    if (i < 0 || i >= 6) return nullptr;
+    return kKernelNames[i];
+}
+
+extern "C" int moe_launches_per_forward(moe_ctx *h, int n_tokens) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    return n_tokens > 0 ? 6 : 0;
+}
+
+extern "C" int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream) {
+    if (!h || timeout_us <= 0 || timeout_us > 10000000) return MOE_ERR_INVALID_ARG;
+    return launch_selftest_timeout(h->status, timeout_us, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,296 @@
+// moe_internal.cuh -- shared definitions of the sm_100a MoE kernels: parameter
+// blocks, device status codes, and thin inline-PTX wrappers for mbarriers,
+// TMA bulk-tensor copies and the tcgen05 (5th-generation tensor core / TMEM)
+// instructions. Formats follow the PTX ISA for sm_100a.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 8;
+
+// ---------------------------------------------------------------------------
+// Device status word (one int per context). Kernels OR in flag bits; the host
+// maps them to moe_err codes.
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusBounds = 2;
+
+__device__ __forceinline__ void set_status(int *status, int bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// ---------------------------------------------------------------------------
+// Parameter blocks
+
+struct RouteParams {
+    const void *x;          // [N][d] f32 or bf16
+    const float *gain;      // [d]
+    const float *router_w;  // [E][d]
+    const float *bias;      // [E]
+    void *xn;               // [N][d] normalised rows, dtype of x (expert input)
+    int32_t *idx;           // [N][k]
+    float *wts;             // [N][k]
+    int32_t *hist;          // [gridDim.x][E] per-CTA expert counts
+    int N, d, E, k;
+    float eps, scale;
+};
+
+struct DispatchParams {
+    const int32_t *idx;     // [N][k]
+    const int32_t *hist;    // [nblk][E]
+    int32_t *base;          // [nblk][E] scatter base per (route CTA, expert)
+    int32_t *counts;        // [E]
+    int32_t *offsets;       // [E+1]
+    int32_t *mt_start;      // [E+1] prefix of per-expert row tiles (tile rows = tile_m)
+    int32_t *perm;          // [N*k]
+    int32_t *inv;           // [N*k]
+    const void *xn;         // [N][d]
+    void *xp;               // [N*k][d] rows of xn in grouped order
+    int *status;
+    int N, d, E, k, nblk, toks_per_blk, tile_m, elem_bytes;
+};
+
+struct CombineParams {
+    const void *x;          // [N][d]
+    const void *y;          // [N*k][d] expert outputs in grouped order
+    const float *wts;       // [N][k]
+    const int32_t *inv;     // [N*k]
+    void *out;              // [N][d]
+    int *status;
+    int N, d, k;
+};
+
+struct GroupedParams {
+    // shared by the SIMT and the tensor-core grouped GEMMs
+    const int32_t *offsets;   // [E+1] row range of each expert in xp / act / y
+    const int32_t *mt_start;  // [E+1] prefix of per-expert row tiles
+    const void *a;            // gate/up: xp [rows][d]; down: act [rows][I]
+    const void *w;            // gate/up: [E][2I][d]; down: [E][d][I]
+    void *c;                  // gate/up: act [rows][I]; down: y [rows][d]
+    int *status;
+    int E, d, I;
+    int rows_cap;             // allocated rows of a and c
+};
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (one per translation unit)
+
+int launch_route(const RouteParams &p, int dtype, int toks_per_blk, cudaStream_t s);
+int launch_dispatch_scan(const DispatchParams &p, cudaStream_t s);
+int launch_dispatch_scatter(const DispatchParams &p, cudaStream_t s);
+int launch_combine(const CombineParams &p, int dtype, cudaStream_t s);
+int launch_gemm_simt_gate_up(const GroupedParams &p, int max_mtiles, cudaStream_t s);
+int launch_gemm_simt_down(const GroupedParams &p, int max_mtiles, cudaStream_t s);
+constexpr int kSimtTileM = 64;
+constexpr int kTcTileM = 128;
+
+struct TcMaps {
+    CUtensorMap a_gate_up;  // xp  [rows][d],     box 64 x 128
+    CUtensorMap w_gate_up;  // W   [E*2I][d],     box 64 x 128
+    CUtensorMap a_down;     // act [rows][I],     box 64 x 128
+    CUtensorMap w_down;     // Wd  [E*d][I],      box 64 x 256
+};
+int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu,
+                  const void *wd, int rows_cap, int E, int d, int I);
+int launch_gemm_tc_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
+int launch_gemm_tc_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
+int launch_selftest_timeout(int *status, int timeout_us, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Small device helpers
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t u) {
+    return __uint_as_float(static_cast<uint32_t>(u) << 16);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase of `bar` with the given parity to complete, giving up at
+// `deadline` (globaltimer ns). Returns false on time-out.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline) {
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && globaltimer_ns() > deadline) return false;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA (bulk tensor copies global -> shared, completion on an mbarrier)
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, int x, int y,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Same with an L2 eviction-priority hint (a createpolicy value).
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *m, int x, int y,
+                                                 uint64_t *bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05: TMEM allocation, MMA, commit, TMEM -> register loads
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile stored with the
+// 128-byte swizzle (rows of 128 B, 8-row atoms of 1024 B): start address,
+// leading-byte offset 16 B (unused for this layout), stride-byte offset 1024 B
+// between 8-row groups, descriptor version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(1) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
+// fp32 accumulator, for an M x N tile.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4)                                   // D format: f32
+           | (1u << 7)                                 // A format: bf16
+           | (1u << 10)                                // B format: bf16
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives (once) on `bar` when all previously issued tcgen05.mma of this
+// thread have completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives TMEM
+// lane (lane base + i), columns [col, col + 32).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+}  // namespace moe

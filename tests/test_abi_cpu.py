@@ -1,0 +1,79 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, and exports every
+entry point include/moe.h declares. Host-side validation is checked where it
+runs before any device call."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import sigmoid_bias_top_b200 as sb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert "moe_create" in names and "moe_forward" in names and "moe_destroy" in names
+    L = sb.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_library_is_sm100a_build():
+    data = open(sb.LIB_PATH, "rb").read()
+    assert b"sm_100a" in data or b"compute_100a" in data
+
+
+def test_strerror_covers_codes():
+    for code, name in sb.ERRORS.items():
+        msg = sb.strerror(code)
+        assert msg and msg != "unknown error", (code, name)
+    assert sb.strerror(12345) == "unknown error"
+
+
+def _weights(dtype=sb.MOE_BF16, ptr=256):
+    return sb.MoeWeights(dtype, ptr, ptr, ptr, ptr, ptr, 1.0)
+
+
+def _create(d, E, I, k, w, max_tokens=16):
+    h = ctypes.c_void_p(1234)
+    rc = sb.lib().moe_create(d, E, I, k, 1e-6, ctypes.byref(w) if w is not None else None,
+                             max_tokens, ctypes.byref(h))
+    return rc, h
+
+
+def test_create_validates_before_touching_the_device():
+    w = _weights()
+    assert _create(2048, 64, 1536, 4, None)[0] == -1            # no weights
+    rc, h = _create(2048, 64, 1536, 9, w)
+    assert rc == -2 and not h.value                              # k > 8, handle cleared
+    assert _create(2048, 4, 1536, 5, w)[0] == -2                 # k > E
+    assert _create(2048, 300, 1536, 4, w)[0] == -2               # E > 256
+    assert _create(2000, 64, 1536, 4, w)[0] == -2                # bf16 d % 64
+    assert _create(2048, 64, 1500, 4, w)[0] == -2                # bf16 I % 64
+    assert _create(2048, 64, 1536, 4, w, max_tokens=0)[0] == -2
+    assert _create(2048, 64, 1536, 4, _weights(dtype=7))[0] == -1
+    assert _create(2048, 64, 1536, 4, _weights(ptr=258))[0] == -3  # misaligned
+    assert _create(2048, 64, 1536, 4, _weights(ptr=0))[0] == -1    # null
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
+def test_create_without_gpu_reports_no_device():
+    rc, h = _create(256, 16, 192, 4, _weights(dtype=sb.MOE_F32))
+    assert rc == -9 and not h.value
+
+
+def test_calls_on_null_handle_are_rejected():
+    L = sb.lib()
+    assert L.moe_forward(None, None, None, 1, None) == -1
+    assert L.moe_status(None) == -1
+    assert L.moe_destroy(None) == 0
+    assert L.moe_profile(None, 1) == -1

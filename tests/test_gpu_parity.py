@@ -1,0 +1,202 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on the five
+workloads and on edge cases. Needs an sm_100 GPU."""
+import numpy as np
+import pytest
+import torch
+
+from sigmoid_bias_top_b200 import MoeError, MoeLayer, workloads as W
+from tests import parity as PA
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def run(w, x=None, layer=None, max_tokens=None, layer_idx=0):
+    if layer is None:
+        layer = W.make_layer(w, layer_idx, DEV)
+    if x is None:
+        x = W.make_x(w, DEV)
+    N = x.shape[0]
+    m = MoeLayer(layer, w.top_k, w.eps, w.routed_scale, max_tokens=max_tokens or max(N, 1))
+    out = m(x)
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    r = m.debug_routing(N)
+    torch.cuda.synchronize()
+    return m, x, layer, out, r
+
+
+def full_check(w, x, layer, out, r, tokens=None):
+    x_cpu, l_cpu = x.cpu(), PA.to_cpu_layer(layer)
+    ref, idx, n_near = PA.check_routing(x_cpu, l_cpu, w.top_k, w.eps, w.routed_scale, r)
+    d = PA.check_dispatch(idx, w.n_experts, r)
+    if tokens is None:
+        tokens = np.arange(x.shape[0])
+    elif isinstance(tokens, str):
+        tokens = PA.sample_tokens(x.shape[0], idx, d["offsets"], n_random=128)
+    err, derr = PA.check_outputs(x_cpu, l_cpu, w.top_k, w.eps, w.routed_scale, out, idx,
+                                 tokens, w.dtype)
+    return {"err": err, "delta_err": derr, "near_ties": n_near, "counts": d["counts"]}
+
+
+def test_tiny_f32_full():
+    w = W.TINY_F32
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r)
+
+
+def test_decode_full():
+    w = W.DECODE
+    m, x, layer, out, r = run(w)
+    res = full_check(w, x, layer, out, r)
+    assert (res["counts"] > 0).sum() >= 45
+
+
+def test_prefill_sampled():
+    w = W.PREFILL
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r, tokens="sample")
+
+
+def test_skewed_sampled():
+    w = W.SKEWED
+    m, x, layer, out, r = run(w)
+    res = full_check(w, x, layer, out, r, tokens="sample")
+    c = np.sort(res["counts"])[::-1]
+    assert 0.4 <= c[:8].sum() / c.sum() <= 0.6
+    assert (res["counts"] < 16).sum() >= 4
+
+
+def test_stacked_decode_every_block_routing():
+    """38 chained blocks h = x + MoE(RMSNorm(x)); every block's routing checked
+    against the oracle on that block's GPU input (teacher forcing), outputs of
+    blocks 1, 19 and 38 checked on sampled tokens."""
+    w = W.STACKED
+    x = W.make_x(w, DEV)
+    out_blocks = {0, 18, 37}
+    for l in range(w.n_layers):
+        layer = W.make_layer(w, l, DEV)
+        m = MoeLayer(layer, w.top_k, w.eps, w.routed_scale, max_tokens=w.n_tokens)
+        y = m(x)
+        torch.cuda.synchronize()
+        assert m.status() == 0
+        r = m.debug_routing(w.n_tokens)
+        x_cpu = x.cpu()
+        l_cpu = {k: v.cpu() for k, v in layer.items() if k in ("norm_gain", "router_w", "bias")}
+        ref, idx, _ = PA.check_routing(x_cpu, l_cpu, w.top_k, w.eps, w.routed_scale, r)
+        PA.check_dispatch(idx, w.n_experts, r)
+        if l in out_blocks:
+            toks = np.random.default_rng(l).choice(w.n_tokens, 24, replace=False)
+            PA.check_outputs(x_cpu, PA.to_cpu_layer(layer), w.top_k, w.eps, w.routed_scale,
+                             y, idx, toks, w.dtype)
+        m.close()
+        del layer
+        x = y
+
+
+SMALL_BF16 = W.Workload(name="small_bf16", n_tokens=300, d=320, n_experts=16, top_k=4,
+                        d_ff=320, dtype="bf16", seed=11, gain_jitter=0.02, router_std=0.06,
+                        bias_kind="uniform", bias_halfwidth=0.05, gate_up_std=0.05,
+                        down_std=0.05)
+
+
+def test_ragged_bf16_tiles():
+    """d and I not multiples of the 256/128 tile widths; N not a tile multiple."""
+    m, x, layer, out, r = run(SMALL_BF16)
+    full_check(SMALL_BF16, x, layer, out, r)
+
+
+def test_all_experts_selected():
+    w = SMALL_BF16.scaled(n_experts=4, top_k=4, d=128, d_ff=128, n_tokens=50)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r)
+
+
+def test_one_expert_takes_every_token():
+    """k = 1 with a dominant bias: one expert gets 1000 rows (8 row tiles), the
+    other experts stay empty."""
+    w = SMALL_BF16.scaled(n_experts=8, top_k=1, d=256, d_ff=256, n_tokens=1000)
+    layer = W.make_layer(w, 0, DEV)
+    layer["bias"] = torch.zeros_like(layer["bias"])
+    layer["bias"][3] = 5.0
+    m, x, layer, out, r = run(w, layer=layer)
+    res = full_check(w, x, layer, out, r)
+    assert res["counts"][3] == 1000 and res["counts"].sum() == 1000
+
+
+@pytest.mark.parametrize("n", [1, 7, 129])
+def test_small_batches_decode_shapes(n):
+    w = W.DECODE.scaled(n_tokens=n)
+    m, x, layer, out, r = run(w, max_tokens=256)
+    full_check(w, x, layer, out, r)
+
+
+def test_fp32_ragged():
+    w = W.TINY_F32.scaled(n_tokens=77, d=100, d_ff=70, n_experts=12, top_k=3)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r)
+
+
+def test_deterministic_in_place_and_host_path():
+    w = W.DECODE.scaled(n_tokens=64)
+    layer = W.make_layer(w, 0, DEV)
+    x = W.make_x(w, DEV)
+    m = MoeLayer(layer, w.top_k, w.eps, max_tokens=64)
+    a = m(x)
+    b = m(x)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    xi = x.clone()
+    m(xi, out=xi)
+    torch.cuda.synchronize()
+    assert torch.equal(xi, a)
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    m.forward_host(xh, oh)
+    assert torch.equal(oh, a.cpu())
+    assert m.status() == 0
+
+
+def test_zero_tokens_and_limits():
+    w = W.DECODE.scaled(n_tokens=16)
+    layer = W.make_layer(w, 0, DEV)
+    m = MoeLayer(layer, w.top_k, w.eps, max_tokens=16)
+    x = W.make_x(w, DEV)
+    empty = x[:0]
+    m(empty, out=torch.empty_like(empty))
+    big = W.make_x(w, DEV, n_tokens=17)
+    with pytest.raises(MoeError) as ei:
+        m(big)
+    assert ei.value.code == -4
+    raw = torch.empty(16 * 2048 * 2 + 8, dtype=torch.uint8, device=DEV)
+    mis = raw[2:2 + 16 * 2048 * 2].view(torch.bfloat16).view(16, 2048)
+    with pytest.raises(MoeError) as ei:
+        m(mis)
+    assert ei.value.code == -3
+    torch.cuda.synchronize()
+    assert m.status() == 0
+
+
+def test_bounded_wait_reports_timeout():
+    w = W.TINY_F32
+    layer = W.make_layer(w, 0, DEV)
+    m = MoeLayer(layer, w.top_k, w.eps, max_tokens=64)
+    m.selftest_timeout(2000)
+    assert m.status() == -7
+    assert m.status() == 0
+    out = m(W.make_x(w, DEV))
+    torch.cuda.synchronize()
+    assert m.status() == 0 and torch.isfinite(out).all()
+
+
+def test_bad_shapes_rejected():
+    layer = W.make_layer(SMALL_BF16, 0, DEV)
+    bad = dict(layer)
+    bad["w_gate_up"] = layer["w_gate_up"][:, :, :200].contiguous()   # d = 200, not % 64
+    with pytest.raises(MoeError) as ei:
+        MoeLayer(bad, 4, 1e-6)
+    assert ei.value.code == -2
+    with pytest.raises(MoeError) as ei:
+        MoeLayer(layer, 17, 1e-6)                                    # k > E
+    assert ei.value.code == -2
