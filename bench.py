@@ -173,7 +173,7 @@ def run_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
     N = w.n_tokens
-    layers = make_layers(w, dev, ROTATE)
+    layers = make_layers(w, dev, args.rotate)
     mods = [MoeLayer(l, w.top_k, w.eps, w.routed_scale, max_tokens=N) for l in layers]
     n_rot = len(mods) if w.n_layers == 1 else 1
     xs = [W.make_x(w, dev, seed=w.seed + 17 * rank + i) for i in range(max(n_rot, 2))]
@@ -385,6 +385,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--rotate", type=int, default=ROTATE,
+                    help="distinct weight copies cycled through (single-layer workloads)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

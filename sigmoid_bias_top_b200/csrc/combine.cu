@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     constexpr int V = P::V;
     const int t = blockIdx.x;
     const int k = p.k;
+    if (t == 0)  // the dispatch has consumed the chunk histogram: clear it for the next forward
+        for (int i = threadIdx.x; i < p.chunk_hist_n; i += kThreads) p.chunk_hist[i] = 0;
     const int nvec = p.d / V;
     int rows[kMaxTopK];
     float w[kMaxTopK];

@@ -1,6 +1,7 @@
-// dispatch.cu -- grouping of the N*k token-expert assignments by expert:
-// a deterministic counting sort ordered by (expert, token), with no atomics on
-// the order-defining path.
+// dispatch.cu -- grouping of the N*k token-expert assignments by expert: a
+// deterministic counting sort ordered by (expert, token), with no atomics on
+// the order-defining path, plus the copy of each assignment's normalised row
+// into its grouped position.
 //
 // The page ("LFM2.5-24B-A2B: Biased Routing, Short Convolutions and Ten KV
 // Caches", flozi.net, English page, section "What to verify in a deployment")
@@ -8,127 +9,226 @@
 // router has two different scores" notes that a batch can activate many or all
 // experts with uneven loads, so dispatch and regrouping matter.
 //
-// The route kernel already wrote one expert histogram per route CTA (a block
-// of consecutive tokens). Here:
-//   scan:    column prefix sums over the route CTAs give, for every (CTA,
-//            expert), the first row that CTA's tokens take in the expert's
-//            group; the per-expert counts and their exclusive prefix
-//            (offsets) follow, plus the prefix of per-expert row tiles that
-//            the grouped GEMMs schedule their work by.
-//   scatter: each CTA ranks its own assignments among equal experts in
-//            (token, slot) order, writes perm / inv, and copies the
-//            normalised rows into grouped order (xp).
+// Tokens are split into chunks of chunk_tokens consecutive tokens; the route
+// kernels have already added each chunk's per-expert counts to chunk_hist.
+// `replicas` CTAs per chunk then each
+//   1. read the whole (chunks x E) histogram and form the per-expert totals,
+//      their exclusive prefix over experts (offsets) and the prefix over the
+//      chunks before their own (CTA 0 also publishes offsets, counts and the
+//      prefix of per-expert row tiles that the grouped GEMMs schedule by);
+//   2. rank the chunk's assignments among equal experts in (token, slot)
+//      order: each warp takes a contiguous slice, counts it per expert in
+//      rounds of 32 (__match_any_sync), the warps' counts are prefixed, and a
+//      second pass assigns positions;
+//   3. replica 0 writes perm (grouped row -> assignment t*k+j) and inv (the
+//      reverse); replica r writes the normalised rows of every replicas-th
+//      assignment, one warp per row: xp[row] = x[t] * rinv[t] * gain, the same
+//      fp32 products as the router's input, rounded once to the storage type.
+// The grouped rows let the gate/up GEMM load contiguous 128-row TMA boxes.
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kScanThreads = 1024;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 
-__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(DispatchParams p) {
-    __shared__ int seg_sum[kScanThreads];
-    __shared__ int cnt[kMaxExperts];
-    const int E = p.E, nblk = p.nblk;
-    int G = 1;  // threads per expert: largest power of two with G * E <= 1024
-    while (G * 2 * E <= kScanThreads) G *= 2;
-    const int tid = threadIdx.x;
-    const int e = tid / G, g = tid % G;
-    const int L = (nblk + G - 1) / G;
-    const int b0 = g * L, b1 = min(nblk, b0 + L);
-    const bool active = e < E;
-
-    int local = 0;
-    if (active)
-        for (int b = b0; b < b1; ++b) local += p.hist[static_cast<size_t>(b) * E + e];
-    seg_sum[tid] = local;
+// Exclusive prefix sum of v over threads 0..n-1 (n <= kThreads); every thread
+// of the block must call it. Returns the prefix; *total gets the sum.
+__device__ __forceinline__ int block_exclusive_scan(int v, int n, int *warp_sums, int *total) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int x = tid < n ? v : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
-    // exclusive prefix of the G segments of expert e, and the expert's total
-    int before = 0, total = 0;
-    if (active) {
-        for (int q = 0; q < G; ++q) {
-            const int v = seg_sum[e * G + q];
-            if (q < g) before += v;
-            total += v;
+    if (warp == 0) {
+        int w = lane < kWarps ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < kWarps; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
         }
-        if (g == 0) cnt[e] = total;
+        if (lane < kWarps) warp_sums[lane] = w;  // inclusive
     }
     __syncthreads();
-    if (tid == 0) {
-        int off = 0, mt = 0;
-        for (int x = 0; x < E; ++x) {
-            p.offsets[x] = off;
-            p.mt_start[x] = mt;
-            p.counts[x] = cnt[x];
-            off += cnt[x];
-            mt += (cnt[x] + p.tile_m - 1) / p.tile_m;
-        }
-        p.offsets[E] = off;
-        p.mt_start[E] = mt;
-    }
-    __syncthreads();
-    if (active) {
-        int run = p.offsets[e] + before;
-        for (int b = b0; b < b1; ++b) {
-            const size_t i = static_cast<size_t>(b) * E + e;
-            p.base[i] = run;
-            run += p.hist[i];
-        }
-    }
+    const int before = warp > 0 ? warp_sums[warp - 1] : 0;
+    *total = warp_sums[kWarps - 1];
+    const int incl = x + before;
+    __syncthreads();  // warp_sums may be reused by the next call
+    return incl - (tid < n ? v : 0);
 }
 
-constexpr int kScatterThreads = 256;
+__global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
+    extern __shared__ int4 smem_v[];
+    const int E = p.E, nchunk = p.nchunk, k = p.k, d = p.d;
+    float *gs = reinterpret_cast<float *>(smem_v);      // [d] RMSNorm gain
+    int *hist = reinterpret_cast<int *>(gs + d);        // [nchunk][E]
+    int *base = hist + nchunk * E;                      // [E] this chunk's first row per expert
+    int *wcnt = base + E;                               // [kWarps][E]
+    int *pos_s = wcnt + kWarps * E;                     // [chunk_tokens * k]
+    __shared__ int warp_sums[kWarps];
+    const int c = blockIdx.x / p.replicas, rep = blockIdx.x % p.replicas;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-__global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(DispatchParams p) {
-    __shared__ int pos_s[kMaxTopK * 8];
-    const int b = blockIdx.x;
-    const int t0 = b * p.toks_per_blk;
-    const int ntok = min(p.toks_per_blk, p.N - t0);
-    const int k = p.k, E = p.E;
-    const int na = ntok * k;
-    const int total = p.N * k;
-    const int32_t *idx = p.idx + static_cast<size_t>(t0) * k;
-    if (threadIdx.x < na) {
-        const int a = threadIdx.x;
-        const int e = idx[a];
-        int pos = -1;
-        if (e >= 0 && e < E) {
-            int rank = 0;
-            for (int q = 0; q < a; ++q) rank += (idx[q] == e);
-            pos = p.base[static_cast<size_t>(b) * E + e] + rank;
-            if (pos < 0 || pos >= total) pos = -1;
+    for (int i = tid; i < d / 4; i += kThreads)
+        reinterpret_cast<float4 *>(gs)[i] = __ldg(reinterpret_cast<const float4 *>(p.gain) + i);
+    for (int i = tid; i < nchunk * E; i += kThreads) hist[i] = p.chunk_hist[i];
+    for (int i = tid; i < kWarps * E; i += kThreads) wcnt[i] = 0;
+    __syncthreads();
+
+    // 1. per-expert totals, chunk prefix, expert prefix (E <= kThreads)
+    int before = 0, all = 0;
+    if (tid < E) {
+        for (int q = 0; q < nchunk; ++q) {
+            const int v = hist[q * E + tid];
+            before += q < c ? v : 0;
+            all += v;
         }
-        if (pos < 0) {
-            set_status(p.status, kStatusBounds);
-        } else {
-            p.perm[pos] = t0 * k + a;
-            p.inv[t0 * k + a] = pos;
+    }
+    int total_rows = 0, total_tiles = 0;
+    const int off = block_exclusive_scan(all, E, warp_sums, &total_rows);
+    const int tiles = (all + p.tile_m - 1) / p.tile_m;
+    const int mt = block_exclusive_scan(tiles, E, warp_sums, &total_tiles);
+    if (tid < E) {
+        base[tid] = off + before;
+        if (blockIdx.x == 0) {
+            p.offsets[tid] = off;
+            p.counts[tid] = all;
+            p.mt_start[tid] = mt;
         }
-        pos_s[a] = pos;
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        p.offsets[E] = total_rows;
+        p.mt_start[E] = total_tiles;
     }
     __syncthreads();
-    if (p.xp == nullptr) return;
-    const int nvec = p.d * p.elem_bytes / 16;
-    const uint4 *src = static_cast<const uint4 *>(p.xn);
-    uint4 *dst = static_cast<uint4 *>(p.xp);
-    for (int i = threadIdx.x; i < na * nvec; i += kScatterThreads) {
-        const int a = i / nvec, v = i - a * nvec;
-        const int pos = pos_s[a];
-        if (pos >= 0)
-            dst[static_cast<size_t>(pos) * nvec + v] =
-                src[static_cast<size_t>(t0 + a / k) * nvec + v];
+
+    // 2. this chunk's assignments a = t*k + j, t in [t0, t1)
+    const int t0 = c * p.chunk_tokens;
+    const int t1 = min(p.N, t0 + p.chunk_tokens);
+    const int a0 = t0 * k, na = max(0, (t1 - t0) * k);
+    const int per_warp = (na + kWarps - 1) / kWarps;
+    const int wa0 = a0 + warp * per_warp, wa1 = min(a0 + na, wa0 + per_warp);
+
+    // pass 1: per-warp expert counts
+    for (int r = wa0; r < wa1; r += 32) {
+        const int a = r + lane;
+        const bool act = a < wa1;
+        const unsigned live = __ballot_sync(0xffffffffu, act);
+        const int e = act ? p.idx[a] : -1;
+        const bool ok = act && e >= 0 && e < E;
+        const unsigned same = __match_any_sync(0xffffffffu, ok ? e : -1);
+        if (ok && (same & live & ((1u << lane) - 1u)) == 0)  // first lane of its group
+            wcnt[warp * E + e] += __popc(same & live);
+        if (act && !ok) set_status(p.status, kStatusBounds);
+    }
+    __syncthreads();
+    if (tid < E) {  // exclusive prefix over warps, from the chunk's base
+        int run = base[tid];
+        for (int w = 0; w < kWarps; ++w) {
+            const int v = wcnt[w * E + tid];
+            wcnt[w * E + tid] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    // pass 2: positions
+    const int total = p.N * k;
+    for (int r = wa0; r < wa1; r += 32) {
+        const int a = r + lane;
+        const bool act = a < wa1;
+        const unsigned live = __ballot_sync(0xffffffffu, act);
+        const int e = act ? p.idx[a] : -1;
+        const bool ok = act && e >= 0 && e < E;
+        const unsigned same = __match_any_sync(0xffffffffu, ok ? e : -1) & live;
+        int pos = -1;
+        if (ok) pos = wcnt[warp * E + e] + __popc(same & ((1u << lane) - 1u));
+        __syncwarp();
+        if (ok && (same & ((1u << lane) - 1u)) == 0) wcnt[warp * E + e] += __popc(same);
+        __syncwarp();
+        if (ok && (pos < 0 || pos >= total)) {
+            set_status(p.status, kStatusBounds);
+            pos = -1;
+        }
+        if (act) pos_s[a - a0] = ok ? pos : -1;
+        if (ok && pos >= 0 && rep == 0) {
+            p.perm[pos] = a;
+            p.inv[a] = pos;
+        }
+    }
+    __syncthreads();
+
+    // 3. normalised rows, one warp per row, 16-byte vectors, 8 loads in flight
+    const int vpr = d * p.elem_bytes / 16;  // vectors per row
+    const int epv = 16 / p.elem_bytes;      // elements per vector
+    const uint4 *xv = static_cast<const uint4 *>(p.x);
+    uint4 *xpv = static_cast<uint4 *>(p.xp);
+    constexpr int U = 8;
+    for (int i = rep + warp * p.replicas; i < na; i += kWarps * p.replicas) {
+        const int pos = pos_s[i];
+        if (pos < 0) continue;
+        const int t = (a0 + i) / k;
+        const float r = p.rinv[t];
+        const uint4 *src = xv + static_cast<size_t>(t) * vpr;
+        uint4 *dst = xpv + static_cast<size_t>(pos) * vpr;
+        for (int v0 = 0; v0 < vpr; v0 += 32 * U) {
+            uint4 raw[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < vpr) raw[u] = src[v];
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v >= vpr) continue;
+                const float *g = gs + v * epv;
+                uint4 o;
+                if (p.elem_bytes == 2) {
+                    const float4 g0 = *reinterpret_cast<const float4 *>(g);
+                    const float4 g1 = *reinterpret_cast<const float4 *>(g + 4);
+                    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+                    uint32_t q[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                            bf16_to_f32(w[h] & 0xFFFFu) * r * gg[2 * h],
+                            bf16_to_f32(w[h] >> 16) * r * gg[2 * h + 1]);
+                        q[h] = *reinterpret_cast<uint32_t *>(&b2);
+                    }
+                    o = make_uint4(q[0], q[1], q[2], q[3]);
+                } else {
+                    const float4 g0 = *reinterpret_cast<const float4 *>(g);
+                    o = make_uint4(__float_as_uint(__uint_as_float(raw[u].x) * r * g0.x),
+                                   __float_as_uint(__uint_as_float(raw[u].y) * r * g0.y),
+                                   __float_as_uint(__uint_as_float(raw[u].z) * r * g0.z),
+                                   __float_as_uint(__uint_as_float(raw[u].w) * r * g0.w));
+                }
+                dst[v] = o;
+            }
+        }
     }
 }
 
 }  // namespace
 
-int launch_dispatch_scan(const DispatchParams &p, cudaStream_t s) {
-    dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+size_t dispatch_smem(int nchunk, int E, int chunk_assign, int d) {
+    return (static_cast<size_t>(d) + static_cast<size_t>(nchunk) * E + E +
+            static_cast<size_t>(kWarps) * E + static_cast<size_t>(chunk_assign)) * 4;
 }
 
-int launch_dispatch_scatter(const DispatchParams &p, cudaStream_t s) {
-    if (p.toks_per_blk * p.k > kMaxTopK * 8) return MOE_ERR_INVALID_ARG;
-    dispatch_scatter_kernel<<<p.nblk, kScatterThreads, 0, s>>>(p);
+int launch_dispatch(const DispatchParams &p, cudaStream_t s) {
+    const size_t smem = dispatch_smem(p.nchunk, p.E, p.chunk_tokens * p.k, p.d);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    dispatch_kernel<<<p.nchunk * p.replicas, kThreads, smem, s>>>(p);
     return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -5,7 +5,8 @@
 // and Ten KV Caches" (flozi.net, English page, section "The router has two
 // different scores") runs as two grouped contractions over the expert-grouped
 // rows (section "What to verify in a deployment": tokens grouped by expert):
-//   gate/up: act[r][f] = silu(xp[r] . Wg_e[f]) * (xp[r] . Wu_e[f])
+//   gate/up: act[r][f] = silu(xp[r] . Wg_e[f]) * (xp[r] . Wu_e[f]), xp[r] the
+//            normalised row of the token that grouped row r belongs to
 //            The packed [2I][d] matrix of expert e gives one 256-wide B tile
 //            per 128 output features: 128 gate rows then the 128 matching up
 //            rows, loaded as two TMA boxes into one operand. The accumulator
@@ -160,17 +161,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int total = mts[E] * NT;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- TMA producer ----------------
-            int s = 0;
-            uint32_t ph = 0;
-            uint32_t issued_parity[STAGES];
-            bool issued[STAGES];
-            for (int i = 0; i < STAGES; ++i) issued[i] = false;
-            for (int item = blockIdx.x; item < total && !aborted(ctl); item += gridDim.x) {
-                const Item it = decode(item, NT, mts, offs, E);
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) break;
+        // ---------------- TMA producer (whole warp) ----------------
+        // lane 0 issues; A by one box, B by one box (down) or two (gate/up)
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t issued_parity[STAGES];
+        bool issued[STAGES];
+        for (int i = 0; i < STAGES; ++i) issued[i] = false;
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            if (__shfl_sync(0xffffffffu, aborted(ctl) ? 1 : 0, 0)) break;
+            const Item it = decode(item, NT, mts, offs, E);
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb) {
+                int got = 1;
+                if (lane == 0) got = wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+                if (lane == 0) {
                     uint8_t *sa = smem + s * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
                     mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
@@ -182,16 +188,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         tma_load_2d(sb, &tmB, kb * BK, it.e * p.d + it.nt * BN, &ctl->full[s]);
                     }
-                    issued[s] = true;
-                    issued_parity[s] = ph;
-                    if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
+                issued[s] = true;
+                issued_parity[s] = ph;
+                if (++s == STAGES) { s = 0; ph ^= 1u; }
             }
-            if (aborted(ctl)) {  // let our own copies land before the CTA exits
-                const uint64_t dl = globaltimer_ns() + kWaitNs;
-                for (int i = 0; i < STAGES; ++i)
-                    if (issued[i]) mbar_wait(&ctl->full[i], issued_parity[i], dl);
-            }
+            if (!ok) break;
+        }
+        if (lane == 0 && aborted(ctl)) {  // let our own copies land before the CTA exits
+            const uint64_t dl = globaltimer_ns() + kWaitNs;
+            for (int i = 0; i < STAGES; ++i)
+                if (issued[i]) mbar_wait(&ctl->full[i], issued_parity[i], dl);
         }
     } else if (warp == 1) {
         if (lane == 0) {

@@ -3,12 +3,13 @@
 // forward of the sigmoid-bias top-k MoE block.
 //
 // Launch sequence (all on the caller's stream, no host synchronisation):
-//   1 route            RMSNorm + fp32 router + sigmoid + biased top-k + weights
-//   2 dispatch_scan    per-expert counts, offsets, row-tile prefix, scatter bases
-//   3 dispatch_scatter perm / inv, rows copied into expert-grouped order
-//   4 gate_up          grouped GEMM + SiLU(gate)*up (tcgen05 for bf16, SIMT for fp32)
-//   5 down             grouped GEMM
-//   6 combine          out = x + sum_j w_j y_j in fixed slot order
+//   1 route     RMSNorm + fp32 router + sigmoid + biased top-k + weights, and the
+//               per-chunk expert histogram
+//   2 dispatch  per-expert counts, offsets, row-tile prefix, perm / inv
+//   3 gate_up   grouped GEMM over rows gathered through perm, SiLU(gate)*up
+//               (tcgen05 for bf16, SIMT for fp32)
+//   4 down      grouped GEMM
+//   5 combine   out = x + sum_j w_j y_j in fixed slot order
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -31,11 +32,11 @@ struct moe_ctx {
     size_t elem;  // bytes per element of x / experts
 
     void *ws;  // one allocation, carved below
-    void *xn, *xp, *act, *y, *x_stage, *out_stage;
-    int32_t *idx, *hist, *base, *counts, *offsets, *mt_start, *perm, *inv;
-    float *wts;
+    void *xp, *act, *y, *x_stage, *out_stage;
+    int32_t *idx, *chunk_hist, *counts, *offsets, *mt_start, *perm, *inv;
+    float *wts, *router_wt, *router_wg, *rinv;
     int *status;
-    int rows_cap;
+    int rows_cap, e_pad, max_chunks;
 
     TcMaps maps;
     bool use_tc;
@@ -51,17 +52,21 @@ struct moe_ctx {
     long long n_fwd;
 };
 
-static const char *kKernelNames[6] = {"route", "dispatch_scan", "dispatch_scatter",
-                                      "gate_up", "down", "combine"};
+static const char *kKernelNames[] = {"route", "dispatch", "gate_up", "down", "combine"};
+constexpr int kLaunches = 5;
+constexpr int kChunkAssign = 512;  // assignments per dispatch chunk (target)
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static int toks_per_route_block(int N, int d, int E) {
-    // enough route CTAs to cover the SMs before packing tokens together, and
-    // the per-CTA rows (fp32 xn + scores) within 160 KB of shared memory
-    int tt = N >= 8 * 148 ? 8 : N >= 4 * 148 ? 4 : N >= 2 * 148 ? 2 : 1;
-    while (tt > 1 && static_cast<size_t>(tt) * (d + E) * 4 + E * 4 > 160 * 1024) tt /= 2;
-    return tt;
+// Token chunks of the dispatch: about kChunkAssign assignments each, a whole
+// number of route groups (32 tokens), histogram within 64 KB of shared memory.
+static void chunk_plan(int N, int k, int max_chunks, int *nchunk, int *chunk_tokens) {
+    int n = (N * k + kChunkAssign - 1) / kChunkAssign;
+    n = n < 1 ? 1 : n > max_chunks ? max_chunks : n;
+    int ct = (N + n - 1) / n;
+    ct = (ct + 31) / 32 * 32;
+    *chunk_tokens = ct;
+    *nchunk = (N + ct - 1) / ct;
 }
 
 extern "C" const char *moe_strerror(int code) {
@@ -123,28 +128,32 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->use_tc = (w->dtype == MOE_BF16);
     h->rows_cap = max_tokens * top_k;
 
+    h->e_pad = (n_experts + 63) / 64 * 64;
+    h->max_chunks = 16384 / n_experts < 256 ? 16384 / n_experts : 256;
+
     // workspace layout (every block 256-byte aligned)
     const size_t N = max_tokens, R = h->rows_cap, E = n_experts;
     const size_t sizes[] = {
-        N * d * h->elem,            // xn
-        R * d * h->elem,            // xp
-        R * d_ff * h->elem,         // act
-        R * d * h->elem,            // y
-        N * d * h->elem,            // x_stage
-        N * d * h->elem,            // out_stage
-        N * top_k * 4,              // idx
-        N * E * 4,                  // hist (one row per route CTA; at most N CTAs)
-        N * E * 4,                  // base
-        E * 4,                      // counts
-        (E + 1) * 4,                // offsets
-        (E + 1) * 4,                // mt_start
-        R * 4,                      // perm
-        R * 4,                      // inv
-        N * top_k * 4,              // wts
-        256,                        // status
+        R * d * h->elem,                      // xp
+        R * d_ff * h->elem,                   // act
+        R * d * h->elem,                      // y
+        N * d * h->elem,                      // x_stage
+        N * d * h->elem,                      // out_stage
+        N * top_k * 4,                        // idx
+        static_cast<size_t>(h->max_chunks) * E * 4,  // chunk_hist
+        E * 4,                                // counts
+        (E + 1) * 4,                          // offsets
+        (E + 1) * 4,                          // mt_start
+        R * 4,                                // perm
+        R * 4,                                // inv
+        N * top_k * 4,                        // wts
+        static_cast<size_t>(d) * h->e_pad * 4,  // router_wt
+        N * 4,                                // rinv
+        E * static_cast<size_t>(d) * 4,       // router_wg
+        256,                                  // status
     };
     const int nblocks = sizeof(sizes) / sizeof(sizes[0]);
-    size_t total = 0, off[16];
+    size_t total = 0, off[20];
     for (int i = 0; i < nblocks; ++i) {
         off[i] = total;
         total += (sizes[i] + 255) & ~static_cast<size_t>(255);
@@ -156,19 +165,28 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         return MOE_ERR_OOM;
     }
     uint8_t *b = static_cast<uint8_t *>(h->ws);
-    h->xn = b + off[0]; h->xp = b + off[1]; h->act = b + off[2]; h->y = b + off[3];
-    h->x_stage = b + off[4]; h->out_stage = b + off[5];
-    h->idx = reinterpret_cast<int32_t *>(b + off[6]);
-    h->hist = reinterpret_cast<int32_t *>(b + off[7]);
-    h->base = reinterpret_cast<int32_t *>(b + off[8]);
-    h->counts = reinterpret_cast<int32_t *>(b + off[9]);
-    h->offsets = reinterpret_cast<int32_t *>(b + off[10]);
-    h->mt_start = reinterpret_cast<int32_t *>(b + off[11]);
-    h->perm = reinterpret_cast<int32_t *>(b + off[12]);
-    h->inv = reinterpret_cast<int32_t *>(b + off[13]);
-    h->wts = reinterpret_cast<float *>(b + off[14]);
-    h->status = reinterpret_cast<int *>(b + off[15]);
+    h->xp = b + off[0]; h->act = b + off[1]; h->y = b + off[2];
+    h->x_stage = b + off[3]; h->out_stage = b + off[4];
+    h->idx = reinterpret_cast<int32_t *>(b + off[5]);
+    h->chunk_hist = reinterpret_cast<int32_t *>(b + off[6]);
+    h->counts = reinterpret_cast<int32_t *>(b + off[7]);
+    h->offsets = reinterpret_cast<int32_t *>(b + off[8]);
+    h->mt_start = reinterpret_cast<int32_t *>(b + off[9]);
+    h->perm = reinterpret_cast<int32_t *>(b + off[10]);
+    h->inv = reinterpret_cast<int32_t *>(b + off[11]);
+    h->wts = reinterpret_cast<float *>(b + off[12]);
+    h->router_wt = reinterpret_cast<float *>(b + off[13]);
+    h->rinv = reinterpret_cast<float *>(b + off[14]);
+    h->router_wg = reinterpret_cast<float *>(b + off[15]);
+    h->status = reinterpret_cast<int *>(b + off[16]);
     if (cudaMemset(h->ws, 0, total) != cudaSuccess) {
+        cudaFree(h->ws);
+        delete h;
+        return MOE_ERR_CUDA;
+    }
+    if (launch_prepare_router(w->router_w, w->norm_gain, h->router_wg, h->router_wt, n_experts,
+                              h->e_pad, d, 0) != MOE_OK ||
+        cudaDeviceSynchronize() != cudaSuccess) {
         cudaFree(h->ws);
         delete h;
         return MOE_ERR_CUDA;
@@ -227,32 +245,39 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
         if ((rc = (expr)) != MOE_OK) return rc; \
     } while (0)
 
-    const int tt = toks_per_route_block(N, h->d, h->E);
-    const int nblk = (N + tt - 1) / tt;
+    int tt = 0;
+    const int kind = route_plan(N, h->d, h->E, &tt);
+    int nchunk = 1, chunk_tokens = N;
+    chunk_plan(N, h->k, h->max_chunks, &nchunk, &chunk_tokens);
     const int tile_m = h->use_tc ? kTcTileM : kSimtTileM;
 
     MOE_MARK();
     RouteParams rp;
-    rp.x = x; rp.gain = h->w.norm_gain; rp.router_w = h->w.router_w; rp.bias = h->w.expert_bias;
-    rp.xn = h->xn; rp.idx = h->idx; rp.wts = h->wts; rp.hist = h->hist;
-    rp.N = N; rp.d = h->d; rp.E = h->E; rp.k = h->k; rp.eps = h->eps; rp.scale = h->scale;
-    MOE_TRY(launch_route(rp, h->dtype, tt, s));
+    rp.x = x; rp.gain = h->w.norm_gain; rp.router_w = h->w.router_w; rp.router_wt = h->router_wt;
+    rp.router_wg = h->router_wg;
+    rp.bias = h->w.expert_bias; rp.rinv = h->rinv; rp.idx = h->idx; rp.wts = h->wts;
+    rp.chunk_hist = h->chunk_hist; rp.status = h->status;
+    rp.N = N; rp.d = h->d; rp.E = h->E; rp.k = h->k; rp.e_pad = h->e_pad;
+    rp.chunk_tokens = chunk_tokens; rp.eps = h->eps; rp.scale = h->scale;
+    MOE_TRY(launch_route(rp, h->dtype, kind, tt, s));
     MOE_MARK();
 
     DispatchParams dp;
-    dp.idx = h->idx; dp.hist = h->hist; dp.base = h->base; dp.counts = h->counts;
+    dp.idx = h->idx; dp.chunk_hist = h->chunk_hist; dp.counts = h->counts;
     dp.offsets = h->offsets; dp.mt_start = h->mt_start; dp.perm = h->perm; dp.inv = h->inv;
-    dp.xn = h->xn; dp.xp = h->xp; dp.status = h->status;
-    dp.N = N; dp.d = h->d; dp.E = h->E; dp.k = h->k; dp.nblk = nblk; dp.toks_per_blk = tt;
-    dp.tile_m = tile_m; dp.elem_bytes = static_cast<int>(h->elem);
-    MOE_TRY(launch_dispatch_scan(dp, s));
-    MOE_MARK();
-    MOE_TRY(launch_dispatch_scatter(dp, s));
+    dp.status = h->status; dp.x = x; dp.gain = h->w.norm_gain; dp.rinv = h->rinv; dp.xp = h->xp;
+    dp.N = N; dp.d = h->d; dp.E = h->E; dp.k = h->k; dp.nchunk = nchunk;
+    dp.chunk_tokens = chunk_tokens; dp.tile_m = tile_m;
+    dp.elem_bytes = static_cast<int>(h->elem);
+    // several CTAs per chunk share the row copies: about four CTAs per SM in all
+    dp.replicas = (4 * h->n_sm + nchunk - 1) / nchunk;
+    if (dp.replicas > 64) dp.replicas = 64;
+    MOE_TRY(launch_dispatch(dp, s));
     MOE_MARK();
 
     GroupedParams gp;
     gp.offsets = h->offsets; gp.mt_start = h->mt_start; gp.status = h->status;
-    gp.E = h->E; gp.d = h->d; gp.I = h->I; gp.rows_cap = h->rows_cap;
+    gp.E = h->E; gp.d = h->d; gp.I = h->I; gp.k = h->k; gp.rows_cap = h->rows_cap;
     const int max_mtiles = (N * h->k + tile_m - 1) / tile_m + h->E;
 
     gp.a = h->xp; gp.w = h->w.w_gate_up; gp.c = h->act;
@@ -271,6 +296,7 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
 
     CombineParams cp;
     cp.x = x; cp.y = h->y; cp.wts = h->wts; cp.inv = h->inv; cp.out = out; cp.status = h->status;
+    cp.chunk_hist = h->chunk_hist; cp.chunk_hist_n = nchunk * h->E;
     cp.N = N; cp.d = h->d; cp.k = h->k;
     MOE_TRY(launch_combine(cp, h->dtype, s));
     MOE_MARK();
@@ -387,13 +413,13 @@ extern "C" int moe_kernel_times(moe_ctx *h, float *ms, int n) {
 
 extern "C" const char *moe_kernel_name(moe_ctx *h, int i) {
     (void)h;
-    if (i < 0 || i >= 6) return nullptr;
+    if (i < 0 || i >= kLaunches) return nullptr;
     return kKernelNames[i];
 }
 
 extern "C" int moe_launches_per_forward(moe_ctx *h, int n_tokens) {
     if (!h) return MOE_ERR_INVALID_ARG;
-    return n_tokens > 0 ? 6 : 0;
+    return n_tokens > 0 ? kLaunches : 0;
 }
 
 extern "C" int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream) {

@@ -33,28 +33,32 @@ struct RouteParams {
     const void *x;          // [N][d] f32 or bf16
     const float *gain;      // [d]
     const float *router_w;  // [E][d]
+    const float *router_wg; // [E][d] router matrix times gain (column-wise)
+    const float *router_wt; // [d][e_pad] the same transposed, zero-padded columns
     const float *bias;      // [E]
-    void *xn;               // [N][d] normalised rows, dtype of x (expert input)
+    float *rinv;            // [N] 1 / sqrt(mean(x^2) + eps) per token
     int32_t *idx;           // [N][k]
     float *wts;             // [N][k]
-    int32_t *hist;          // [gridDim.x][E] per-CTA expert counts
-    int N, d, E, k;
+    int32_t *chunk_hist;    // [nchunk][E] per token-chunk expert counts (added to)
+    int *status;
+    int N, d, E, k, e_pad, chunk_tokens;
     float eps, scale;
 };
 
 struct DispatchParams {
-    const int32_t *idx;     // [N][k]
-    const int32_t *hist;    // [nblk][E]
-    int32_t *base;          // [nblk][E] scatter base per (route CTA, expert)
-    int32_t *counts;        // [E]
-    int32_t *offsets;       // [E+1]
-    int32_t *mt_start;      // [E+1] prefix of per-expert row tiles (tile rows = tile_m)
-    int32_t *perm;          // [N*k]
-    int32_t *inv;           // [N*k]
-    const void *xn;         // [N][d]
-    void *xp;               // [N*k][d] rows of xn in grouped order
+    const void *x;             // [N][d] block input
+    const float *gain;         // [d]
+    const float *rinv;         // [N]
+    void *xp;                  // [N*k][d] normalised rows in grouped order (dtype of x)
+    const int32_t *idx;        // [N][k]
+    const int32_t *chunk_hist; // [nchunk][E]
+    int32_t *counts;           // [E]
+    int32_t *offsets;          // [E+1]
+    int32_t *mt_start;         // [E+1] prefix of per-expert row tiles (tile rows = tile_m)
+    int32_t *perm;             // [N*k] grouped row -> assignment t*k+j
+    int32_t *inv;              // [N*k] assignment -> grouped row
     int *status;
-    int N, d, E, k, nblk, toks_per_blk, tile_m, elem_bytes;
+    int N, d, E, k, nchunk, chunk_tokens, tile_m, replicas, elem_bytes;
 };
 
 struct CombineParams {
@@ -63,28 +67,35 @@ struct CombineParams {
     const float *wts;       // [N][k]
     const int32_t *inv;     // [N*k]
     void *out;              // [N][d]
+    int32_t *chunk_hist;    // zeroed here for the next forward
+    int chunk_hist_n;
     int *status;
     int N, d, k;
 };
 
 struct GroupedParams {
     // shared by the SIMT and the tensor-core grouped GEMMs
-    const int32_t *offsets;   // [E+1] row range of each expert in xp / act / y
+    const int32_t *offsets;   // [E+1] row range of each expert in the grouped order
     const int32_t *mt_start;  // [E+1] prefix of per-expert row tiles
     const void *a;            // gate/up: xp [rows][d]; down: act [rows][I]
     const void *w;            // gate/up: [E][2I][d]; down: [E][d][I]
     void *c;                  // gate/up: act [rows][I]; down: y [rows][d]
     int *status;
-    int E, d, I;
-    int rows_cap;             // allocated rows of a and c
+    int E, d, I, k;
+    int rows_cap;             // allocated grouped rows (act, y)
 };
 
 // ---------------------------------------------------------------------------
-// Host-side launchers (one per translation unit)
+// Host-side launchers
 
-int launch_route(const RouteParams &p, int dtype, int toks_per_blk, cudaStream_t s);
-int launch_dispatch_scan(const DispatchParams &p, cudaStream_t s);
-int launch_dispatch_scatter(const DispatchParams &p, cudaStream_t s);
+constexpr int kRouteSmall = 0, kRouteLarge = 1;
+bool route_small_ok(int d, int E);
+int route_plan(int N, int d, int E, int *toks_per_group);
+int launch_route(const RouteParams &p, int dtype, int kind, int toks_per_group, cudaStream_t s);
+int launch_prepare_router(const float *w, const float *gain, float *wg, float *wt, int E,
+                          int e_pad, int d, cudaStream_t s);
+size_t dispatch_smem(int nchunk, int E, int chunk_assign, int d);
+int launch_dispatch(const DispatchParams &p, cudaStream_t s);
 int launch_combine(const CombineParams &p, int dtype, cudaStream_t s);
 int launch_gemm_simt_gate_up(const GroupedParams &p, int max_mtiles, cudaStream_t s);
 int launch_gemm_simt_down(const GroupedParams &p, int max_mtiles, cudaStream_t s);
@@ -97,8 +108,8 @@ struct TcMaps {
     CUtensorMap a_down;     // act [rows][I],     box 64 x 128
     CUtensorMap w_down;     // Wd  [E*d][I],      box 64 x 256
 };
-int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu,
-                  const void *wd, int rows_cap, int E, int d, int I);
+int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, const void *wd,
+                  int rows_cap, int E, int d, int I);
 int launch_gemm_tc_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_gemm_tc_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_selftest_timeout(int *status, int timeout_us, cudaStream_t s);
@@ -177,6 +188,36 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, int
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0).
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes,
+                                              uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared (L2 only); src_bytes < 16 zero-fills.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// One arrival on `bar` once all of this thread's prior cp.async copies land
+// (the barrier's expected count must include it).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Orders shared-memory writes made through the generic proxy (st.shared,
+// cp.async) before later async-proxy reads (tcgen05.mma operands).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Same with an L2 eviction-priority hint (a createpolicy value).

@@ -1,5 +1,5 @@
 // route.cu -- fused pre-FFN RMSNorm, fp32 router, per-logit sigmoid, biased
-// top-k selection and weight normalisation (one kernel, SIMT fp32).
+// top-k selection and weight normalisation (SIMT fp32, no tensor cores).
 //
 // Follows "LFM2.5-24B-A2B: Biased Routing, Short Convolutions and Ten KV
 // Caches" (flozi.net, English page), section "The router has two different
@@ -10,23 +10,34 @@
 // fp32 (the FP8 release leaves the router gates unquantised, page 5, "Für
 // Engineers"), fed by the fp32 normalised row, never by its bf16 copy.
 //
-// One CTA of 256 threads handles TT consecutive tokens:
-//   A) one warp per token: sum of squares (fixed lane-strided order, then a
-//      butterfly), xn = x * (1/sqrt(ms + eps)) * gain kept in fp32 in shared
-//      memory and stored in the storage dtype for the experts;
-//   B) warp w owns experts w, w+8, ...; lanes split d in float4 chunks; each
-//      router row chunk is read once from L2 and used for all TT tokens;
-//      partial dot products are reduced across the warp;
-//   C) one warp per token: sigmoid, c = s + b, k rounds of a warp arg-max
-//      (ties to the lower expert index), weights, per-CTA expert histogram.
+// Two kernels, chosen by batch size:
+// The RMSNorm gain is folded into the router matrix once, at context creation
+// (W' = W_r * gain, column-wise), and 1/rms is applied to each token's dot
+// products: l_e = rinv * sum_j x_j W'_ej, the same value as W_r[e] . xn up to
+// fp32 rounding, with no per-element scaling in the inner loops.
+//   small batches: a cluster of 8 CTAs per group of TT tokens; CTA r stages
+//     its E/8 rows of W' in shared memory (one bulk copy, in flight while the
+//     1/rms factors are computed) and computes their logits (lanes split d,
+//     warp reduction); the logits go to CTA 0 through distributed shared
+//     memory, which then selects and normalises;
+//   large batches: one CTA per 32 tokens computes the 32 x 64 logit tile as a
+//     register-tiled SGEMM over d (4 x 4 outputs per thread, double-buffered
+//     shared-memory chunks of x and of W' transposed to [d][E]); its two
+//     halves take alternate chunks and their partial sums are added in a
+//     fixed order.
+// Both end with the same per-token selection: sigmoid, c = s + b, k rounds of
+// a warp arg-max (ties to the lower expert index), weights, and the count of
+// selected experts added to the token chunk's histogram (the dispatch input).
+// They store the per-token 1/rms; the dispatch writes the normalised rows
+// (x * rinv * gain, the same fp32 products) in grouped order for the experts.
+#include <cooperative_groups.h>
+
 #include "moe_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace moe {
 namespace {
-
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kEB = 8;  // experts per register block in phase B
 
 template <typename T>
 struct Vec4;
@@ -62,189 +73,429 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-template <typename T, int TT>
-__global__ void __launch_bounds__(kThreads) route_kernel(RouteParams p) {
-    extern __shared__ float4 smem_f4[];
-    float *xn_s = reinterpret_cast<float *>(smem_f4);  // [TT][d]
-    float *sc = xn_s + TT * p.d;                       // [TT][E] logits, then scores
-    int *hist = reinterpret_cast<int *>(sc + TT * p.E);  // [E]
-
-    const int d = p.d, E = p.E, k = p.k;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * TT;
-    const int ntok = min(TT, p.N - t0);
-
-    for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
-
-    // A) RMSNorm
-    for (int tl = warp; tl < TT; tl += kWarps) {
-        float *row_s = xn_s + tl * d;
-        if (tl < ntok) {
-            const T *xr = static_cast<const T *>(p.x) + static_cast<size_t>(t0 + tl) * d;
-            T *xo = static_cast<T *>(p.xn) + static_cast<size_t>(t0 + tl) * d;
-            float ss = 0.f;
-            for (int j = lane * 4; j < d; j += 128) {
-                float4 v = Vec4<T>::load(xr + j);
-                ss += v.x * v.x;
-                ss += v.y * v.y;
-                ss += v.z * v.z;
-                ss += v.w * v.w;
-            }
-            ss = warp_sum(ss);
-            const float rinv = 1.0f / sqrtf(ss / static_cast<float>(d) + p.eps);
-            for (int j = lane * 4; j < d; j += 128) {
-                float4 v = Vec4<T>::load(xr + j);
-                float4 g = *reinterpret_cast<const float4 *>(p.gain + j);
-                float4 o = make_float4(v.x * rinv * g.x, v.y * rinv * g.y, v.z * rinv * g.z,
-                                       v.w * rinv * g.w);
-                *reinterpret_cast<float4 *>(row_s + j) = o;
-                Vec4<T>::store(xo + j, o);
-            }
-        } else {
-            for (int j = lane * 4; j < d; j += 128)
-                *reinterpret_cast<float4 *>(row_s + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+// 1 / sqrt(mean(x^2) + eps) of one row, by one warp: lane-strided partial
+// sums in ascending column order (eight loads in flight), then a butterfly.
+template <typename T>
+__device__ __forceinline__ float row_rinv(const T *xr, int d, float eps, int lane) {
+    constexpr int B = 8;
+    float ss = 0.f;
+    for (int base = lane * 4; base < d; base += 128 * B) {
+        float4 v[B];
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int j = base + u * 128;
+            v[u] = j < d ? Vec4<T>::load(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            ss += v[u].x * v[u].x;
+            ss += v[u].y * v[u].y;
+            ss += v[u].z * v[u].z;
+            ss += v[u].w * v[u].w;
         }
     }
-    __syncthreads();
-
-    // B) logits l[t][e] = W_r[e] . xn_t
-    for (int eb0 = warp * kEB; eb0 < E; eb0 += kWarps * kEB) {
-        float acc[kEB][TT];
-#pragma unroll
-        for (int i = 0; i < kEB; ++i)
-#pragma unroll
-            for (int t = 0; t < TT; ++t) acc[i][t] = 0.f;
-        for (int j = lane * 4; j < d; j += 128) {
-            float4 wv[kEB];
-#pragma unroll
-            for (int i = 0; i < kEB; ++i) {
-                const int e = eb0 + i;
-                wv[i] = (e < E) ? __ldg(reinterpret_cast<const float4 *>(
-                                      p.router_w + static_cast<size_t>(e) * d + j))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                const float4 xv = *reinterpret_cast<const float4 *>(xn_s + t * d + j);
-#pragma unroll
-                for (int i = 0; i < kEB; ++i) {
-                    float a = acc[i][t];
-                    a = fmaf(wv[i].x, xv.x, a);
-                    a = fmaf(wv[i].y, xv.y, a);
-                    a = fmaf(wv[i].z, xv.z, a);
-                    a = fmaf(wv[i].w, xv.w, a);
-                    acc[i][t] = a;
-                }
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kEB; ++i)
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                const float v = warp_sum(acc[i][t]);
-                const int e = eb0 + i;
-                if (lane == 0 && e < E) sc[t * E + e] = v;
-            }
-    }
-    __syncthreads();
-
-    // C) sigmoid, biased top-k, normalised unbiased weights
-    for (int tl = warp; tl < ntok; tl += kWarps) {
-        float c_reg[kMaxExperts / 32];
-        uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
-        float *srow = sc + tl * E;
-#pragma unroll
-        for (int i = 0; i < kMaxExperts / 32; ++i) {
-            const int e = lane + 32 * i;
-            c_reg[i] = -INFINITY;
-            if (e < E) {
-                const float s = 1.0f / (1.0f + expf(-srow[e]));
-                const float c = s + p.bias[e];
-                c_reg[i] = (c == c) ? c : -INFINITY;  // a NaN score never wins
-                srow[e] = s;  // each lane rewrites only its own experts
-            } else {
-                taken |= 1u << i;
-            }
-        }
-        __syncwarp();
-        int sel[kMaxTopK];
-        float ssel[kMaxTopK];
-        for (int j = 0; j < k; ++j) {
-            float bc = -INFINITY;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < kMaxExperts / 32; ++i) {
-                const int e = lane + 32 * i;
-                // ascending e within a lane: ties keep the lower index
-                if (!(taken & (1u << i)) && (c_reg[i] > bc || be == 0x7fffffff)) {
-                    bc = c_reg[i];
-                    be = e;
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                if (oe != 0x7fffffff && (be == 0x7fffffff || oc > bc || (oc == bc && oe < be))) {
-                    bc = oc;
-                    be = oe;
-                }
-            }
-            // k <= E guarantees an untaken expert exists, so be < E here
-            sel[j] = be;
-            ssel[j] = srow[be];
-#pragma unroll
-            for (int i = 0; i < kMaxExperts / 32; ++i)
-                if (lane + 32 * i == be) taken |= 1u << i;
-        }
-        if (lane == 0) {
-            float sum = 0.f;
-            for (int j = 0; j < k; ++j) sum += ssel[j];
-            const float den = sum + p.eps;
-            const size_t t = static_cast<size_t>(t0 + tl);
-            for (int j = 0; j < k; ++j) {
-                p.idx[t * k + j] = sel[j];
-                p.wts[t * k + j] = p.scale * (ssel[j] / den);
-                atomicAdd(&hist[sel[j]], 1);
-            }
-        }
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kThreads)
-        p.hist[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+    ss = warp_sum(ss);
+    return 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
 }
 
-template <typename T, int TT>
-int launch_tt(const RouteParams &p, cudaStream_t s) {
-    const int nblk = (p.N + TT - 1) / TT;
-    const size_t smem = (static_cast<size_t>(TT) * p.d + static_cast<size_t>(TT) * p.E) * 4 +
-                        static_cast<size_t>(p.E) * 4;
-    auto kern = route_kernel<T, TT>;
-    if (smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess)
-            return MOE_ERR_CUDA;
+// Selection and weights of one token by one warp. srow[E] holds its logits
+// (overwritten with the sigmoid scores); the result goes to idx/wts row t and
+// the expert counts to hist (shared).
+__device__ __forceinline__ void select_token(const RouteParams &p, float *srow, size_t t,
+                                             int *hist, int lane) {
+    const int E = p.E, k = p.k;
+    float c_reg[kMaxExperts / 32];
+    uint32_t taken = 0;  // bit i: expert lane + 32 i is unavailable
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+        const int e = lane + 32 * i;
+        c_reg[i] = -INFINITY;
+        if (e < E) {
+            const float s = 1.0f / (1.0f + expf(-srow[e]));
+            const float c = s + p.bias[e];
+            c_reg[i] = (c == c) ? c : -INFINITY;  // a NaN score never wins
+            srow[e] = s;  // each lane rewrites only its own experts
+        } else {
+            taken |= 1u << i;
+        }
     }
-    kern<<<nblk, kThreads, smem, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    __syncwarp();
+    int sel[kMaxTopK];
+    float ssel[kMaxTopK];
+    for (int j = 0; j < k; ++j) {
+        float bc = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kMaxExperts / 32; ++i) {
+            // ascending expert index within a lane: ties keep the lower index
+            if (!(taken & (1u << i)) && (c_reg[i] > bc || be == 0x7fffffff)) {
+                bc = c_reg[i];
+                be = lane + 32 * i;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (oe != 0x7fffffff && (be == 0x7fffffff || oc > bc || (oc == bc && oe < be))) {
+                bc = oc;
+                be = oe;
+            }
+        }
+        // k <= E guarantees an untaken expert exists, so be < E here
+        sel[j] = be;
+        ssel[j] = srow[be];
+#pragma unroll
+        for (int i = 0; i < kMaxExperts / 32; ++i)
+            if (lane + 32 * i == be) taken |= 1u << i;
+    }
+    if (lane == 0) {
+        float sum = 0.f;
+        for (int j = 0; j < k; ++j) sum += ssel[j];
+        const float den = sum + p.eps;
+        for (int j = 0; j < k; ++j) {
+            p.idx[t * k + j] = sel[j];
+            p.wts[t * k + j] = p.scale * (ssel[j] / den);
+            atomicAdd(&hist[sel[j]], 1);
+        }
+    }
+}
+
+// Adds a CTA's expert counts to the histogram of the token chunk it lies in.
+__device__ __forceinline__ void flush_hist(const RouteParams &p, const int *hist, int t0) {
+    int32_t *row = p.chunk_hist + static_cast<size_t>(t0 / p.chunk_tokens) * p.E;
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        if (hist[e]) atomicAdd(&row[e], hist[e]);
+}
+
+// ---------------------------------------------------------------------------
+// Small batches: cluster of 8 CTAs, CTA r owns experts [r*EG, (r+1)*EG).
+
+constexpr int kSmallThreads = 256;
+constexpr int kClusterCtas = 8;
+
+template <typename T, int TPW, int EG>
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kSmallThreads)
+    route_small_kernel(RouteParams p) {
+    constexpr int TT = 8 * TPW;  // tokens per cluster
+    extern __shared__ float4 smem_f4[];
+    float *wsl = reinterpret_cast<float *>(smem_f4);  // [EG][d] router rows times gain
+    float *sc = wsl + EG * p.d;                       // [TT][E] (used in CTA 0)
+    int *hist = reinterpret_cast<int *>(sc + TT * p.E);
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int d = p.d, E = p.E;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = (blockIdx.x / kClusterCtas) * TT;
+    const int e0 = rank * EG;
+
+    // router rows of this CTA -> shared memory, one bulk copy in flight while
+    // the normalisation factors are computed
+    __shared__ uint64_t wbar;
+    if (threadIdx.x == 0) {
+        mbar_init(&wbar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const uint32_t wbytes = static_cast<uint32_t>(EG) * d * 4;
+    if (threadIdx.x == 0) {
+        const float *src = p.router_wg + static_cast<size_t>(e0) * d;
+        mbar_arrive_expect_tx(&wbar, wbytes);
+        for (uint32_t off = 0; off < wbytes; off += 32768u)
+            bulk_copy_g2s(wsl + off / 4, src + off / 4, min(32768u, wbytes - off), &wbar);
+    }
+    for (int e = threadIdx.x; e < E; e += kSmallThreads) hist[e] = 0;
+
+    // normalisation factors of this warp's tokens
+    float rinv[TPW];
+    const T *xr[TPW];
+#pragma unroll
+    for (int i = 0; i < TPW; ++i) {
+        const int t = t0 + warp * TPW + i;
+        const bool valid = t < p.N;
+        xr[i] = static_cast<const T *>(p.x) + static_cast<size_t>(valid ? t : 0) * d;
+        rinv[i] = valid ? row_rinv<T>(xr[i], d, p.eps, lane) : 0.f;
+        if (valid && rank == 0 && lane == 0) p.rinv[t] = rinv[i];
+    }
+    if (!mbar_wait(&wbar, 0, globaltimer_ns() + 1000000000ull)) set_status(p.status, kStatusTimeout);
+    __syncthreads();
+
+    // acc[e][i] = sum_j x[t_i][j] * (W_r[e][j] * gain[j]); the logit is rinv * acc
+    float acc[EG][TPW];
+#pragma unroll
+    for (int e = 0; e < EG; ++e)
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) acc[e][i] = 0.f;
+#pragma unroll 4
+    for (int j = lane * 4; j < d; j += 128) {
+        float4 xv[TPW];
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) xv[i] = Vec4<T>::load(xr[i] + j);
+#pragma unroll
+        for (int e = 0; e < EG; ++e) {
+            const float4 w = *reinterpret_cast<const float4 *>(wsl + e * d + j);
+#pragma unroll
+            for (int i = 0; i < TPW; ++i) {
+                float a = acc[e][i];
+                a = fmaf(w.x, xv[i].x, a);
+                a = fmaf(w.y, xv[i].y, a);
+                a = fmaf(w.z, xv[i].z, a);
+                a = fmaf(w.w, xv[i].w, a);
+                acc[e][i] = a;
+            }
+        }
+    }
+    float *sc0 = cluster.map_shared_rank(sc, 0);
+#pragma unroll
+    for (int e = 0; e < EG; ++e)
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+            const float v = warp_sum(acc[e][i]) * rinv[i];
+            if (lane == 0) sc0[(warp * TPW + i) * E + e0 + e] = v;
+        }
+    cluster.sync();
+    if (rank != 0) return;
+
+    const int ntok = min(TT, p.N - t0);
+    for (int tl = warp; tl < ntok; tl += kSmallThreads / 32)
+        select_token(p, sc + tl * E, static_cast<size_t>(t0 + tl), hist, lane);
+    __syncthreads();
+    flush_hist(p, hist, t0);
+}
+
+// ---------------------------------------------------------------------------
+// Large batches: 32 tokens x all experts per CTA, register-tiled SGEMM; the
+// two halves of the CTA take alternate d-chunks and their partial sums are
+// added in a fixed order.
+
+constexpr int kLargeThreads = 256;
+constexpr int LT = 32;   // tokens per CTA
+constexpr int LKC = 32;  // d per shared-memory chunk
+constexpr int LXS = LT + 4;
+constexpr int kGroupThreads = 128;
+
+size_t large_smem(int E) {
+    return (2 * 2 * LKC * LXS + 2 * 2 * LKC * 64 + LT * 64 + LT * static_cast<size_t>(E) + LT) * 4 +
+           static_cast<size_t>(E) * 4;
 }
 
 template <typename T>
-int launch_t(const RouteParams &p, int tt, cudaStream_t s) {
-    switch (tt) {
-        case 1: return launch_tt<T, 1>(p, s);
-        case 2: return launch_tt<T, 2>(p, s);
-        case 4: return launch_tt<T, 4>(p, s);
-        case 8: return launch_tt<T, 8>(p, s);
+__global__ void __launch_bounds__(kLargeThreads) route_large_kernel(RouteParams p) {
+    extern __shared__ float4 smem_f4[];
+    float *xs_all = reinterpret_cast<float *>(smem_f4);        // [2 grp][2 buf][LKC][LXS]
+    float *ws_all = xs_all + 2 * 2 * LKC * LXS;                // [2 grp][2 buf][LKC][64]
+    float *red = ws_all + 2 * 2 * LKC * 64;                    // [LT][64] second half's sums
+    float *sc = red + LT * 64;                                 // [LT][E]
+    float *rinv_s = sc + LT * p.E;                             // [LT]
+    int *hist = reinterpret_cast<int *>(rinv_s + LT);          // [E]
+
+    const int d = p.d, E = p.E, Ep = p.e_pad;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = tid / kGroupThreads, gt = tid % kGroupThreads;
+    const int t0 = blockIdx.x * LT;
+    const int ntok = min(LT, p.N - t0);
+    for (int e = tid; e < E; e += kLargeThreads) hist[e] = 0;
+    for (int tl = warp; tl < LT; tl += kLargeThreads / 32) {
+        const float r = tl < ntok ? row_rinv<T>(static_cast<const T *>(p.x) +
+                                                    static_cast<size_t>(t0 + tl) * d,
+                                                d, p.eps, lane)
+                                  : 0.f;
+        if (lane == 0) {
+            rinv_s[tl] = r;
+            if (tl < ntok) p.rinv[t0 + tl] = r;
+        }
+    }
+    __syncthreads();
+
+    // loader roles: x -- token xt (the lane, so the transposed stores of a
+    // warp hit 32 distinct banks), 8 consecutive columns at xq*8 (the warp);
+    // W'^T -- 4 float4 slots
+    const int xt = gt & 31, xq = gt >> 5;
+    const bool xvalid = xt < ntok;
+    const T *xrow = static_cast<const T *>(p.x) + static_cast<size_t>(xvalid ? t0 + xt : 0) * d;
+    // compute roles: tokens ty*4.., experts tx*4..
+    const int ty = gt >> 4, tx = gt & 15;
+    const int nchunk = (d + LKC - 1) / LKC;
+    const int rounds = (nchunk + 1) / 2;  // chunk 2*r + grp in round r
+    float *xs_g = xs_all + grp * 2 * LKC * LXS;
+    float *ws_g = ws_all + grp * 2 * LKC * 64;
+
+    for (int eb = 0; eb < E; eb += 64) {
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+        float4 xa, xb, wv[4];
+        auto fetch = [&](int c) {
+            const int k0 = c * LKC;
+            const int j = k0 + xq * 8;
+            if (c < nchunk && j < d) {
+                xa = Vec4<T>::load(xrow + j);
+                xb = (j + 4 < d) ? Vec4<T>::load(xrow + j + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                xa = xb = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int slot = gt + kGroupThreads * i;  // 512 float4 = 32 rows x 16
+                const int row = k0 + (slot >> 4), col = eb + (slot & 15) * 4;
+                wv[i] = (c < nchunk && row < d)
+                            ? __ldg(reinterpret_cast<const float4 *>(
+                                  p.router_wt + static_cast<size_t>(row) * Ep + col))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        };
+        fetch(grp);
+        for (int r = 0; r < rounds; ++r) {
+            const int c = 2 * r + grp;
+            const int buf = r & 1;
+            float *xs = xs_g + buf * LKC * LXS;
+            float *ws = ws_g + buf * LKC * 64;
+            const float v[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xs[(xq * 8 + q) * LXS + xt] = v[q];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int slot = gt + kGroupThreads * i;
+                *reinterpret_cast<float4 *>(&ws[(slot >> 4) * 64 + (slot & 15) * 4]) = wv[i];
+            }
+            __syncthreads();
+            fetch(c + 2);
+#pragma unroll
+            for (int kk = 0; kk < LKC; ++kk) {
+                const float4 a = *reinterpret_cast<const float4 *>(&xs[kk * LXS + ty * 4]);
+                const float4 b = *reinterpret_cast<const float4 *>(&ws[kk * 64 + tx * 4]);
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            }
+        }
+        if (grp == 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) red[(ty * 4 + i) * 64 + tx * 4 + j] = acc[i][j];
+        __syncthreads();
+        if (grp == 0)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int e = eb + tx * 4 + j;
+                    if (e < E)
+                        sc[(ty * 4 + i) * E + e] =
+                            (acc[i][j] + red[(ty * 4 + i) * 64 + tx * 4 + j]) * rinv_s[ty * 4 + i];
+                }
+        __syncthreads();
+    }
+
+    for (int tl = warp; tl < ntok; tl += kLargeThreads / 32)
+        select_token(p, sc + tl * E, static_cast<size_t>(t0 + tl), hist, lane);
+    __syncthreads();
+    flush_hist(p, hist, t0);
+}
+
+template <typename K>
+int set_smem(K kern, size_t smem) {
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+template <typename T, int TPW, int EG>
+int launch_small(const RouteParams &p, cudaStream_t s) {
+    constexpr int TT = 8 * TPW;
+    const int groups = (p.N + TT - 1) / TT;
+    const size_t smem = (static_cast<size_t>(EG) * p.d + static_cast<size_t>(TT) * p.E) * 4 +
+                        static_cast<size_t>(p.E) * 4;
+    auto kern = route_small_kernel<T, TPW, EG>;
+    if (set_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
+    kern<<<groups * kClusterCtas, kSmallThreads, smem, s>>>(p);
+    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <typename T, int TPW>
+int launch_small_eg(const RouteParams &p, cudaStream_t s) {
+    switch (p.E / kClusterCtas) {
+        case 1: return launch_small<T, TPW, 1>(p, s);
+        case 2: return launch_small<T, TPW, 2>(p, s);
+        case 4: return launch_small<T, TPW, 4>(p, s);
+        case 8: return launch_small<T, TPW, 8>(p, s);
+        case 16: return launch_small<T, TPW, 16>(p, s);
         default: return MOE_ERR_INVALID_ARG;
+    }
+}
+
+template <typename T>
+int launch_small_t(const RouteParams &p, int tt, cudaStream_t s) {
+    switch (tt) {
+        case 8: return launch_small_eg<T, 1>(p, s);
+        case 16: return launch_small_eg<T, 2>(p, s);
+        case 32: return launch_small_eg<T, 4>(p, s);
+        default: return MOE_ERR_INVALID_ARG;
+    }
+}
+
+template <typename T>
+int launch_large(const RouteParams &p, cudaStream_t s) {
+    const size_t smem = large_smem(p.E);
+    auto kern = route_large_kernel<T>;
+    if (set_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
+    kern<<<(p.N + LT - 1) / LT, kLargeThreads, smem, s>>>(p);
+    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// W' = W_r * gain (column-wise), stored as [E][d] (wg) and as [d][e_pad] with
+// zero columns past E (wt).
+__global__ void prepare_router_kernel(const float *w, const float *gain, float *wg, float *wt,
+                                      int E, int e_pad, int d) {
+    const size_t n = static_cast<size_t>(d) * e_pad;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const int j = static_cast<int>(i / e_pad), e = static_cast<int>(i % e_pad);
+        const float v = e < E ? w[static_cast<size_t>(e) * d + j] * gain[j] : 0.f;
+        wt[i] = v;
+        if (e < E) wg[static_cast<size_t>(e) * d + j] = v;
     }
 }
 
 }  // namespace
 
-int launch_route(const RouteParams &p, int dtype, int toks_per_blk, cudaStream_t s) {
-    if (dtype == MOE_F32) return launch_t<float>(p, toks_per_blk, s);
-    return launch_t<__nv_bfloat16>(p, toks_per_blk, s);
+int launch_prepare_router(const float *w, const float *gain, float *wg, float *wt, int E,
+                          int e_pad, int d, cudaStream_t s) {
+    prepare_router_kernel<<<256, 256, 0, s>>>(w, gain, wg, wt, E, e_pad, d);
+    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool route_small_ok(int d, int E) {
+    if (E % kClusterCtas != 0) return false;
+    const int eg = E / kClusterCtas;
+    if (eg != 1 && eg != 2 && eg != 4 && eg != 8 && eg != 16) return false;
+    return static_cast<size_t>(eg) * d * 4 + 32 * static_cast<size_t>(E) * 4 <= 160 * 1024;
+}
+
+int route_plan(int N, int d, int E, int *toks_per_group) {
+    // the cluster kernel while its groups give fewer CTAs than the tiled
+    // kernel would need to fill the GPU twice; the tiled kernel beyond
+    if (route_small_ok(d, E) && N < 4096) {
+        *toks_per_group = N <= 64 ? 8 : N <= 256 ? 16 : 32;
+        return kRouteSmall;
+    }
+    *toks_per_group = LT;
+    return kRouteLarge;
+}
+
+int launch_route(const RouteParams &p, int dtype, int kind, int toks_per_group, cudaStream_t s) {
+    if (kind == kRouteSmall)
+        return dtype == MOE_F32 ? launch_small_t<float>(p, toks_per_group, s)
+                                : launch_small_t<__nv_bfloat16>(p, toks_per_group, s);
+    return dtype == MOE_F32 ? launch_large<float>(p, s) : launch_large<__nv_bfloat16>(p, s);
 }
 
 }  // namespace moe
