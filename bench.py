@@ -205,8 +205,6 @@ def run_ours(args, w, world, rank, local):
         active.append(int((np.diff(off) > 0).sum()))
     torch.cuda.synchronize()
 
-    for m in mods:
-        m.profile(True)
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -222,6 +220,14 @@ def run_ours(args, w, world, rank, local):
     clk = clocks.stop()
     barrier(world)
     local_s = e0.elapsed_time(e1) / 1e3
+    # per-kernel durations: a second pass of the same steps with CUDA events
+    # recorded between the launches on the launching stream (the events
+    # separate the launches, so these durations include launch gaps)
+    for m in mods:
+        m.profile(True)
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
     ktimes = {}
     for m in mods:
         for name, ms in m.kernel_times().items():

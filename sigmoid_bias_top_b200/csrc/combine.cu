@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     constexpr int V = P::V;
     const int t = blockIdx.x;
     const int k = p.k;
+    pdl_trigger();
+    pdl_wait();
     if (t == 0)  // the dispatch has consumed the chunk histogram: clear it for the next forward
         for (int i = threadIdx.x; i < p.chunk_hist_n; i += kThreads) p.chunk_hist[i] = 0;
     const int nvec = p.d / V;
@@ -89,11 +91,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
 }  // namespace
 
 int launch_combine(const CombineParams &p, int dtype, cudaStream_t s) {
-    if (dtype == MOE_F32)
-        combine_kernel<F32x4><<<p.N, kThreads, 0, s>>>(p);
-    else
-        combine_kernel<Bf16x8><<<p.N, kThreads, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (dtype == MOE_F32) return launch_k(combine_kernel<F32x4>, dim3(p.N), dim3(kThreads), 0, s, p);
+    return launch_k(combine_kernel<Bf16x8>, dim3(p.N), dim3(kThreads), 0, s, p);
 }
 
 }  // namespace moe

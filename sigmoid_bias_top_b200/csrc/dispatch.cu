@@ -74,8 +74,10 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
     const int c = blockIdx.x / p.replicas, rep = blockIdx.x % p.replicas;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    for (int i = tid; i < d / 4; i += kThreads)
+    for (int i = tid; i < d / 4; i += kThreads)  // a layer parameter: no earlier kernel writes it
         reinterpret_cast<float4 *>(gs)[i] = __ldg(reinterpret_cast<const float4 *>(p.gain) + i);
+    pdl_trigger();
+    pdl_wait();
     for (int i = tid; i < nchunk * E; i += kThreads) hist[i] = p.chunk_hist[i];
     for (int i = tid; i < kWarps * E; i += kThreads) wcnt[i] = 0;
     __syncthreads();
@@ -224,12 +226,8 @@ size_t dispatch_smem(int nchunk, int E, int chunk_assign, int d) {
 
 int launch_dispatch(const DispatchParams &p, cudaStream_t s) {
     const size_t smem = dispatch_smem(p.nchunk, p.E, p.chunk_tokens * p.k, p.d);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    dispatch_kernel<<<p.nchunk * p.replicas, kThreads, smem, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (ensure_smem(dispatch_kernel, smem) != MOE_OK) return MOE_ERR_CUDA;
+    return launch_k(dispatch_kernel, dim3(p.nchunk * p.replicas), dim3(kThreads), smem, s, p);
 }
 
 }  // namespace moe

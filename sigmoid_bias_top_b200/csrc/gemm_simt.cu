@@ -45,6 +45,8 @@ __global__ void __launch_bounds__(kThreads) grouped_simt_kernel(GroupedParams p)
     __shared__ float Bs[GATE_UP ? 2 : 1][BK][BN + 4];
     const int E = p.E;
     const int mt = blockIdx.x;
+    pdl_trigger();
+    pdl_wait();
     if (mt >= p.mt_start[E]) return;
     const int e = find_expert(p.mt_start, E, mt);
     const int row0 = p.offsets[e] + (mt - p.mt_start[e]) * BM;
@@ -121,15 +123,13 @@ __global__ void __launch_bounds__(kThreads) grouped_simt_kernel(GroupedParams p)
 }  // namespace
 
 int launch_gemm_simt_gate_up(const GroupedParams &p, int max_mtiles, cudaStream_t s) {
-    dim3 grid(max_mtiles, (p.I + BN - 1) / BN);
-    grouped_simt_kernel<float, true><<<grid, kThreads, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_k(grouped_simt_kernel<float, true>, dim3(max_mtiles, (p.I + BN - 1) / BN),
+                    dim3(kThreads), 0, s, p);
 }
 
 int launch_gemm_simt_down(const GroupedParams &p, int max_mtiles, cudaStream_t s) {
-    dim3 grid(max_mtiles, (p.d + BN - 1) / BN);
-    grouped_simt_kernel<float, false><<<grid, kThreads, 0, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_k(grouped_simt_kernel<float, false>, dim3(max_mtiles, (p.d + BN - 1) / BN),
+                    dim3(kThreads), 0, s, p);
 }
 
 }  // namespace moe

@@ -124,10 +124,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
-    for (int i = threadIdx.x; i <= E; i += kThreads) {
-        mts[i] = p.mt_start[i];
-        offs[i] = p.offsets[i];
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&ctl->full[s], 1);
@@ -148,6 +144,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+    }
+    // everything above overlaps the previous kernel; the schedule below is its output
+    pdl_trigger();
+    pdl_wait();
+    for (int i = threadIdx.x; i <= E; i += kThreads) {
+        mts[i] = p.mt_start[i];
+        offs[i] = p.offsets[i];
     }
     tc_fence_before();
     __syncthreads();
@@ -373,11 +376,8 @@ int launch(const CUtensorMap &a, const CUtensorMap &b, const GroupedParams &p, i
            cudaStream_t s) {
     auto kern = grouped_tc_kernel<GATE_UP>;
     const size_t smem = smem_bytes(p.E);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    kern<<<n_sm, kThreads, smem, s>>>(a, b, p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
+    return launch_k(kern, dim3(n_sm), dim3(kThreads), smem, s, a, b, p);
 }
 
 }  // namespace

@@ -14,6 +14,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "moe_internal.cuh"
@@ -67,6 +69,20 @@ static void chunk_plan(int N, int k, int max_chunks, int *nchunk, int *chunk_tok
     ct = (ct + 31) / 32 * 32;
     *chunk_tokens = ct;
     *nchunk = (N + ct - 1) / ct;
+}
+
+int moe::ensure_smem_ptr(const void *kern, size_t smem) {
+    static std::mutex mu;
+    static std::unordered_map<const void *, size_t> set;  // per process (one device each)
+    if (smem <= 48 * 1024) return MOE_OK;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t &cur = set[kern];
+    if (smem <= cur) return MOE_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    cur = smem;
+    return MOE_OK;
 }
 
 extern "C" const char *moe_strerror(int code) {

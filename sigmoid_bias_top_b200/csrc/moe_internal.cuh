@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -115,7 +117,46 @@ int launch_gemm_tc_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaS
 int launch_selftest_timeout(int *status, int timeout_us, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
+// Launch with programmatic dependent launch: the kernel may be scheduled while
+// its predecessor in the stream is still running; it must call pdl_wait()
+// before touching anything the predecessor writes or reads.
+
+template <typename... KArgs, typename... Args>
+inline int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                    Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess
+               ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Raises a kernel's dynamic shared-memory limit (once per kernel and size).
+int ensure_smem_ptr(const void *kern, size_t smem);
+template <typename K>
+inline int ensure_smem(K kern, size_t smem) {
+    return ensure_smem_ptr(reinterpret_cast<const void *>(kern), smem);
+}
+
+// ---------------------------------------------------------------------------
 // Small device helpers
+
+// Lets the next kernel in the stream be scheduled (its pdl_wait still waits
+// for this whole grid to finish).
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the preceding kernel in the stream has completed and its
+// memory operations are visible (returns at once without a predecessor).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t u) {
     return __uint_as_float(static_cast<uint32_t>(u) << 16);

@@ -199,13 +199,15 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kSmallThr
     }
     __syncthreads();
     const uint32_t wbytes = static_cast<uint32_t>(EG) * d * 4;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0) {  // the router copy depends on no earlier kernel
         const float *src = p.router_wg + static_cast<size_t>(e0) * d;
         mbar_arrive_expect_tx(&wbar, wbytes);
         for (uint32_t off = 0; off < wbytes; off += 32768u)
             bulk_copy_g2s(wsl + off / 4, src + off / 4, min(32768u, wbytes - off), &wbar);
     }
     for (int e = threadIdx.x; e < E; e += kSmallThreads) hist[e] = 0;
+    pdl_trigger();
+    pdl_wait();
 
     // normalisation factors of this warp's tokens
     float rinv[TPW];
@@ -296,6 +298,8 @@ __global__ void __launch_bounds__(kLargeThreads) route_large_kernel(RouteParams 
     const int t0 = blockIdx.x * LT;
     const int ntok = min(LT, p.N - t0);
     for (int e = tid; e < E; e += kLargeThreads) hist[e] = 0;
+    pdl_trigger();
+    pdl_wait();
     for (int tl = warp; tl < LT; tl += kLargeThreads / 32) {
         const float r = tl < ntok ? row_rinv<T>(static_cast<const T *>(p.x) +
                                                     static_cast<size_t>(t0 + tl) * d,
@@ -399,14 +403,6 @@ __global__ void __launch_bounds__(kLargeThreads) route_large_kernel(RouteParams 
     flush_hist(p, hist, t0);
 }
 
-template <typename K>
-int set_smem(K kern, size_t smem) {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    return MOE_OK;
-}
 
 template <typename T, int TPW, int EG>
 int launch_small(const RouteParams &p, cudaStream_t s) {
@@ -415,9 +411,8 @@ int launch_small(const RouteParams &p, cudaStream_t s) {
     const size_t smem = (static_cast<size_t>(EG) * p.d + static_cast<size_t>(TT) * p.E) * 4 +
                         static_cast<size_t>(p.E) * 4;
     auto kern = route_small_kernel<T, TPW, EG>;
-    if (set_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
-    kern<<<groups * kClusterCtas, kSmallThreads, smem, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
+    return launch_k(kern, dim3(groups * kClusterCtas), dim3(kSmallThreads), smem, s, p);
 }
 
 template <typename T, int TPW>
@@ -446,9 +441,8 @@ template <typename T>
 int launch_large(const RouteParams &p, cudaStream_t s) {
     const size_t smem = large_smem(p.E);
     auto kern = route_large_kernel<T>;
-    if (set_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
-    kern<<<(p.N + LT - 1) / LT, kLargeThreads, smem, s>>>(p);
-    return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
+    return launch_k(kern, dim3((p.N + LT - 1) / LT), dim3(kLargeThreads), smem, s, p);
 }
 
 // W' = W_r * gain (column-wise), stored as [E][d] (wg) and as [d][e_pad] with
