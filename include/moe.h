@@ -127,6 +127,27 @@ int moe_launches_per_forward(moe_ctx *h, int n_tokens);
  * records MOE_ERR_DEVICE_TIMEOUT in the status word. The context stays usable. */
 int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream);
 
+/* Routing of a batch with no device allocation: for callers that cannot
+ * allocate device memory where they route (while a stream is being captured
+ * into a CUDA graph, in serving loops that forbid allocator calls because
+ * they may synchronise the device, or under a memory planner that owns all
+ * device memory). The page describes no such entry point; it is an interface
+ * of this library only. Computes, for x[n_tokens][d] (dtype MOE_F32 or
+ * MOE_BF16) and the fp32 norm_gain[d], router_w[E][d], expert_bias[E], the
+ * same idx[n_tokens][top_k] (int32, slot order) and w[n_tokens][top_k] (fp32)
+ * as moe_forward's routing (see moe_debug_routing). All pointers are device
+ * pointers owned by the caller; x, norm_gain and router_w 16-byte aligned.
+ * Limits of the fixed scratch: n_tokens <= 4096 (else MOE_ERR_TOO_MANY_TOKENS),
+ * n_experts <= 64 and d <= 2048 (else MOE_ERR_UNSUPPORTED_SHAPE), d % 4 == 0,
+ * 1 <= top_k <= min(n_experts, 8). The scratch is one array compiled into the
+ * library, about 1.1 MB on every GPU that loads it, held until the process
+ * exits; a device's first call looks its address up (make that first call
+ * before any stream capture). Calls share the array: calls that overlap on
+ * the GPU race, calls ordered on one stream do not. Asynchronous on stream. */
+int moe_route_noalloc(const void *x, int dtype, const float *norm_gain, const float *router_w,
+                      const float *expert_bias, int n_tokens, int d, int n_experts, int top_k,
+                      float eps, float routed_scale, int32_t *idx, float *w, void *stream);
+
 /* Static description of a moe_err code. */
 const char *moe_strerror(int code);
 

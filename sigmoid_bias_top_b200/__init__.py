@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.moe_kernel_name.restype = ctypes.c_char_p
         L.moe_launches_per_forward.argtypes = [P, I]
         L.moe_selftest_timeout.argtypes = [P, I, P]
+        L.moe_route_noalloc.argtypes = [P, I, P, P, P, I, I, I, I, F, F, P, P, P]
+        L.moe_route_noalloc.restype = I
         L.moe_strerror.argtypes = [I]
         L.moe_strerror.restype = ctypes.c_char_p
         for f in (L.moe_create, L.moe_forward, L.moe_forward_host, L.moe_destroy,
@@ -89,6 +91,28 @@ def _stream_ptr(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def route_noalloc(x, layer: Dict, top_k: int, eps: float = 1e-6, routed_scale: float = 1.0,
+                  idx=None, w=None, stream=None):
+    """Routing without device allocation (moe_route_noalloc): returns (idx, w).
+
+    For callers that must not allocate device memory at this point (stream
+    capture, allocator-free serving loops); idx and w may be passed in
+    preallocated so that the call itself allocates nothing."""
+    import torch
+    n, d = x.shape
+    E = layer["router_w"].shape[0]
+    if idx is None:
+        idx = torch.empty(n, top_k, dtype=torch.int32, device=x.device)
+    if w is None:
+        w = torch.empty(n, top_k, dtype=torch.float32, device=x.device)
+    dt = MOE_BF16 if x.dtype == torch.bfloat16 else MOE_F32
+    _check(lib().moe_route_noalloc(x.data_ptr(), dt, layer["norm_gain"].data_ptr(),
+                                   layer["router_w"].data_ptr(), layer["bias"].data_ptr(), n, d, E,
+                                   top_k, eps, routed_scale, idx.data_ptr(), w.data_ptr(),
+                                   _stream_ptr(stream)), "moe_route_noalloc")
+    return idx, w
 
 
 class MoeLayer:
