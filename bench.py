@@ -272,7 +272,10 @@ def run_ours(args, w, world, rank, local):
     bpe = 2 if w.dtype == "bf16" else 4
     if N * w.top_k / max(U, 1) < 64:  # weight-streaming regime: HBM-bound
         bound = "hbm"
-        if dom == "gate_up":
+        if dom == "experts":   # both contractions in one launch
+            work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + A.down_bytes(U, w.d, w.d_ff, bpe)
+                    + 2 * n_assign * (w.d + w.d_ff) * bpe)
+        elif dom == "gate_up":
             work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe)
         elif dom == "down":
             work = A.down_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe

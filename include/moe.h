@@ -116,7 +116,9 @@ int moe_debug_routing(moe_ctx *h, int32_t *idx, float *w, int32_t *perm,
  * was recorded, or a negative moe_err. moe_profile(h, 0) stops recording. */
 int moe_profile(moe_ctx *h, int enable);
 int moe_kernel_times(moe_ctx *h, float *ms, int n);
-/* Name of kernel i of the forward's launch sequence (static string), or NULL. */
+/* Name of kernel i of the last forward's launch sequence (static string), or
+ * NULL: route, dispatch, gate_up, down, combine; or route, dispatch, experts,
+ * combine when the batch was small enough for the fused expert kernel. */
 const char *moe_kernel_name(moe_ctx *h, int i);
 
 /* Number of kernel launches one forward makes for n_tokens tokens. */

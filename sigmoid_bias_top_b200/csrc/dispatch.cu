@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
         p.offsets[E] = total_rows;
         p.mt_start[E] = total_tiles;
     }
+    if (blockIdx.x == 0 && p.sched)
+        for (int i = tid; i < p.sched_n; i += kThreads) p.sched[i] = 0;
     __syncthreads();
 
     // 2. this chunk's assignments a = t*k + j, t in [t0, t1)

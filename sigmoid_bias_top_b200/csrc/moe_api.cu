@@ -41,9 +41,12 @@ struct moe_ctx {
     int rows_cap, e_pad, max_chunks;
 
     TcMaps maps;
+    void *decode_maps;   // tensor maps of the fused small-batch kernel
+    int32_t *sched;      // [1 + E] its work counter and per-expert completion counts
     bool use_tc;
 
     int last_n;
+    bool last_fused;  // the last forward used the fused small-batch expert kernel
 
     // profiling: a ring of event sets, one set (kEvPerFwd events) per forward
     bool profile;
@@ -55,7 +58,7 @@ struct moe_ctx {
 };
 
 static const char *kKernelNames[] = {"route", "dispatch", "gate_up", "down", "combine"};
-constexpr int kLaunches = 5;
+static const char *kFusedKernelNames[] = {"route", "dispatch", "experts", "combine"};
 constexpr int kChunkAssign = 512;  // assignments per dispatch chunk (target)
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -166,6 +169,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         static_cast<size_t>(d) * h->e_pad * 4,  // router_wt
         N * 4,                                // rinv
         E * static_cast<size_t>(d) * 4,       // router_wg
+        (E + 1) * 4,                          // sched
         256,                                  // status
     };
     const int nblocks = sizeof(sizes) / sizeof(sizes[0]);
@@ -194,7 +198,8 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->router_wt = reinterpret_cast<float *>(b + off[13]);
     h->rinv = reinterpret_cast<float *>(b + off[14]);
     h->router_wg = reinterpret_cast<float *>(b + off[15]);
-    h->status = reinterpret_cast<int *>(b + off[16]);
+    h->sched = reinterpret_cast<int32_t *>(b + off[16]);
+    h->status = reinterpret_cast<int *>(b + off[17]);
     if (cudaMemset(h->ws, 0, total) != cudaSuccess) {
         cudaFree(h->ws);
         delete h;
@@ -210,6 +215,9 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     if (h->use_tc) {
         rc = tc_build_maps(&h->maps, h->xp, h->act, w->w_gate_up, w->w_down, h->rows_cap,
                            n_experts, d, d_ff);
+        if (rc == MOE_OK)
+            rc = decode_build_maps(&h->decode_maps, h->xp, h->act, w->w_gate_up, w->w_down,
+                                   h->rows_cap, n_experts, d, d_ff);
         if (rc != MOE_OK) {
             cudaFree(h->ws);
             delete h;
@@ -218,6 +226,15 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     }
     *out = h;
     return MOE_OK;
+}
+
+// The fused small-batch expert kernel (both contractions in one persistent
+// launch) serves bf16 layers while the mean load stays at or below
+// kDecodeRowsPerExpert grouped rows per expert; larger batches use the two
+// row-tiled grouped GEMMs.
+static bool use_fused_experts(const moe_ctx *h, int N) {
+    return h->use_tc && static_cast<long long>(N) * h->k <=
+                            static_cast<long long>(kDecodeRowsPerExpert) * h->E;
 }
 
 // Adds the durations of up to `count` (all if < 0) recorded forwards, oldest
@@ -285,6 +302,9 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     dp.N = N; dp.d = h->d; dp.E = h->E; dp.k = h->k; dp.nchunk = nchunk;
     dp.chunk_tokens = chunk_tokens; dp.tile_m = tile_m;
     dp.elem_bytes = static_cast<int>(h->elem);
+    const bool fused = use_fused_experts(h, N);
+    dp.sched = fused ? h->sched : nullptr;
+    dp.sched_n = h->E + 1;
     // several CTAs per chunk share the row copies: about four CTAs per SM in all
     dp.replicas = (4 * h->n_sm + nchunk - 1) / nchunk;
     if (dp.replicas > 64) dp.replicas = 64;
@@ -296,19 +316,27 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     gp.E = h->E; gp.d = h->d; gp.I = h->I; gp.k = h->k; gp.rows_cap = h->rows_cap;
     const int max_mtiles = (N * h->k + tile_m - 1) / tile_m + h->E;
 
-    gp.a = h->xp; gp.w = h->w.w_gate_up; gp.c = h->act;
-    if (h->use_tc)
-        MOE_TRY(launch_gemm_tc_gate_up(h->maps, gp, h->n_sm, s));
-    else
-        MOE_TRY(launch_gemm_simt_gate_up(gp, max_mtiles, s));
-    MOE_MARK();
+    if (fused) {
+        DecodeParams fp;
+        fp.offsets = h->offsets; fp.act = h->act; fp.y = h->y; fp.sched = h->sched;
+        fp.status = h->status; fp.E = h->E; fp.d = h->d; fp.I = h->I;
+        MOE_TRY(launch_decode_experts(h->decode_maps, fp, h->n_sm, s));
+        MOE_MARK();
+    } else {
+        gp.a = h->xp; gp.w = h->w.w_gate_up; gp.c = h->act;
+        if (h->use_tc)
+            MOE_TRY(launch_gemm_tc_gate_up(h->maps, gp, h->n_sm, s));
+        else
+            MOE_TRY(launch_gemm_simt_gate_up(gp, max_mtiles, s));
+        MOE_MARK();
 
-    gp.a = h->act; gp.w = h->w.w_down; gp.c = h->y;
-    if (h->use_tc)
-        MOE_TRY(launch_gemm_tc_down(h->maps, gp, h->n_sm, s));
-    else
-        MOE_TRY(launch_gemm_simt_down(gp, max_mtiles, s));
-    MOE_MARK();
+        gp.a = h->act; gp.w = h->w.w_down; gp.c = h->y;
+        if (h->use_tc)
+            MOE_TRY(launch_gemm_tc_down(h->maps, gp, h->n_sm, s));
+        else
+            MOE_TRY(launch_gemm_simt_down(gp, max_mtiles, s));
+        MOE_MARK();
+    }
 
     CombineParams cp;
     cp.x = x; cp.y = h->y; cp.wts = h->wts; cp.inv = h->inv; cp.out = out; cp.status = h->status;
@@ -323,6 +351,7 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
         h->head++;
     }
     h->last_n = N;
+    h->last_fused = fused;
     return MOE_OK;
 }
 
@@ -366,6 +395,7 @@ extern "C" int moe_destroy(moe_ctx *h) {
     int rc = MOE_OK;
     if (cudaDeviceSynchronize() != cudaSuccess) rc = MOE_ERR_CUDA;
     free_ring(h);
+    if (h->decode_maps) decode_free_maps(h->decode_maps);
     if (cudaFree(h->ws) != cudaSuccess) rc = MOE_ERR_CUDA;
     delete h;
     return rc;
@@ -407,6 +437,7 @@ extern "C" int moe_profile(moe_ctx *h, int enable) {
             if (cudaEventCreate(&h->ring[i]) != cudaSuccess) {
                 h->ring.resize(i);
                 free_ring(h);
+    if (h->decode_maps) decode_free_maps(h->decode_maps);
                 return MOE_ERR_CUDA;
             }
         }
@@ -428,14 +459,15 @@ extern "C" int moe_kernel_times(moe_ctx *h, float *ms, int n) {
 }
 
 extern "C" const char *moe_kernel_name(moe_ctx *h, int i) {
-    (void)h;
-    if (i < 0 || i >= kLaunches) return nullptr;
-    return kKernelNames[i];
+    if (!h) return nullptr;
+    if (h->last_fused) return (i >= 0 && i < 4) ? kFusedKernelNames[i] : nullptr;
+    return (i >= 0 && i < 5) ? kKernelNames[i] : nullptr;
 }
 
 extern "C" int moe_launches_per_forward(moe_ctx *h, int n_tokens) {
     if (!h) return MOE_ERR_INVALID_ARG;
-    return n_tokens > 0 ? kLaunches : 0;
+    if (n_tokens <= 0) return 0;
+    return use_fused_experts(h, n_tokens) ? 4 : 5;
 }
 
 extern "C" int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream) {

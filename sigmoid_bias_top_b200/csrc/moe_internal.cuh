@@ -59,8 +59,9 @@ struct DispatchParams {
     int32_t *mt_start;         // [E+1] prefix of per-expert row tiles (tile rows = tile_m)
     int32_t *perm;             // [N*k] grouped row -> assignment t*k+j
     int32_t *inv;              // [N*k] assignment -> grouped row
+    int32_t *sched;            // [sched_n] cleared for the fused small-batch expert kernel
     int *status;
-    int N, d, E, k, nchunk, chunk_tokens, tile_m, replicas, elem_bytes;
+    int N, d, E, k, nchunk, chunk_tokens, tile_m, replicas, elem_bytes, sched_n;
 };
 
 struct CombineParams {
@@ -85,6 +86,16 @@ struct GroupedParams {
     int *status;
     int E, d, I, k;
     int rows_cap;             // allocated grouped rows (act, y)
+};
+
+struct DecodeParams {
+    // the fused small-batch expert kernel (gate/up and down in one launch)
+    const int32_t *offsets;   // [E+1]
+    void *act;                // [rows][I] written by gate/up items, read by down items
+    void *y;                  // [rows][d]
+    int32_t *sched;           // [1 + E]: claimed-item counter, per-expert finished gate/up items
+    int *status;
+    int E, d, I;
 };
 
 // ---------------------------------------------------------------------------
@@ -115,6 +126,11 @@ int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, c
 int launch_gemm_tc_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_gemm_tc_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_selftest_timeout(int *status, int timeout_us, cudaStream_t s);
+constexpr int kDecodeRowsPerExpert = 32;  // the fused kernel is used up to this mean load
+int decode_build_maps(void **holder, const void *xp, const void *act, const void *wgu,
+                      const void *wd, int rows_cap, int E, int d, int I);
+void decode_free_maps(void *holder);
+int launch_decode_experts(const void *holder, const DecodeParams &p, int n_sm, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Launch with programmatic dependent launch: the kernel may be scheduled while
