@@ -16,10 +16,11 @@
 // products: l_e = rinv * sum_j x_j W'_ej, the same value as W_r[e] . xn up to
 // fp32 rounding, with no per-element scaling in the inner loops.
 //   small batches: a cluster of 8 CTAs per group of TT tokens; CTA r stages
-//     its E/8 rows of W' in shared memory (one bulk copy, in flight while the
-//     1/rms factors are computed) and computes their logits (lanes split d,
-//     warp reduction); the logits go to CTA 0 through distributed shared
-//     memory, which then selects and normalises;
+//     its E/8 rows of W' and the group's rows of x in shared memory (bulk
+//     copies) and computes their logits with its 8 warps tiled over (tokens x
+//     experts), lanes splitting d, in one pass that also sums the squares;
+//     the logits go to CTA 0 through distributed shared memory, which then
+//     selects and normalises;
 //   large batches: one CTA per 32 tokens computes the 32 x 64 logit tile as a
 //     register-tiled SGEMM over d (4 x 4 outputs per thread, double-buffered
 //     shared-memory chunks of x and of W' transposed to [d][E]); its two
@@ -98,66 +99,72 @@ __device__ __forceinline__ float row_rinv(const T *xr, int d, float eps, int lan
     return 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
 }
 
+// Order-preserving integer image of a float (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Selection and weights of one token by one warp. srow[E] holds its logits
 // (overwritten with the sigmoid scores); the result goes to idx/wts row t and
-// the expert counts to hist (shared).
-__device__ __forceinline__ void select_token(const RouteParams &p, float *srow, size_t t,
-                                             int *hist, int lane) {
+// the expert counts to hist (shared). Each round takes the largest biased
+// score (warp max of its integer image), then the lowest expert index among
+// the lanes holding it: exact fp32 top-k with ties to the lower index.
+__device__ __forceinline__ void select_token(const RouteParams &p, float *srow,
+                                             const float *bias_s, size_t t, int *hist, int lane) {
     const int E = p.E, k = p.k;
-    float c_reg[kMaxExperts / 32];
-    uint32_t taken = 0;  // bit i: expert lane + 32 i is unavailable
+    const int epl = (E + 31) / 32;  // experts per lane
+    uint32_t key[kMaxExperts / 32];
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
         const int e = lane + 32 * i;
-        c_reg[i] = -INFINITY;
-        if (e < E) {
+        key[i] = 0u;  // below every real key: never selected
+        if (i < epl && e < E) {
             const float s = 1.0f / (1.0f + expf(-srow[e]));
-            const float c = s + p.bias[e];
-            c_reg[i] = (c == c) ? c : -INFINITY;  // a NaN score never wins
+            const float c = s + bias_s[e];
+            key[i] = (c == c) ? float_key(c) : 1u;  // a NaN score ranks below every number
             srow[e] = s;  // each lane rewrites only its own experts
-        } else {
-            taken |= 1u << i;
         }
     }
     __syncwarp();
     int sel[kMaxTopK];
     float ssel[kMaxTopK];
-    for (int j = 0; j < k; ++j) {
-        float bc = -INFINITY;
-        int be = 0x7fffffff;
+    float sum = 0.f;
 #pragma unroll
-        for (int i = 0; i < kMaxExperts / 32; ++i) {
-            // ascending expert index within a lane: ties keep the lower index
-            if (!(taken & (1u << i)) && (c_reg[i] > bc || be == 0x7fffffff)) {
-                bc = c_reg[i];
-                be = lane + 32 * i;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (oe != 0x7fffffff && (be == 0x7fffffff || oc > bc || (oc == bc && oe < be))) {
-                bc = oc;
-                be = oe;
-            }
-        }
-        // k <= E guarantees an untaken expert exists, so be < E here
-        sel[j] = be;
-        ssel[j] = srow[be];
+    for (int j = 0; j < kMaxTopK; ++j) {
+        if (j >= k) break;
+        uint32_t bk = 0u;
+        int bi = 0;
 #pragma unroll
         for (int i = 0; i < kMaxExperts / 32; ++i)
-            if (lane + 32 * i == be) taken |= 1u << i;
+            if (key[i] > bk) {  // ascending expert index: ties keep the lower one
+                bk = key[i];
+                bi = i;
+            }
+        const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t cand = (bk == top && top != 0u) ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu;
+        const uint32_t e = __reduce_min_sync(0xffffffffu, cand);
+        // k <= E: an unselected expert exists, so e < E here
+#pragma unroll
+        for (int i = 0; i < kMaxExperts / 32; ++i)
+            if (static_cast<uint32_t>(lane + 32 * i) == e) key[i] = 0u;
+        sel[j] = static_cast<int>(e);
+        ssel[j] = srow[e];
+        sum += ssel[j];
     }
-    if (lane == 0) {
-        float sum = 0.f;
-        for (int j = 0; j < k; ++j) sum += ssel[j];
+    if (lane < k) {  // lane j writes slot j
         const float den = sum + p.eps;
-        for (int j = 0; j < k; ++j) {
-            p.idx[t * k + j] = sel[j];
-            p.wts[t * k + j] = p.scale * (ssel[j] / den);
-            atomicAdd(&hist[sel[j]], 1);
-        }
+        float sj = 0.f;
+        int ej = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+            if (j == lane) {
+                sj = ssel[j];
+                ej = sel[j];
+            }
+        p.idx[t * k + lane] = ej;
+        p.wts[t * k + lane] = p.scale * (sj / den);
+        atomicAdd(&hist[ej], 1);
     }
 }
 
@@ -174,69 +181,101 @@ __device__ __forceinline__ void flush_hist(const RouteParams &p, const int *hist
 constexpr int kSmallThreads = 256;
 constexpr int kClusterCtas = 8;
 
-template <typename T, int TPW, int EG>
+template <typename T, int TT, int EG>
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kSmallThreads)
     route_small_kernel(RouteParams p) {
-    constexpr int TT = 8 * TPW;  // tokens per cluster
+    // TT tokens per cluster, EG experts per CTA, 8 warps tiled WT x WE
+    constexpr int WE = EG < 4 ? EG : 4;   // warps along the experts
+    constexpr int WT = 8 / WE;            // warps along the tokens
+    constexpr int EPW = EG / WE;          // experts per warp
+    constexpr int TPW = TT / WT;          // tokens per warp
     extern __shared__ float4 smem_f4[];
     float *wsl = reinterpret_cast<float *>(smem_f4);  // [EG][d] router rows times gain
-    float *sc = wsl + EG * p.d;                       // [TT][E] (used in CTA 0)
-    int *hist = reinterpret_cast<int *>(sc + TT * p.E);
+    T *xs = reinterpret_cast<T *>(wsl + EG * p.d);    // [TT][d] this group's rows of x
+    float *sc = reinterpret_cast<float *>(
+        reinterpret_cast<uint8_t *>(xs) + ((static_cast<size_t>(TT) * p.d * sizeof(T) + 15) & ~size_t(15)));
+    float *bias_s = sc + TT * p.E;                    // [E]
+    float *rinv_s = bias_s + p.E;                     // [TT]
+    int *hist = reinterpret_cast<int *>(rinv_s + TT);  // [E]
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
     const int d = p.d, E = p.E;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = (blockIdx.x / kClusterCtas) * TT;
+    const int ntok = min(TT, p.N - t0);
     const int e0 = rank * EG;
 
-    // router rows of this CTA -> shared memory, one bulk copy in flight while
-    // the normalisation factors are computed
-    __shared__ uint64_t wbar;
+    // layer parameters first (no earlier kernel writes them): the router rows
+    // by one bulk copy, the bias into shared memory
+    __shared__ uint64_t wbar, xbar;
     if (threadIdx.x == 0) {
         mbar_init(&wbar, 1);
+        mbar_init(&xbar, 1);
         fence_mbar_init();
     }
     __syncthreads();
     const uint32_t wbytes = static_cast<uint32_t>(EG) * d * 4;
-    if (threadIdx.x == 0) {  // the router copy depends on no earlier kernel
+    if (threadIdx.x == 0) {
         const float *src = p.router_wg + static_cast<size_t>(e0) * d;
         mbar_arrive_expect_tx(&wbar, wbytes);
         for (uint32_t off = 0; off < wbytes; off += 32768u)
             bulk_copy_g2s(wsl + off / 4, src + off / 4, min(32768u, wbytes - off), &wbar);
     }
-    for (int e = threadIdx.x; e < E; e += kSmallThreads) hist[e] = 0;
+    for (int e = threadIdx.x; e < E; e += kSmallThreads) {
+        hist[e] = 0;
+        bias_s[e] = p.bias[e];
+    }
     pdl_trigger();
     pdl_wait();
+    // this group's rows of x (consecutive tokens) by one bulk copy
+    const uint32_t xbytes = static_cast<uint32_t>(ntok) * d * sizeof(T);
+    if (threadIdx.x == 0) {
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(static_cast<const T *>(p.x) +
+                                                               static_cast<size_t>(t0) * d);
+        mbar_arrive_expect_tx(&xbar, xbytes);
+        for (uint32_t off = 0; off < xbytes; off += 32768u)
+            bulk_copy_g2s(reinterpret_cast<uint8_t *>(xs) + off, src + off,
+                          min(32768u, xbytes - off), &xbar);
+    }
+    const uint64_t dl = globaltimer_ns() + 1000000000ull;
+    if (!mbar_wait(&wbar, 0, dl) || !mbar_wait(&xbar, 0, dl)) set_status(p.status, kStatusTimeout);
 
-    // normalisation factors of this warp's tokens
-    float rinv[TPW];
+    // warps tile (token groups x expert groups): warp = wt * WE + we takes
+    // tokens [wt*TPW, +TPW) and experts [we*EPW, +EPW) of this CTA, so each
+    // row of x and of W' read from shared memory feeds several outputs.
+    // Lanes take 4 columns of each 128-column chunk.
+    const int we = warp % WE, wt = warp / WE;
     const T *xr[TPW];
 #pragma unroll
     for (int i = 0; i < TPW; ++i) {
-        const int t = t0 + warp * TPW + i;
-        const bool valid = t < p.N;
-        xr[i] = static_cast<const T *>(p.x) + static_cast<size_t>(valid ? t : 0) * d;
-        rinv[i] = valid ? row_rinv<T>(xr[i], d, p.eps, lane) : 0.f;
-        if (valid && rank == 0 && lane == 0) p.rinv[t] = rinv[i];
+        const int tl = wt * TPW + i;
+        xr[i] = xs + static_cast<size_t>(tl < ntok ? tl : 0) * d;
     }
-    if (!mbar_wait(&wbar, 0, globaltimer_ns() + 1000000000ull)) set_status(p.status, kStatusTimeout);
-    __syncthreads();
-
-    // acc[e][i] = sum_j x[t_i][j] * (W_r[e][j] * gain[j]); the logit is rinv * acc
-    float acc[EG][TPW];
+    const float *wr = wsl + static_cast<size_t>(we * EPW) * d;
+    float acc[EPW][TPW], ss[TPW];
 #pragma unroll
-    for (int e = 0; e < EG; ++e)
+    for (int i = 0; i < TPW; ++i) {
+        ss[i] = 0.f;
 #pragma unroll
-        for (int i = 0; i < TPW; ++i) acc[e][i] = 0.f;
+        for (int e = 0; e < EPW; ++e) acc[e][i] = 0.f;
+    }
 #pragma unroll 4
     for (int j = lane * 4; j < d; j += 128) {
         float4 xv[TPW];
 #pragma unroll
-        for (int i = 0; i < TPW; ++i) xv[i] = Vec4<T>::load(xr[i] + j);
+        for (int i = 0; i < TPW; ++i) {
+            xv[i] = Vec4<T>::load(xr[i] + j);
+            if (we == 0) {  // the first expert group also sums the squares
+                ss[i] += xv[i].x * xv[i].x;
+                ss[i] += xv[i].y * xv[i].y;
+                ss[i] += xv[i].z * xv[i].z;
+                ss[i] += xv[i].w * xv[i].w;
+            }
+        }
 #pragma unroll
-        for (int e = 0; e < EG; ++e) {
-            const float4 w = *reinterpret_cast<const float4 *>(wsl + e * d + j);
+        for (int e = 0; e < EPW; ++e) {
+            const float4 w = *reinterpret_cast<const float4 *>(wr + e * d + j);
 #pragma unroll
             for (int i = 0; i < TPW; ++i) {
                 float a = acc[e][i];
@@ -248,20 +287,33 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kSmallThr
             }
         }
     }
-    float *sc0 = cluster.map_shared_rank(sc, 0);
-#pragma unroll
-    for (int e = 0; e < EG; ++e)
+    if (we == 0) {
 #pragma unroll
         for (int i = 0; i < TPW; ++i) {
-            const float v = warp_sum(acc[e][i]) * rinv[i];
-            if (lane == 0) sc0[(warp * TPW + i) * E + e0 + e] = v;
+            const int tl = wt * TPW + i;
+            const float tot = warp_sum(ss[i]);
+            if (lane == 0) {
+                const float r = tl < ntok ? 1.0f / sqrtf(tot / static_cast<float>(d) + p.eps) : 0.f;
+                rinv_s[tl] = r;
+                if (tl < ntok && rank == 0) p.rinv[t0 + tl] = r;
+            }
+        }
+    }
+    __syncthreads();
+    float *sc0 = cluster.map_shared_rank(sc, 0);
+#pragma unroll
+    for (int e = 0; e < EPW; ++e)
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+            const int tl = wt * TPW + i;
+            const float v = warp_sum(acc[e][i]) * rinv_s[tl];
+            if (lane == 0) sc0[tl * E + e0 + we * EPW + e] = v;
         }
     cluster.sync();
     if (rank != 0) return;
 
-    const int ntok = min(TT, p.N - t0);
     for (int tl = warp; tl < ntok; tl += kSmallThreads / 32)
-        select_token(p, sc + tl * E, static_cast<size_t>(t0 + tl), hist, lane);
+        select_token(p, sc + tl * E, bias_s, static_cast<size_t>(t0 + tl), hist, lane);
     __syncthreads();
     flush_hist(p, hist, t0);
 }
@@ -279,7 +331,7 @@ constexpr int kGroupThreads = 128;
 
 size_t large_smem(int E) {
     return (2 * 2 * LKC * LXS + 2 * 2 * LKC * 64 + LT * 64 + LT * static_cast<size_t>(E) + LT) * 4 +
-           static_cast<size_t>(E) * 4;
+           2 * static_cast<size_t>(E) * 4;
 }
 
 template <typename T>
@@ -290,14 +342,18 @@ __global__ void __launch_bounds__(kLargeThreads) route_large_kernel(RouteParams 
     float *red = ws_all + 2 * 2 * LKC * 64;                    // [LT][64] second half's sums
     float *sc = red + LT * 64;                                 // [LT][E]
     float *rinv_s = sc + LT * p.E;                             // [LT]
-    int *hist = reinterpret_cast<int *>(rinv_s + LT);          // [E]
+    float *bias_s = rinv_s + LT;                               // [E]
+    int *hist = reinterpret_cast<int *>(bias_s + p.E);         // [E]
 
     const int d = p.d, E = p.E, Ep = p.e_pad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int grp = tid / kGroupThreads, gt = tid % kGroupThreads;
     const int t0 = blockIdx.x * LT;
     const int ntok = min(LT, p.N - t0);
-    for (int e = tid; e < E; e += kLargeThreads) hist[e] = 0;
+    for (int e = tid; e < E; e += kLargeThreads) {
+        hist[e] = 0;
+        bias_s[e] = p.bias[e];
+    }
     pdl_trigger();
     pdl_wait();
     for (int tl = warp; tl < LT; tl += kLargeThreads / 32) {
@@ -398,31 +454,34 @@ __global__ void __launch_bounds__(kLargeThreads) route_large_kernel(RouteParams 
     }
 
     for (int tl = warp; tl < ntok; tl += kLargeThreads / 32)
-        select_token(p, sc + tl * E, static_cast<size_t>(t0 + tl), hist, lane);
+        select_token(p, sc + tl * E, bias_s, static_cast<size_t>(t0 + tl), hist, lane);
     __syncthreads();
     flush_hist(p, hist, t0);
 }
 
 
-template <typename T, int TPW, int EG>
+size_t small_smem(int EG, int TT, int d, int E, int elem) {
+    return static_cast<size_t>(EG) * d * 4 + ((static_cast<size_t>(TT) * d * elem + 15) & ~size_t(15)) +
+           (static_cast<size_t>(TT) * E + 2 * static_cast<size_t>(E) + TT) * 4;
+}
+
+template <typename T, int TT, int EG>
 int launch_small(const RouteParams &p, cudaStream_t s) {
-    constexpr int TT = 8 * TPW;
     const int groups = (p.N + TT - 1) / TT;
-    const size_t smem = (static_cast<size_t>(EG) * p.d + static_cast<size_t>(TT) * p.E) * 4 +
-                        static_cast<size_t>(p.E) * 4;
-    auto kern = route_small_kernel<T, TPW, EG>;
+    const size_t smem = small_smem(EG, TT, p.d, p.E, sizeof(T));
+    auto kern = route_small_kernel<T, TT, EG>;
     if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
     return launch_k(kern, dim3(groups * kClusterCtas), dim3(kSmallThreads), smem, s, p);
 }
 
-template <typename T, int TPW>
+template <typename T, int TT>
 int launch_small_eg(const RouteParams &p, cudaStream_t s) {
     switch (p.E / kClusterCtas) {
-        case 1: return launch_small<T, TPW, 1>(p, s);
-        case 2: return launch_small<T, TPW, 2>(p, s);
-        case 4: return launch_small<T, TPW, 4>(p, s);
-        case 8: return launch_small<T, TPW, 8>(p, s);
-        case 16: return launch_small<T, TPW, 16>(p, s);
+        case 1: return launch_small<T, TT, 1>(p, s);
+        case 2: return launch_small<T, TT, 2>(p, s);
+        case 4: return launch_small<T, TT, 4>(p, s);
+        case 8: return launch_small<T, TT, 8>(p, s);
+        case 16: return launch_small<T, TT, 16>(p, s);
         default: return MOE_ERR_INVALID_ARG;
     }
 }
@@ -430,9 +489,9 @@ int launch_small_eg(const RouteParams &p, cudaStream_t s) {
 template <typename T>
 int launch_small_t(const RouteParams &p, int tt, cudaStream_t s) {
     switch (tt) {
-        case 8: return launch_small_eg<T, 1>(p, s);
-        case 16: return launch_small_eg<T, 2>(p, s);
-        case 32: return launch_small_eg<T, 4>(p, s);
+        case 8: return launch_small_eg<T, 8>(p, s);
+        case 16: return launch_small_eg<T, 16>(p, s);
+        case 32: return launch_small_eg<T, 32>(p, s);
         default: return MOE_ERR_INVALID_ARG;
     }
 }
@@ -471,14 +530,17 @@ bool route_small_ok(int d, int E) {
     if (E % kClusterCtas != 0) return false;
     const int eg = E / kClusterCtas;
     if (eg != 1 && eg != 2 && eg != 4 && eg != 8 && eg != 16) return false;
-    return static_cast<size_t>(eg) * d * 4 + 32 * static_cast<size_t>(E) * 4 <= 160 * 1024;
+    return small_smem(eg, 8, d, E, 4) <= 200 * 1024;  // at least the 8-token groups fit
 }
 
 int route_plan(int N, int d, int E, int *toks_per_group) {
     // the cluster kernel while its groups give fewer CTAs than the tiled
-    // kernel would need to fill the GPU twice; the tiled kernel beyond
+    // kernel would need to fill the GPU twice; the tiled kernel beyond. The
+    // group shrinks until its router rows and token rows fit in shared memory.
     if (route_small_ok(d, E) && N < 4096) {
-        *toks_per_group = N <= 64 ? 8 : N <= 256 ? 16 : 32;
+        int tt = N <= 64 ? 8 : N <= 256 ? 16 : 32;
+        while (tt > 8 && small_smem(E / kClusterCtas, tt, d, E, 4) > 200 * 1024) tt /= 2;
+        *toks_per_group = tt;
         return kRouteSmall;
     }
     *toks_per_group = LT;
