@@ -237,3 +237,10 @@ def test_both_expert_paths_agree():
     torch.cuda.synchronize()
     rel = (o_big.float() - o_small.float()).norm(dim=1) / o_small.float().norm(dim=1)
     assert rel.max().item() < 1e-2
+
+
+def test_fp32_large_batch_tiled_router():
+    """A large fp32 batch (ragged N) goes through the d-split cluster router."""
+    w = W.TINY_F32.scaled(n_tokens=4100)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r, tokens="sample")
