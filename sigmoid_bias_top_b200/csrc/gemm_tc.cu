@@ -391,6 +391,8 @@ int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, c
     if ((rc = encode_2d(&m->a_down, act, rows_cap, I, BM)) != MOE_OK) return rc;
     if ((rc = encode_2d(&m->w_down, wd, static_cast<uint64_t>(E) * d, I, BN)) != MOE_OK)
         return rc;
+    if ((rc = encode_2d(&m->w_down_half, wd, static_cast<uint64_t>(E) * d, I, BN / 2)) != MOE_OK)
+        return rc;
     return MOE_OK;
 }
 

@@ -6,9 +6,13 @@
 //   1 route     RMSNorm + fp32 router + sigmoid + biased top-k + weights, and the
 //               per-chunk expert histogram
 //   2 dispatch  per-expert counts, offsets, row-tile prefix, perm / inv
-//   3 gate_up   grouped GEMM over rows gathered through perm, SiLU(gate)*up
-//               (tcgen05 for bf16, SIMT for fp32)
+//   3 gate_up   grouped GEMM over the grouped normalised rows, SiLU(gate)*up
+//               (tcgen05 for bf16: 128-row tiles on single CTAs, or 256-row
+//               tiles on CTA pairs once the mean load reaches 256 rows per
+//               expert; SIMT for fp32)
 //   4 down      grouped GEMM
+// (bf16 batches of at most 32 rows per expert on average fuse 3 and 4 into one
+// persistent kernel.)
 //   5 combine   out = x + sum_j w_j y_j in fixed slot order
 #include <stdio.h>
 #include <stdlib.h>
@@ -44,6 +48,7 @@ struct moe_ctx {
     void *decode_maps;   // tensor maps of the fused small-batch kernel
     int32_t *sched;      // [1 + E] its work counter and per-expert completion counts
     bool use_tc;
+    int pair_mode;       // CTA-pair GEMMs: -1 by load, 0 never, 1 whenever not fused
 
     int last_n;
     bool last_fused;  // the last forward used the fused small-batch expert kernel
@@ -146,6 +151,12 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->elem = (w->dtype == MOE_F32) ? 4 : 2;
     h->use_tc = (w->dtype == MOE_BF16);
     h->rows_cap = max_tokens * top_k;
+    {
+        // MOE_TC_PAIR=0 / 1 overrides the choice between the single-CTA and
+        // the CTA-pair grouped GEMMs (both compute the same result).
+        const char *e = getenv("MOE_TC_PAIR");
+        h->pair_mode = (e && e[0] == '0') ? 0 : (e && e[0] == '1') ? 1 : -1;
+    }
 
     h->e_pad = (n_experts + 63) / 64 * 64;
     h->max_chunks = 16384 / n_experts < 256 ? 16384 / n_experts : 256;
@@ -237,6 +248,15 @@ static bool use_fused_experts(const moe_ctx *h, int N) {
                             static_cast<long long>(kDecodeRowsPerExpert) * h->E;
 }
 
+// Row-tiled bf16 GEMMs on CTA pairs (256-row tiles) once the mean load fills
+// a pair tile; below that the padding of 256-row tiles costs more than the
+// halved operand traffic per MMA saves.
+static bool use_pair_gemms(const moe_ctx *h, int N) {
+    if (!h->use_tc || h->pair_mode == 0) return false;
+    if (h->pair_mode == 1) return true;
+    return static_cast<long long>(N) * h->k >= static_cast<long long>(kTcPairTileM) * h->E;
+}
+
 // Adds the durations of up to `count` (all if < 0) recorded forwards, oldest
 // first, to the per-kernel sums.
 static int accumulate(moe_ctx *h, long long count) {
@@ -282,7 +302,9 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     const int kind = route_plan(N, h->d, h->E, &tt);
     int nchunk = 1, chunk_tokens = N;
     chunk_plan(N, h->k, h->max_chunks, &nchunk, &chunk_tokens);
-    const int tile_m = h->use_tc ? kTcTileM : kSimtTileM;
+    const bool fused = use_fused_experts(h, N);
+    const bool pair = !fused && use_pair_gemms(h, N);
+    const int tile_m = !h->use_tc ? kSimtTileM : pair ? kTcPairTileM : kTcTileM;
 
     MOE_MARK();
     RouteParams rp;
@@ -302,7 +324,6 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     dp.N = N; dp.d = h->d; dp.E = h->E; dp.k = h->k; dp.nchunk = nchunk;
     dp.chunk_tokens = chunk_tokens; dp.tile_m = tile_m;
     dp.elem_bytes = static_cast<int>(h->elem);
-    const bool fused = use_fused_experts(h, N);
     dp.sched = fused ? h->sched : nullptr;
     dp.sched_n = h->E + 1;
     // several CTAs per chunk share the row copies: about four CTAs per SM in all
@@ -324,14 +345,18 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
         MOE_MARK();
     } else {
         gp.a = h->xp; gp.w = h->w.w_gate_up; gp.c = h->act;
-        if (h->use_tc)
+        if (pair)
+            MOE_TRY(launch_gemm_tc2_gate_up(h->maps, gp, h->n_sm, s));
+        else if (h->use_tc)
             MOE_TRY(launch_gemm_tc_gate_up(h->maps, gp, h->n_sm, s));
         else
             MOE_TRY(launch_gemm_simt_gate_up(gp, max_mtiles, s));
         MOE_MARK();
 
         gp.a = h->act; gp.w = h->w.w_down; gp.c = h->y;
-        if (h->use_tc)
+        if (pair)
+            MOE_TRY(launch_gemm_tc2_down(h->maps, gp, h->n_sm, s));
+        else if (h->use_tc)
             MOE_TRY(launch_gemm_tc_down(h->maps, gp, h->n_sm, s));
         else
             MOE_TRY(launch_gemm_simt_down(gp, max_mtiles, s));

@@ -120,12 +120,17 @@ struct TcMaps {
     CUtensorMap w_gate_up;  // W   [E*2I][d],     box 64 x 128
     CUtensorMap a_down;     // act [rows][I],     box 64 x 128
     CUtensorMap w_down;     // Wd  [E*d][I],      box 64 x 256
+    CUtensorMap w_down_half;  // Wd [E*d][I],     box 64 x 128 (CTA-pair kernels)
 };
 int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, const void *wd,
                   int rows_cap, int E, int d, int I);
 int launch_gemm_tc_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_gemm_tc_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_selftest_timeout(int *status, int timeout_us, cudaStream_t s);
+// The same contractions on CTA pairs (256-row tiles, grouped with tile_m 256).
+constexpr int kTcPairTileM = 256;
+int launch_gemm_tc2_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
+int launch_gemm_tc2_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 constexpr int kDecodeRowsPerExpert = 32;  // the fused kernel is used up to this mean load
 int decode_build_maps(void **holder, const void *xp, const void *act, const void *wgu,
                       const void *wd, int rows_cap, int E, int d, int I);
