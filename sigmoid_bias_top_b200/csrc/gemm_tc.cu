@@ -371,6 +371,28 @@ int encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// 4-D bf16 view of the packed gate/up matrix [E*2I][d] for the CTA-pair
+// kernel: element (k, y, z, g) = row 16 g + y + z I, column k, i.e. 16-row
+// group g of the gate block (z = 0) or the up row I further (z = 1). Groups
+// run up to E*2I - I rows, so every addressed row lies inside the matrix; a
+// box of {64, 16, 2, 4} lands in shared memory as 16 gate rows, the matching
+// 16 up rows, the next 16 gate rows, ... (128 rows, 128-byte swizzle).
+int encode_gate_up_4d(CUtensorMap *m, const void *base, int E, int d, int I) {
+    EncodeTiledFn enc = get_encoder();
+    if (!enc) return MOE_ERR_CUDA;
+    const uint64_t groups = (static_cast<uint64_t>(E) * 2 * I - I) / 16;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), 16, 2, groups};
+    const cuuint64_t row = static_cast<cuuint64_t>(d) * 2;
+    const cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(I), row * 16};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(BK), 16, 2, 4};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 template <bool GATE_UP>
 int launch(const CUtensorMap &a, const CUtensorMap &b, const GroupedParams &p, int n_sm,
            cudaStream_t s) {
@@ -391,6 +413,8 @@ int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, c
     if ((rc = encode_2d(&m->a_down, act, rows_cap, I, BM)) != MOE_OK) return rc;
     if ((rc = encode_2d(&m->w_down, wd, static_cast<uint64_t>(E) * d, I, BN)) != MOE_OK)
         return rc;
+    if (I % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((rc = encode_gate_up_4d(&m->w_gate_up_4d, wgu, E, d, I)) != MOE_OK) return rc;
     if ((rc = encode_2d(&m->w_down_half, wd, static_cast<uint64_t>(E) * d, I, BN / 2)) != MOE_OK)
         return rc;
     return MOE_OK;

@@ -1,28 +1,40 @@
-// gemm_tc2.cu -- the row-tiled grouped expert GEMMs on CTA pairs
-// (tcgen05.mma.cta_group::2): one MMA computes a 256-row x 256-column tile.
+// gemm_tc2.cu -- the grouped expert GEMMs of large batches on CTA pairs
+// (tcgen05.mma.cta_group::2), with the weights as the 256-row MMA operand and
+// the tokens as the N operand ("swap AB").
 //
 // The gated SiLU expert of "LFM2.5-24B-A2B: Biased Routing, Short Convolutions
 // and Ten KV Caches" (flozi.net, English page, section "The router has two
 // different scores") over the rows grouped by expert (section "What to verify
-// in a deployment"), for batches with many rows per expert:
+// in a deployment"):
 //   gate/up: act[r][f] = silu(xp[r] . Wg_e[f]) * (xp[r] . Wu_e[f])
 //   down:    y[r][n]   = act[r] . Wd_e[n]
-// A cluster of two CTAs shares each tile: CTA r of the pair stages 128 rows of
-// the A operand (its half of M) and 128 rows of the B operand (its half of N:
-// for gate/up the leader holds the gate rows and the peer the matching up
-// rows, so accumulator columns 0..127 are gate and 128..255 up in both CTAs'
-// TMEM). Per CTA a stage is 32 KB (A 16 KB + B 16 KB) instead of 48 KB for a
-// 128 x 256 single-CTA tile, which cuts the L2-to-SM traffic per MMA by a
-// third, and 6 stages fit.
-//
+// computed transposed, D[feature][token] = W_e[feature] . a[token]:
+//   * M = 256 weight rows per tile, 128 in each CTA of the pair. gate/up: a
+//     pair tile covers 128 features; CTA h stages the gate and up rows of
+//     features f0+64h..+63 interleaved in groups of 16 (16 gate rows, the 16
+//     matching up rows, ...) by one 4-D TMA box, so TMEM lanes l and l+16 of
+//     every 32-lane quarter hold gate and up of one feature. down: CTA h
+//     stages Wd rows n0+128h..+127.
+//   * N = the tokens of one expert's tile, a multiple of 16 up to 256; CTA h
+//     stages tokens N/2*h..+N/2-1 and the MMA reads both halves. An expert's
+//     c rows are split into ceil(c/256) tiles of equal size rounded up to 16,
+//     so at most 15 padded columns per tile are computed, where 256-row tiles
+//     of the untransposed product would pad up to 255 rows per expert.
+// Per CTA a stage is 16 KB of weights and a 128-row box of tokens (16 KB, of
+// which the MMA reads N/2 rows), 6 stages.
 // Both CTAs' TMA loads complete on the leader's full barrier (the leader
 // expects the pair's bytes); the leader's single MMA thread issues the
-// cta_group::2 MMAs and commits to both CTAs' barriers with
-// tcgen05.commit.multicast::cluster (no load uses multicast). Each CTA's
-// epilogue reads its own 128 TMEM lanes (its rows) and arrives remotely on the
-// leader's accumulator-empty barrier. All waits are bounded (1 s) and report
-// MOE_ERR_DEVICE_TIMEOUT; the pair meets at a cluster barrier before TMEM is
-// freed.
+// cta_group::2 MMAs and its commits arrive on both CTAs' barriers
+// (tcgen05.commit with a CTA mask; no load uses multicast). Each CTA's
+// epilogue reads its own 128 TMEM lanes and arrives remotely on the leader's
+// accumulator-empty barrier. In gate/up the gate and up values of a feature
+// sit in lanes 16 apart of one warp: the two threads swap half of each
+// 32-token chunk by a register shuffle and each finishes 16 tokens.
+// Eight epilogue warps, two per TMEM lane quarter, split each tile's token
+// columns in 64-column chunks, so the TMEM drain (shuffles, SiLU, stores)
+// keeps up with the MMAs of the next tile.
+// All waits are bounded (1 s) and report MOE_ERR_DEVICE_TIMEOUT; the pair
+// meets at a cluster barrier before TMEM is freed.
 #include <cooperative_groups.h>
 
 #include "moe_internal.cuh"
@@ -32,19 +44,20 @@ namespace cg = cooperative_groups;
 namespace moe {
 namespace {
 
-constexpr int BM = 128;      // rows per CTA (the pair: 256)
-constexpr int PM = 2 * BM;   // rows per pair tile
-constexpr int BN = 256;      // MMA N (each CTA stages 128 rows of B)
+constexpr int WM = 128;       // weight rows per CTA (MMA M = 256 per pair)
+constexpr int TN = 256;       // most tokens per tile (MMA N)
 constexpr int BK = 64;
 constexpr int UK = 16;
 constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = (BN / 2) * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB per CTA
-constexpr int TMEM_COLS = 2 * BN;
-constexpr int kThreads = 192;
+constexpr int A_BYTES = WM * BK * 2;              // 16 KB
+constexpr int B_ROWS = TN / 2;                    // token rows per CTA
+constexpr int B_BYTES = B_ROWS * BK * 2;          // one 128-row box (rows past N/2 unused)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB
+constexpr int TMEM_COLS = 2 * TN;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint64_t kWaitNs = 1000000000ull;
-constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // shared::cluster address of the pair's even CTA
+constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // shared::cluster address in the pair's even CTA
 
 struct Ctl {
     uint64_t full[STAGES];
@@ -68,12 +81,26 @@ __device__ __forceinline__ bool aborted(Ctl *ctl) {
     return *reinterpret_cast<volatile int *>(&ctl->abort) != 0;
 }
 
+// Tile load whose completion is counted on the barrier at the same offset in
+// the pair's even CTA.
 __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m, int x, int y,
                                                  uint64_t *bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar) & kPeerBitMask)
+        : "memory");
+}
+
+// gate/up weight box: {64 K, 16 rows, gate|up, 4 row groups} of the 4-D view
+// W[group][gate|up][row][k]; w = first 16-row group.
+__device__ __forceinline__ void tma_load_4d_pair(void *dst, const CUtensorMap *m, int x, int w,
+                                                 uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(0), "r"(0), "r"(w),
+        "r"(smem_u32(bar) & kPeerBitMask)
         : "memory");
 }
 
@@ -87,7 +114,7 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
         : "memory");
 }
 
-// Arrives on `bar` in both CTAs of the pair once the issued MMAs complete.
+// One arrival on `bar` in both CTAs of the pair once the issued MMAs complete.
 __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
@@ -96,11 +123,13 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
         : "memory");
 }
 
+// Arrival on the barrier at the same offset in CTA `rank` of the cluster. It
+// orders only this thread's earlier TMEM reads (fenced by the caller), not its
+// global stores, which nobody waits for.
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank) {
     uint32_t remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(rank));
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote)
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 
 __device__ __forceinline__ int find_expert(const int32_t *mts, int E, int q) {
@@ -112,34 +141,36 @@ __device__ __forceinline__ int find_expert(const int32_t *mts, int E, int q) {
     return lo;
 }
 
+// Work item: expert e, weight tile wt, token tile of `rows` tokens from
+// grouped row t0, computed with N = rows rounded up to 16.
 struct Item {
-    int e, nt, row0, rows;  // row0 / rows: this CTA's half of the pair tile
+    int e, wt, t0, rows, N;
 };
 
-__device__ __forceinline__ Item decode(int item, int NT, const int32_t *mts, const int32_t *offs,
-                                       int E, int half) {
+__device__ __forceinline__ Item decode(int item, int NW, const int32_t *mts, const int32_t *offs,
+                                       int E) {
     Item it;
-    it.e = find_expert(mts, E, item / NT);
-    const int mcount = mts[it.e + 1] - mts[it.e];
-    const int local = item - mts[it.e] * NT;
-    it.nt = local / mcount;
-    const int m = local - it.nt * mcount;
-    it.row0 = offs[it.e] + m * PM + half * BM;
-    it.rows = max(0, min(BM, offs[it.e + 1] - it.row0));
+    it.e = find_expert(mts, E, item / NW);
+    const int ntt = mts[it.e + 1] - mts[it.e];
+    const int local = item - mts[it.e] * NW;
+    it.wt = local / ntt;
+    const int tt = local - it.wt * ntt;
+    const int c = offs[it.e + 1] - offs[it.e];
+    const int ts = ((c + ntt - 1) / ntt + 15) & ~15;
+    it.t0 = offs[it.e] + tt * ts;
+    it.rows = min(ts, c - tt * ts);
+    it.N = (it.rows + 15) & ~15;
     return it;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
+// g * sigmoid(g) with the fast exponential and division (the result is
+// rounded to bf16); saturates to g for large g and to -0 for large -g.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <bool GATE_UP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    grouped_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
-                       const __grid_constant__ CUtensorMap tmB, GroupedParams p) {
+    grouped_tc2_kernel(const __grid_constant__ CUtensorMap tmW,
+                       const __grid_constant__ CUtensorMap tmT, GroupedParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -148,7 +179,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int32_t *offs = mts + (p.E + 1);                        // [E+1]
 
     cg::cluster_group cluster = cg::this_cluster();
-    const int half = static_cast<int>(cluster.block_rank());  // 0 = leader
+    const int half = static_cast<int>(cluster.block_rank());  // 0: the leader
     const bool leader = half == 0;
     const int pair = blockIdx.x / 2, npairs = gridDim.x / 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,13 +192,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], 2 * 128);  // both CTAs' epilogue threads
+            mbar_init(&ctl->tempty[b], 2 * kEpiWarps);  // one per epilogue warp of both CTAs
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {  // same warp in both CTAs: one allocation for the pair
+    if (warp == 1) {  // the same warp in both CTAs: one allocation for the pair
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&ctl->tmem_base)),
                      "r"(TMEM_COLS)
@@ -175,8 +206,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmT);
     }
     pdl_trigger();
     pdl_wait();
@@ -190,41 +221,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = ctl->tmem_base;
 
     const int NOUT = GATE_UP ? p.I : p.d;
-    const int NT = GATE_UP ? (p.I + 127) / 128 : (p.d + BN - 1) / BN;
+    const int NW = GATE_UP ? (p.I + 127) / 128 : (p.d + 2 * WM - 1) / (2 * WM);
     const int K = GATE_UP ? p.d : p.I;
     const int nk = (K + BK - 1) / BK;
-    const int total = mts[E] * NT;
+    const int total = mts[E] * NW;
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer (both CTAs) ----------------
+            // weight row (2-D, down) or first 16-row group (4-D, gate/up) of an item
+            auto wcoord = [&](const Item &it) {
+                return GATE_UP ? (it.e * 2 * p.I + it.wt * 128 + half * 64) / 16
+                               : it.e * p.d + it.wt * 2 * WM + half * WM;
+            };
             int s = 0;
             uint32_t ph = 0;
             uint32_t issued_parity[STAGES];
             bool issued[STAGES];
             for (int i = 0; i < STAGES; ++i) issued[i] = false;
             for (int item = pair; item < total && !aborted(ctl); item += npairs) {
-                const Item it = decode(item, NT, mts, offs, E, half);
+                const Item it = decode(item, NW, mts, offs, E);
+                const int trow = it.t0 + half * (it.N / 2);
+                const int wc = wcoord(it);
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) { ok = false; break; }
                     uint8_t *sa = smem + s * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
                     if (leader) mbar_arrive_expect_tx(&ctl->full[s], 2 * STAGE_BYTES);
-                    tma_load_2d_pair(sa, &tmA, kb * BK, it.row0, &ctl->full[s]);
-                    int rb;
-                    if (GATE_UP)  // leader: gate rows, peer: the matching up rows
-                        rb = it.e * 2 * p.I + it.nt * 128 + (half ? p.I : 0);
+                    if (GATE_UP)
+                        tma_load_4d_pair(sa, &tmW, kb * BK, wc, &ctl->full[s]);
                     else
-                        rb = it.e * p.d + it.nt * BN + half * (BN / 2);
-                    tma_load_2d_pair(sb, &tmB, kb * BK, rb, &ctl->full[s]);
+                        tma_load_2d_pair(sa, &tmW, kb * BK, wc, &ctl->full[s]);
+                    tma_load_2d_pair(sb, &tmT, kb * BK, trow, &ctl->full[s]);
                     issued[s] = true;
                     issued_parity[s] = ph;
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
             }
-            if (aborted(ctl) && leader) {  // our copies complete on the leader's barriers
+            if (aborted(ctl) && leader) {  // the pair's copies complete on the leader's barriers
                 const uint64_t dl = globaltimer_ns() + kWaitNs;
                 for (int i = 0; i < STAGES; ++i)
                     if (issued[i]) mbar_wait(&ctl->full[i], issued_parity[i], dl);
@@ -233,17 +269,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---------------- MMA issuer (leader only) ----------------
-            constexpr uint32_t idesc = idesc_bf16_f32(PM, BN);
             int s = 0;
             uint32_t ph = 0;
             int tile = 0;
             bool any = false;
             for (int item = pair; item < total && !aborted(ctl); item += npairs, ++tile) {
+                const Item it = decode(item, NW, mts, offs, E);
+                const uint32_t idesc = idesc_bf16_f32(2 * WM, it.N);
                 const int buf = tile & 1;
                 const uint32_t use = static_cast<uint32_t>(tile >> 1);
                 if (!wait_bar(&ctl->tempty[buf], (use & 1u) ^ 1u, ctl, p.status)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * TN);
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!wait_bar(&ctl->full[s], ph, ctl, p.status)) { ok = false; break; }
@@ -271,71 +308,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5, both CTAs) ----------------
-        const int q = warp & 3;
-        const int r = q * 32 + lane;
+        // ---------------- epilogue (warps 2..9, both CTAs) ----------------
+        const int q = warp & 3;            // TMEM lane quarter of this warp
+        const int c_first = ((warp - 2) >> 2) * 64;  // its 64-column chunks, every kEpiWarps/4-th
+        __nv_bfloat16 *c = static_cast<__nv_bfloat16 *>(p.c);
         int tile = 0;
         for (int item = pair; item < total && !aborted(ctl); item += npairs, ++tile) {
             const int buf = tile & 1;
             const uint32_t use = static_cast<uint32_t>(tile >> 1);
             if (!wait_bar(&ctl->tfull[buf], use & 1u, ctl, p.status)) break;
             tc_fence_after();
-            const Item it = decode(item, NT, mts, offs, E, half);
-            const uint32_t t_row = tmem_base + static_cast<uint32_t>(buf * BN) +
-                                   (static_cast<uint32_t>(q * 32) << 16);
-            const bool valid = r < it.rows && it.row0 + r < p.rows_cap;
-            __nv_bfloat16 *crow = static_cast<__nv_bfloat16 *>(p.c) +
-                                  static_cast<size_t>(valid ? it.row0 + r : 0) * NOUT;
+            const Item it = decode(item, NW, mts, offs, E);
+            const uint32_t t_lane = tmem_base + static_cast<uint32_t>(buf * TN) +
+                                    (static_cast<uint32_t>(q * 32) << 16);
+            const int nvalid = min(it.rows, p.rows_cap - it.t0);  // tokens stored
             if (GATE_UP) {
+                // lanes 0..15: gate of features f, lanes 16..31: up of the same f
+                const bool is_gate = lane < 16;
+                const int f = it.wt * 128 + half * 64 + q * 16 + (lane & 15);
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(t_row + c, g);
-                    tmem_ld_32x32b_x32(t_row + 128 + c, u);
+                for (int c0 = c_first; c0 < it.N; c0 += 64 * (kEpiWarps / 4)) {
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(t_lane + c0, v[0]);
+                    tmem_ld_32x32b_x32(t_lane + c0 + 32, v[1]);
                     tmem_ld_wait();
-                    const int f0 = it.nt * 128 + c;
-                    if (valid) {
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            if (f0 + v * 8 + 8 <= NOUT) {
-                                uint4 o;
-                                o.x = pack_bf16x2(silu_mul(__uint_as_float(g[v * 8 + 0]), __uint_as_float(u[v * 8 + 0])),
-                                                  silu_mul(__uint_as_float(g[v * 8 + 1]), __uint_as_float(u[v * 8 + 1])));
-                                o.y = pack_bf16x2(silu_mul(__uint_as_float(g[v * 8 + 2]), __uint_as_float(u[v * 8 + 2])),
-                                                  silu_mul(__uint_as_float(g[v * 8 + 3]), __uint_as_float(u[v * 8 + 3])));
-                                o.z = pack_bf16x2(silu_mul(__uint_as_float(g[v * 8 + 4]), __uint_as_float(u[v * 8 + 4])),
-                                                  silu_mul(__uint_as_float(g[v * 8 + 5]), __uint_as_float(u[v * 8 + 5])));
-                                o.w = pack_bf16x2(silu_mul(__uint_as_float(g[v * 8 + 6]), __uint_as_float(u[v * 8 + 6])),
-                                                  silu_mul(__uint_as_float(g[v * 8 + 7]), __uint_as_float(u[v * 8 + 7])));
-                                *reinterpret_cast<uint4 *>(crow + f0 + v * 8) = o;
-                            }
+                    for (int h = 0; h < 2; ++h) {
+                        // the gate thread finishes tokens 0..15 of the chunk, the up thread 16..31
+                        const int tb = c0 + h * 32 + (is_gate ? 0 : 16);
+                        const int lim = f < NOUT ? nvalid - tb : 0;
+                        __nv_bfloat16 *dst = c + static_cast<size_t>(it.t0 + tb) * NOUT + f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float mine_lo = __uint_as_float(v[h][j]);
+                            const float mine_hi = __uint_as_float(v[h][16 + j]);
+                            const float got = __shfl_xor_sync(0xffffffffu, is_gate ? mine_hi : mine_lo, 16);
+                            const float g = is_gate ? mine_lo : got;
+                            const float u = is_gate ? got : mine_hi;
+                            if (j < lim) *dst = __float2bfloat16_rn(silu(g) * u);
+                            dst += NOUT;
                         }
                     }
                 }
             } else {
+                const int n = it.wt * 2 * WM + half * WM + q * 32 + lane;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t a[32];
-                    tmem_ld_32x32b_x32(t_row + c, a);
+                for (int c0 = c_first; c0 < it.N; c0 += 64 * (kEpiWarps / 4)) {
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(t_lane + c0, v[0]);
+                    tmem_ld_32x32b_x32(t_lane + c0 + 32, v[1]);
                     tmem_ld_wait();
-                    const int n0 = it.nt * BN + c;
-                    if (valid) {
+                    if (n < NOUT) {
+                        const int lim = nvalid - c0;
+                        __nv_bfloat16 *dst = c + static_cast<size_t>(it.t0 + c0) * NOUT + n;
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            if (n0 + v * 8 + 8 <= NOUT) {
-                                uint4 o;
-                                o.x = pack_bf16x2(__uint_as_float(a[v * 8 + 0]), __uint_as_float(a[v * 8 + 1]));
-                                o.y = pack_bf16x2(__uint_as_float(a[v * 8 + 2]), __uint_as_float(a[v * 8 + 3]));
-                                o.z = pack_bf16x2(__uint_as_float(a[v * 8 + 4]), __uint_as_float(a[v * 8 + 5]));
-                                o.w = pack_bf16x2(__uint_as_float(a[v * 8 + 6]), __uint_as_float(a[v * 8 + 7]));
-                                *reinterpret_cast<uint4 *>(crow + n0 + v * 8) = o;
-                            }
+                        for (int j = 0; j < 64; ++j) {
+                            if (j < lim) *dst = __float2bfloat16_rn(__uint_as_float(v[j >> 5][j & 31]));
+                            dst += NOUT;
                         }
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive_remote(&ctl->tempty[buf], 0);  // the leader's barrier
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(&ctl->tempty[buf], 0);  // the leader's barrier
         }
     }
 
@@ -355,8 +391,8 @@ size_t smem_bytes(int E) {
     return 1024 + STAGES * STAGE_BYTES + sizeof(Ctl) + 2 * (E + 1) * sizeof(int32_t);
 }
 
-// CTA pairs that can be resident at once (an SM left without a partner in its
-// GPC cannot host half a pair), at most one per two SMs.
+// CTA pairs that can be resident at once (an SM without a partner in its GPC
+// cannot host half a pair), at most one pair per two SMs.
 int resident_pairs(const void *kern, size_t smem, int n_sm) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(n_sm / 2 * 2);
@@ -371,25 +407,25 @@ int resident_pairs(const void *kern, size_t smem, int n_sm) {
 }
 
 template <bool GATE_UP>
-int launch(const CUtensorMap &a, const CUtensorMap &b, const GroupedParams &p, int n_sm,
+int launch(const CUtensorMap &w, const CUtensorMap &t, const GroupedParams &p, int n_sm,
            cudaStream_t s) {
     auto kern = grouped_tc2_kernel<GATE_UP>;
     const size_t smem = smem_bytes(p.E);
     if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
-    static int pairs[2] = {0, 0};  // per kernel; the same device model throughout a process
+    static int pairs[2] = {0, 0};  // per kernel, for the device model of the process
     if (pairs[GATE_UP] == 0)
         pairs[GATE_UP] = resident_pairs(reinterpret_cast<const void *>(kern), smem, n_sm);
-    return launch_k(kern, dim3(2 * pairs[GATE_UP]), dim3(kThreads), smem, s, a, b, p);
+    return launch_k(kern, dim3(2 * pairs[GATE_UP]), dim3(kThreads), smem, s, w, t, p);
 }
 
 }  // namespace
 
 int launch_gemm_tc2_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s) {
-    return launch<true>(m.a_gate_up, m.w_gate_up, p, n_sm, s);
+    return launch<true>(m.w_gate_up_4d, m.a_gate_up, p, n_sm, s);
 }
 
 int launch_gemm_tc2_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s) {
-    return launch<false>(m.a_down, m.w_down_half, p, n_sm, s);
+    return launch<false>(m.w_down_half, m.a_down, p, n_sm, s);
 }
 
 }  // namespace moe

@@ -7,9 +7,9 @@
 //               per-chunk expert histogram
 //   2 dispatch  per-expert counts, offsets, row-tile prefix, perm / inv
 //   3 gate_up   grouped GEMM over the grouped normalised rows, SiLU(gate)*up
-//               (tcgen05 for bf16: 128-row tiles on single CTAs, or 256-row
-//               tiles on CTA pairs once the mean load reaches 256 rows per
-//               expert; SIMT for fp32)
+//               (tcgen05 for bf16: 128-row tiles on single CTAs, or tiles of
+//               256 weight rows x up to 256 tokens on CTA pairs once the mean
+//               load reaches 256 rows per expert; SIMT for fp32)
 //   4 down      grouped GEMM
 // (bf16 batches of at most 32 rows per expert on average fuse 3 and 4 into one
 // persistent kernel.)
@@ -248,9 +248,8 @@ static bool use_fused_experts(const moe_ctx *h, int N) {
                             static_cast<long long>(kDecodeRowsPerExpert) * h->E;
 }
 
-// Row-tiled bf16 GEMMs on CTA pairs (256-row tiles) once the mean load fills
-// a pair tile; below that the padding of 256-row tiles costs more than the
-// halved operand traffic per MMA saves.
+// bf16 GEMMs on CTA pairs (256 weight rows x up to 256 tokens) once the mean
+// load fills a token tile.
 static bool use_pair_gemms(const moe_ctx *h, int N) {
     if (!h->use_tc || h->pair_mode == 0) return false;
     if (h->pair_mode == 1) return true;

@@ -120,14 +120,17 @@ struct TcMaps {
     CUtensorMap w_gate_up;  // W   [E*2I][d],     box 64 x 128
     CUtensorMap a_down;     // act [rows][I],     box 64 x 128
     CUtensorMap w_down;     // Wd  [E*d][I],      box 64 x 256
-    CUtensorMap w_down_half;  // Wd [E*d][I],     box 64 x 128 (CTA-pair kernels)
+    // the CTA-pair kernels (weights as the M operand, tokens as N)
+    CUtensorMap w_gate_up_4d;  // W as [group][gate|up][16 rows][d], box 64 x 16 x 2 x 4
+    CUtensorMap w_down_half;   // Wd [E*d][I],   box 64 x 128
 };
 int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, const void *wd,
                   int rows_cap, int E, int d, int I);
 int launch_gemm_tc_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_gemm_tc_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_selftest_timeout(int *status, int timeout_us, cudaStream_t s);
-// The same contractions on CTA pairs (256-row tiles, grouped with tile_m 256).
+// The same contractions on CTA pairs: 256 weight rows x up to 256 tokens per
+// tile (experts split into token tiles of at most kTcPairTileM rows).
 constexpr int kTcPairTileM = 256;
 int launch_gemm_tc2_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_gemm_tc2_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
