@@ -404,6 +404,11 @@ int launch(const CUtensorMap &a, const CUtensorMap &b, const GroupedParams &p, i
 
 }  // namespace
 
+int tc_encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows) {
+    return encode_2d(m, base, rows, cols, box_rows);
+}
+
 int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, const void *wd,
                   int rows_cap, int E, int d, int I) {
     int rc;

@@ -4,7 +4,9 @@
 //
 // Launch sequence (all on the caller's stream, no host synchronisation):
 //   1 route     RMSNorm + fp32 router + sigmoid + biased top-k + weights, and the
-//               per-chunk expert histogram
+//               per-chunk expert histogram (SIMT fp32; for bf16 batches of 512
+//               tokens and more the router GEMM runs on the tensor cores with
+//               the router matrix split into three bf16 parts)
 //   2 dispatch  per-expert counts, offsets, row-tile prefix, perm / inv
 //   3 gate_up   grouped GEMM over the grouped normalised rows, SiLU(gate)*up
 //               (tcgen05 for bf16: 128-row tiles on single CTAs, or tiles of
@@ -41,6 +43,10 @@ struct moe_ctx {
     void *xp, *act, *y, *x_stage, *out_stage;
     int32_t *idx, *chunk_hist, *counts, *offsets, *mt_start, *perm, *inv;
     float *wts, *router_wt, *router_wg, *rinv;
+    void *router_w3;     // bf16 [3E][d]: W' split into three bf16 matrices (tensor-core router)
+    CUtensorMap w3_map;  // its TMA map (box 64 x 3E)
+    bool route_tc;       // the tensor-core router is available (bf16, E % 16 == 0, 3E <= 240)
+    int route_tc_mode;   // -1 by batch size, 0 never, 1 whenever available
     int *status;
     int rows_cap, e_pad, max_chunks;
 
@@ -156,7 +162,11 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         // the CTA-pair grouped GEMMs (both compute the same result).
         const char *e = getenv("MOE_TC_PAIR");
         h->pair_mode = (e && e[0] == '0') ? 0 : (e && e[0] == '1') ? 1 : -1;
+        // MOE_ROUTE_TC=0 / 1 likewise for the tensor-core and the SIMT routers
+        e = getenv("MOE_ROUTE_TC");
+        h->route_tc_mode = (e && e[0] == '0') ? 0 : (e && e[0] == '1') ? 1 : -1;
     }
+    h->route_tc = h->use_tc && route_tc_ok(d, n_experts);
 
     h->e_pad = (n_experts + 63) / 64 * 64;
     h->max_chunks = 16384 / n_experts < 256 ? 16384 / n_experts : 256;
@@ -182,6 +192,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         E * static_cast<size_t>(d) * 4,       // router_wg
         (E + 1) * 4,                          // sched
         256,                                  // status
+        3 * E * static_cast<size_t>(d) * 2,   // router_w3
     };
     const int nblocks = sizeof(sizes) / sizeof(sizes[0]);
     size_t total = 0, off[20];
@@ -211,6 +222,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->router_wg = reinterpret_cast<float *>(b + off[15]);
     h->sched = reinterpret_cast<int32_t *>(b + off[16]);
     h->status = reinterpret_cast<int *>(b + off[17]);
+    h->router_w3 = b + off[18];
     if (cudaMemset(h->ws, 0, total) != cudaSuccess) {
         cudaFree(h->ws);
         delete h;
@@ -218,6 +230,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     }
     if (launch_prepare_router(w->router_w, w->norm_gain, h->router_wg, h->router_wt, n_experts,
                               h->e_pad, d, 0) != MOE_OK ||
+        (h->route_tc && launch_split_router(h->router_wg, h->router_w3, n_experts, d, 0) != MOE_OK) ||
         cudaDeviceSynchronize() != cudaSuccess) {
         cudaFree(h->ws);
         delete h;
@@ -229,6 +242,9 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         if (rc == MOE_OK)
             rc = decode_build_maps(&h->decode_maps, h->xp, h->act, w->w_gate_up, w->w_down,
                                    h->rows_cap, n_experts, d, d_ff);
+        if (rc == MOE_OK && h->route_tc)
+            rc = tc_encode_2d(&h->w3_map, h->router_w3, 3 * static_cast<uint64_t>(n_experts), d,
+                              3 * n_experts);
         if (rc != MOE_OK) {
             cudaFree(h->ws);
             delete h;
@@ -246,6 +262,14 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
 static bool use_fused_experts(const moe_ctx *h, int N) {
     return h->use_tc && static_cast<long long>(N) * h->k <=
                             static_cast<long long>(kDecodeRowsPerExpert) * h->E;
+}
+
+// The tensor-core router (bf16 batches) from kRouteTcMinTokens tokens on; the
+// SIMT routers below that.
+constexpr int kRouteTcMinTokens = 512;
+static bool use_route_tc(const moe_ctx *h, int N) {
+    if (!h->route_tc || h->route_tc_mode == 0) return false;
+    return h->route_tc_mode == 1 || N >= kRouteTcMinTokens;
 }
 
 // bf16 GEMMs on CTA pairs (256 weight rows x up to 256 tokens) once the mean
@@ -313,7 +337,10 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     rp.chunk_hist = h->chunk_hist; rp.status = h->status;
     rp.N = N; rp.d = h->d; rp.E = h->E; rp.k = h->k; rp.e_pad = h->e_pad;
     rp.chunk_tokens = chunk_tokens; rp.eps = h->eps; rp.scale = h->scale;
-    MOE_TRY(launch_route(rp, h->dtype, kind, tt, s));
+    if (use_route_tc(h, N))
+        MOE_TRY(launch_route_tc(rp, h->w3_map, s));
+    else
+        MOE_TRY(launch_route(rp, h->dtype, kind, tt, s));
     MOE_MARK();
 
     DispatchParams dp;

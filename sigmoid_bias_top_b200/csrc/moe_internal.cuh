@@ -101,12 +101,16 @@ struct DecodeParams {
 // ---------------------------------------------------------------------------
 // Host-side launchers
 
-constexpr int kRouteSmall = 0, kRouteLarge = 1;
+constexpr int kRouteSmall = 0, kRouteLarge = 1, kRouteTc = 2;
 bool route_small_ok(int d, int E);
 int route_plan(int N, int d, int E, int *toks_per_group);
 int launch_route(const RouteParams &p, int dtype, int kind, int toks_per_group, cudaStream_t s);
 int launch_prepare_router(const float *w, const float *gain, float *wg, float *wt, int E,
                           int e_pad, int d, cudaStream_t s);
+// The tensor-core router of bf16 batches (W' split into three bf16 matrices).
+bool route_tc_ok(int d, int E);
+int launch_split_router(const float *wg, void *w3, int E, int d, cudaStream_t s);
+int launch_route_tc(const RouteParams &p, const CUtensorMap &w3_map, cudaStream_t s);
 size_t dispatch_smem(int nchunk, int E, int chunk_assign, int d);
 int launch_dispatch(const DispatchParams &p, cudaStream_t s);
 int launch_combine(const CombineParams &p, int dtype, cudaStream_t s);
@@ -124,6 +128,10 @@ struct TcMaps {
     CUtensorMap w_gate_up_4d;  // W as [group][gate|up][16 rows][d], box 64 x 16 x 2 x 4
     CUtensorMap w_down_half;   // Wd [E*d][I],   box 64 x 128
 };
+// 2-D bf16 map of a row-major [rows][cols] matrix, box 64 x box_rows,
+// 128-byte swizzle, zero fill outside.
+int tc_encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows);
 int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, const void *wd,
                   int rows_cap, int E, int d, int I);
 int launch_gemm_tc_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
@@ -391,6 +399,16 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
           "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
         : "r"(taddr)
         : "memory");
 }

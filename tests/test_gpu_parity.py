@@ -278,3 +278,45 @@ def test_single_and_pair_gemms_agree(monkeypatch):
         m.close()
     rel = (outs[0] - outs[1]).norm(dim=1) / outs[1].norm(dim=1)
     assert rel.max().item() < 1e-2
+
+
+def test_tc_router_ragged_small(monkeypatch):
+    """The tensor-core router (forced on) on a ragged batch: 300 tokens (two
+    full 128-token tiles and a tail), d = 320, E = 16."""
+    monkeypatch.setenv("MOE_ROUTE_TC", "1")
+    m, x, layer, out, r = run(SMALL_BF16)
+    full_check(SMALL_BF16, x, layer, out, r)
+
+
+@pytest.mark.parametrize("n_experts,top_k,d,n", [(64, 8, 2048, 777), (80, 6, 128, 513),
+                                                 (16, 1, 64, 129)])
+def test_tc_router_shapes(monkeypatch, n_experts, top_k, d, n):
+    """Expert counts 16..80 (3E = 48..240 MMA columns), top-k 1..8, d from 64,
+    token counts off the tile size; with k = 8 the dispatch chunks hold 64
+    tokens, so a 128-token tile adds to two chunks' histograms."""
+    monkeypatch.setenv("MOE_ROUTE_TC", "1")
+    w = SMALL_BF16.scaled(n_experts=n_experts, top_k=top_k, d=d, d_ff=128, n_tokens=n,
+                          router_std=0.05)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r, tokens="sample")
+
+
+def test_tc_and_simt_routers_agree(monkeypatch):
+    """The same 2048-token batch through both routers: identical expert sets
+    and slot order away from near ties, weights within fp32 rounding."""
+    w = W.PREFILL.scaled(n_tokens=2048)
+    layer = W.make_layer(w, 0, DEV)
+    x = W.make_x(w, DEV)
+    res = []
+    for mode in ("0", "1"):
+        monkeypatch.setenv("MOE_ROUTE_TC", mode)
+        m = MoeLayer(layer, w.top_k, w.eps, max_tokens=w.n_tokens)
+        m(x)
+        torch.cuda.synchronize()
+        assert m.status() == 0
+        r = m.debug_routing(w.n_tokens)
+        res.append((r["idx"].cpu(), r["w"].cpu()))
+        m.close()
+    same = (res[0][0] == res[1][0]).all(dim=1)
+    assert same.float().mean().item() > 0.999
+    torch.testing.assert_close(res[0][1][same], res[1][1][same], rtol=1e-5, atol=1e-7)
