@@ -106,12 +106,37 @@ def traffic_from_profiles(kernel: str, workload: str):
     return float(m.group(1))
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without comments and whitespace runs (string literals kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"':
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            i = src.find("\n", i)
+            i = n if i < 0 else i
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources' code (comments and layout ignored), recorded
+    with each ncu summary so that a changed kernel drops its traffic figure."""
     hs = hashlib.sha256()
     csrc = os.path.join(ROOT, "sigmoid_bias_top_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
         if f.endswith((".cu", ".cuh")):
-            hs.update(open(os.path.join(csrc, f), "rb").read())
+            hs.update(_strip_comments(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
     return hs.hexdigest()[:16]
 
 

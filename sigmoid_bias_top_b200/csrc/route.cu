@@ -7,8 +7,10 @@
 // logit independently, the stored bias is added after the activation and only
 // steers the top-k choice, and the mixture weights are the selected unbiased
 // scores over (their sum + eps), times the routed scale. The router stays in
-// fp32 (the FP8 release leaves the router gates unquantised, page 5, "Für
-// Engineers"), fed by the fp32 normalised row, never by its bf16 copy.
+// fp32 (the FP8 release leaves the router gates unquantised: inferencekey.com,
+// "LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig
+// verbraucht wie ein 2B-Modell", section "Für Engineers"), fed by the fp32
+// normalised row, never by its bf16 copy.
 //
 // Two kernels, chosen by batch size:
 // The RMSNorm gain is folded into the router matrix once, at context creation
