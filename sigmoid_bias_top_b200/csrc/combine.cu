@@ -59,30 +59,39 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     if (t == 0)  // the dispatch has consumed the chunk histogram: clear it for the next forward
         for (int i = threadIdx.x; i < p.chunk_hist_n; i += kThreads) p.chunk_hist[i] = 0;
     const int nvec = p.d / V;
-    int rows[kMaxTopK];
-    float w[kMaxTopK];
     const int total = p.N * k;
-    for (int j = 0; j < k; ++j) {
-        int r = p.inv[static_cast<size_t>(t) * k + j];
-        float wj = p.wts[static_cast<size_t>(t) * k + j];
-        if (r < 0 || r >= total) {  // never read outside y; report instead
-            if (threadIdx.x == 0) set_status(p.status, kStatusBounds);
-            r = 0;
-            wj = 0.f;
-        }
-        rows[j] = r;
-        w[j] = wj;
-    }
     const uint4 *x = static_cast<const uint4 *>(p.x) + static_cast<size_t>(t) * nvec;
     const uint4 *y = static_cast<const uint4 *>(p.y);
     uint4 *out = static_cast<uint4 *>(p.out) + static_cast<size_t>(t) * nvec;
     for (int v = threadIdx.x; v < nvec; v += kThreads) {
         float acc[V], yv[V];
         P::to_f(x[v], acc);
-        for (int j = 0; j < k; ++j) {
-            P::to_f(y[static_cast<size_t>(rows[j]) * nvec + v], yv);
+        // slots in groups of four, the four loads of a group in flight together
+        for (int j0 = 0; j0 < k; j0 += 4) {
+            uint4 raw[4];
+            float wj[4];
 #pragma unroll
-            for (int i = 0; i < V; ++i) acc[i] = fmaf(w[j], yv[i], acc[i]);
+            for (int u = 0; u < 4; ++u) {
+                wj[u] = 0.f;
+                if (j0 + u < k) {
+                    int r = p.inv[static_cast<size_t>(t) * k + j0 + u];
+                    wj[u] = p.wts[static_cast<size_t>(t) * k + j0 + u];
+                    if (r < 0 || r >= total) {  // never read outside y; report instead
+                        set_status(p.status, kStatusBounds);
+                        r = 0;
+                        wj[u] = 0.f;
+                    }
+                    raw[u] = y[static_cast<size_t>(r) * nvec + v];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (j0 + u < k) {
+                    P::to_f(raw[u], yv);
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[i] = fmaf(wj[u], yv[i], acc[i]);
+                }
+            }
         }
         out[v] = P::from_f(acc);
     }

@@ -62,7 +62,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int n, int *warp_sums
     return incl - (tid < n ? v : 0);
 }
 
-__global__ void __launch_bounds__(kThreads) dispatch_kernel(DispatchParams p) {
+__global__ void __launch_bounds__(kThreads, 4) dispatch_kernel(DispatchParams p) {
     extern __shared__ int4 smem_v[];
     const int E = p.E, nchunk = p.nchunk, k = p.k, d = p.d;
     float *gs = reinterpret_cast<float *>(smem_v);      // [d] RMSNorm gain
@@ -229,7 +229,26 @@ size_t dispatch_smem(int nchunk, int E, int chunk_assign, int d) {
 int launch_dispatch(const DispatchParams &p, cudaStream_t s) {
     const size_t smem = dispatch_smem(p.nchunk, p.E, p.chunk_tokens * p.k, p.d);
     if (ensure_smem(dispatch_kernel, smem) != MOE_OK) return MOE_ERR_CUDA;
-    return launch_k(dispatch_kernel, dim3(p.nchunk * p.replicas), dim3(kThreads), smem, s, p);
+    // All CTAs resident at once: a second wave of a few CTAs would repeat the
+    // whole prologue (histogram, ranking) after the first wave's copies.
+    thread_local size_t last_smem = 0;
+    thread_local int last_dev = -1, resident = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (smem != last_smem || dev != last_dev) {
+        int per_sm = 0, n_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_kernel, kThreads, smem) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        resident = per_sm * n_sm;
+        last_smem = smem;
+        last_dev = dev;
+    }
+    DispatchParams q = p;
+    const int fit = resident / p.nchunk;
+    q.replicas = fit < 1 ? 1 : fit < p.replicas ? fit : p.replicas;
+    return launch_k(dispatch_kernel, dim3(q.nchunk * q.replicas), dim3(kThreads), smem, s, q);
 }
 
 }  // namespace moe
