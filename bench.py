@@ -101,7 +101,9 @@ def traffic_from_profiles(kernel: str, workload: str):
     txt = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     h = re.search(r"source_sha256:\s*([0-9a-f]+)", txt)
-    if not m or not h or h.group(1) != kernel_source_hash():
+    f = re.search(r"source_files:\s*(.+)", txt)
+    files = f.group(1).split() if f else None
+    if not m or not h or h.group(1) != kernel_source_hash(files):
         return None
     return float(m.group(1))
 
@@ -129,12 +131,15 @@ def _strip_comments(src: str) -> str:
     return re.sub(r"\s+", " ", "".join(out)).strip()
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources' code (comments and layout ignored), recorded
-    with each ncu summary so that a changed kernel drops its traffic figure."""
+def kernel_source_hash(files=None) -> str:
+    """Hash of kernel source code (comments and layout ignored): of the given
+    csrc files (a kernel's own file and the shared header), else of all of
+    them. Recorded with each ncu summary, so that a changed kernel drops its
+    traffic figure while changes elsewhere keep it."""
     hs = hashlib.sha256()
     csrc = os.path.join(ROOT, "sigmoid_bias_top_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    names = sorted(files) if files else sorted(os.listdir(csrc))
+    for f in names:
         if f.endswith((".cu", ".cuh")):
             hs.update(_strip_comments(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
     return hs.hexdigest()[:16]
