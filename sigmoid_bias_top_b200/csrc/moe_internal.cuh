@@ -205,6 +205,78 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 }
 
 // ---------------------------------------------------------------------------
+// Per-token expert selection shared by the routers
+
+// Order-preserving integer image of a float (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Selection and weights of one token by one warp. srow[E] holds its logits
+// (overwritten with the sigmoid scores); the result goes to idx/wts row t and
+// the expert counts to hist (shared). Each round takes the largest biased
+// score (warp max of its integer image), then the lowest expert index among
+// the lanes holding it: exact fp32 top-k with ties to the lower index.
+__device__ __forceinline__ void select_token(const RouteParams &p, float *srow,
+                                             const float *bias_s, size_t t, int *hist, int lane) {
+    const int E = p.E, k = p.k;
+    const int epl = (E + 31) / 32;  // experts per lane
+    uint32_t key[kMaxExperts / 32];
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = 0u;  // below every real key: never selected
+        if (i < epl && e < E) {
+            const float s = 1.0f / (1.0f + expf(-srow[e]));
+            const float c = s + bias_s[e];
+            key[i] = (c == c) ? float_key(c) : 1u;  // a NaN score ranks below every number
+            srow[e] = s;  // each lane rewrites only its own experts
+        }
+    }
+    __syncwarp();
+    int sel[kMaxTopK];
+    float ssel[kMaxTopK];
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        if (j >= k) break;
+        uint32_t bk = 0u;
+        int bi = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxExperts / 32; ++i)
+            if (key[i] > bk) {  // ascending expert index: ties keep the lower one
+                bk = key[i];
+                bi = i;
+            }
+        const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t cand = (bk == top && top != 0u) ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu;
+        const uint32_t e = __reduce_min_sync(0xffffffffu, cand);
+        // k <= E: an unselected expert exists, so e < E here
+#pragma unroll
+        for (int i = 0; i < kMaxExperts / 32; ++i)
+            if (static_cast<uint32_t>(lane + 32 * i) == e) key[i] = 0u;
+        sel[j] = static_cast<int>(e);
+        ssel[j] = srow[e];
+        sum += ssel[j];
+    }
+    if (lane < k) {  // lane j writes slot j
+        const float den = sum + p.eps;
+        float sj = 0.f;
+        int ej = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+            if (j == lane) {
+                sj = ssel[j];
+                ej = sel[j];
+            }
+        p.idx[t * k + lane] = ej;
+        p.wts[t * k + lane] = p.scale * (sj / den);
+        atomicAdd(&hist[ej], 1);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {

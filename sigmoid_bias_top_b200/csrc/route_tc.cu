@@ -19,17 +19,27 @@
 // l_e = rinv * (D1_e + (D2_e + D3_e)) carries only fp32 accumulation
 // rounding, the same order of error as the SIMT fp32 dot product.
 //
-// One CTA per 128 tokens (192 threads): warp 0 issues the TMA loads of the
+// One CTA per 128 tokens, or a cluster of two splitting K when the pairs fit
+// in one wave (each takes half of the stages; the second leaves its partial
+// dot products and sums of squares in its shared memory, the first reads
+// them through DSMEM after a cluster barrier and adds them in rank order).
+// Per CTA (192 threads): warp 0 issues the TMA loads of the
 // x tile (128 rows x 64) and of [B1; B2; B3] (3E rows x 64) per stage; warp 1
 // allocates TMEM and issues tcgen05.mma; warps 2..5 (thread = token = TMEM
 // lane) sum the squares of their token's row from each shared-memory stage
 // while the MMA runs (the stage is freed once the MMA and the four warps are
-// done with it), then read the 3E accumulator columns of their token, form
-// the logits, and select the top k by insertion in ascending expert order
-// (ties keep the lower index), then write the weights and the expert counts
-// of the token's dispatch chunk. All waits are bounded (1 s) and report
-// MOE_ERR_DEVICE_TIMEOUT.
+// done with it), then read the 3E accumulator columns of their token and
+// leave the partial dot products in shared memory. In the first CTA the same
+// threads add the cluster's partials (rank order), form the logits, compute
+// the sigmoids eight experts at a time and select the top k with a
+// branch-free insertion in ascending expert order (ties keep the lower index),
+// then write the weights and the expert counts of the token's dispatch chunk.
+// All waits are bounded (1 s) and report MOE_ERR_DEVICE_TIMEOUT.
+#include <cooperative_groups.h>
+
 #include "moe_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace moe {
 namespace {
@@ -64,26 +74,25 @@ __device__ __forceinline__ bool aborted(Ctl *ctl) {
     return *reinterpret_cast<volatile int *>(&ctl->abort) != 0;
 }
 
-// Order-preserving integer image of a float (larger float -> larger key).
-__device__ __forceinline__ uint32_t float_key(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
+template <int KS>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ CUtensorMap tmW, RouteParams p, int ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const int E = p.E, k = p.k, NB = 3 * E;
+    const int E = p.E, NB = 3 * E;
     const int stage_bytes = X_BYTES + NB * BK * 2;  // a multiple of 1024 (E % 16 == 0)
     Ctl *ctl = reinterpret_cast<Ctl *>(smem + ns * stage_bytes);
     int *hist = reinterpret_cast<int *>(ctl + 1);  // [kHistChunks][E]
     float *bias_s = reinterpret_cast<float *>(hist + kHistChunks * E);  // [E]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * TM;
+    // KS CTAs (a cluster) share one 128-token tile, CTA `rank` taking the
+    // K stages [kb0, kb1); rank 0 adds the others' partial sums and selects
+    const int rank = KS > 1 ? static_cast<int>(cg::this_cluster().block_rank()) : 0;
+    const int t0 = (blockIdx.x / KS) * TM;
     if (threadIdx.x == 0) {
         for (int s = 0; s < ns; ++s) {
             mbar_init(&ctl->full[s], 1);
@@ -112,7 +121,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
-    const int nk = p.d / BK;
+    const int nk_all = p.d / BK;
+    const int kb0 = rank * nk_all / KS, kb1 = (rank + 1) * nk_all / KS;
+    const int nk = kb1 - kb0;  // stages of this CTA (may be 0 for tiny d)
 
     if (warp == 0) {
         if (lane == 0) {
@@ -126,8 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) break;
                 uint8_t *sx = smem + s * stage_bytes;
                 mbar_arrive_expect_tx(&ctl->full[s], static_cast<uint32_t>(stage_bytes));
-                tma_load_2d(sx, &tmX, kb * BK, t0, &ctl->full[s]);
-                tma_load_2d(sx + X_BYTES, &tmW, kb * BK, 0, &ctl->full[s]);
+                tma_load_2d(sx, &tmX, (kb0 + kb) * BK, t0, &ctl->full[s]);
+                tma_load_2d(sx + X_BYTES, &tmW, (kb0 + kb) * BK, 0, &ctl->full[s]);
                 issued[s] = true;
                 issued_parity[s] = ph;
                 if (++s == ns) { s = 0; ph ^= 1u; }
@@ -156,16 +167,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&ctl->empty[s]);
                 if (++s == ns) { s = 0; ph ^= 1u; }
             }
-            if (nk > 0) {  // publishes the logits; waited for here too, before TMEM is freed
-                umma_commit(&ctl->tfull);
-                mbar_wait(&ctl->tfull, 0, globaltimer_ns() + kWaitNs);
-            }
+            // publishes the partial sums (at once if this CTA had no stages);
+            // waited for here too, before TMEM is freed
+            umma_commit(&ctl->tfull);
+            mbar_wait(&ctl->tfull, 0, globaltimer_ns() + kWaitNs);
         }
     } else {
         // ---------------- squares, then logits and selection (warps 2..5) ----------------
         const int q = warp & 3;      // TMEM lane quarter of this warp
         const int r = q * 32 + lane;  // tile row = token
-        const size_t t = static_cast<size_t>(t0) + r;
         float ss0 = 0.f, ss1 = 0.f;
         int s = 0;
         uint32_t ph = 0;
@@ -196,79 +206,118 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&ctl->empty[s]);
             if (++s == ns) { s = 0; ph ^= 1u; }
         }
-        if (ok && wait_bar(&ctl->tfull, 0, ctl, p.status)) {
-            tc_fence_after();
-            const float rinv = 1.0f / sqrtf((ss0 + ss1) / static_cast<float>(p.d) + p.eps);
-            const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-            // the sigmoid scores to the (now idle) stage memory, [e][row],
-            // eight experts at a time (eight independent exp / divide chains);
-            // the selection is then a rolled pass over the experts
-            float *sc = reinterpret_cast<float *>(smem);
+        // this CTA's partial dot products x . W'_e ([e][row]) and partial sum
+        // of squares ([row]) go to the stage memory, idle once all four
+        // epilogue warps have read their last rows of x (named barrier 1,
+        // reached by every epilogue thread, also after a time-out) and the
+        // MMAs are done (tfull)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        float *part = reinterpret_cast<float *>(smem);
+        float *ssp = part + E * TM;
+        const bool have = ok && wait_bar(&ctl->tfull, 0, ctl, p.status);
+        if (have) tc_fence_after();
+        const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-            for (int c0 = 0; c0 < E; c0 += 8) {  // E % 16 == 0
-                uint32_t d1[8], d2[8], d3[8];
+        for (int c0 = 0; c0 < E; c0 += 8) {  // E % 16 == 0
+            uint32_t d1[8], d2[8], d3[8];
+            if (have && nk > 0) {
                 tmem_ld_32x32b_x8(t_lane + c0, d1);
                 tmem_ld_32x32b_x8(t_lane + E + c0, d2);
                 tmem_ld_32x32b_x8(t_lane + 2 * E + c0, d3);
                 tmem_ld_wait();
+            } else {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float l = rinv * (__uint_as_float(d1[j]) +
-                                            (__uint_as_float(d2[j]) + __uint_as_float(d3[j])));
-                    sc[(c0 + j) * TM + r] = 1.0f / (1.0f + expf(-l));
-                }
+                for (int j = 0; j < 8; ++j) d1[j] = d2[j] = d3[j] = 0u;
             }
-            uint32_t sk[kMaxTopK];
-            int se[kMaxTopK];
-            float sv[kMaxTopK];
-            // the best kMaxTopK in descending order (k <= kMaxTopK: the first
-            // k entries are the top k); fixed length keeps the list in registers
 #pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) { sk[j] = 0u; se[j] = 0; sv[j] = 0.f; }
+            for (int j = 0; j < 8; ++j)
+                part[(c0 + j) * TM + r] =
+                    __uint_as_float(d1[j]) + (__uint_as_float(d2[j]) + __uint_as_float(d3[j]));
+        }
+        ssp[r] = ss0 + ss1;
+    }
+
+    // the partial sums of every CTA of the cluster are in place
+    tc_fence_before();
+    if (KS > 1) cg::this_cluster().sync(); else __syncthreads();
+
+    if (warp >= 2 && rank == 0) {
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const size_t t = static_cast<size_t>(t0) + r;
+        float *part = reinterpret_cast<float *>(smem);
+        float *ssp = part + E * TM;
+        float ss = ssp[r];
+        for (int h = 1; h < KS; ++h) ss += cg::this_cluster().map_shared_rank(ssp, h)[r];
+        const float rinv = 1.0f / sqrtf(ss / static_cast<float>(p.d) + p.eps);
+        // sigmoid scores in place of the partials, eight experts at a time
+        // (independent exp / divide chains); then a rolled selection pass
+        float *sc = part;
 #pragma unroll 1
-            for (int e = 0; e < E; ++e) {
-                const float sg = sc[e * TM + r];
-                const float cb = sg + bias_s[e];
-                const uint32_t key = (cb == cb) ? float_key(cb) : 1u;  // NaN ranks lowest
-                // branch-free insertion: slot i takes the old slot i-1 if the
-                // new key beats it, else the new key if it beats the old slot
-                // i, else keeps its own (an equal key stays behind the earlier,
-                // lower expert); every slot reads only old values
+        for (int c0 = 0; c0 < E; c0 += 8) {
+            float dsum[8];
 #pragma unroll
-                for (int i = kMaxTopK - 1; i >= 0; --i) {
-                    const bool shift = i > 0 && sk[i > 0 ? i - 1 : 0] < key;
-                    const bool place = !shift && sk[i] < key;
-                    if (i > 0) {
-                        sk[i] = shift ? sk[i - 1] : place ? key : sk[i];
-                        se[i] = shift ? se[i - 1] : place ? e : se[i];
-                        sv[i] = shift ? sv[i - 1] : place ? sg : sv[i];
-                    } else {
-                        sk[i] = place ? key : sk[i];
-                        se[i] = place ? e : se[i];
-                        sv[i] = place ? sg : sv[i];
-                    }
+            for (int j = 0; j < 8; ++j) dsum[j] = part[(c0 + j) * TM + r];
+            for (int h = 1; h < KS; ++h) {
+                const float *peer = cg::this_cluster().map_shared_rank(part, h);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) dsum[j] += peer[(c0 + j) * TM + r];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) sc[(c0 + j) * TM + r] = 1.0f / (1.0f + expf(-rinv * dsum[j]));
+        }
+        uint32_t sk[kMaxTopK];
+        int se[kMaxTopK];
+        float sv[kMaxTopK];
+        // the best kMaxTopK in descending order (k <= kMaxTopK: the first
+        // k entries are the top k); fixed length keeps the list in registers
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) { sk[j] = 0u; se[j] = 0; sv[j] = 0.f; }
+#pragma unroll 1
+        for (int e = 0; e < E; ++e) {
+            const float sg = sc[e * TM + r];
+            const float cb = sg + bias_s[e];
+            const uint32_t key = (cb == cb) ? float_key(cb) : 1u;  // NaN ranks lowest
+            // branch-free insertion: slot i takes the old slot i-1 if the
+            // new key beats it, else the new key if it beats the old slot
+            // i, else keeps its own (an equal key stays behind the earlier,
+            // lower expert); every slot reads only old values
+#pragma unroll
+            for (int i = kMaxTopK - 1; i >= 0; --i) {
+                const bool shift = i > 0 && sk[i > 0 ? i - 1 : 0] < key;
+                const bool place = !shift && sk[i] < key;
+                if (i > 0) {
+                    sk[i] = shift ? sk[i - 1] : place ? key : sk[i];
+                    se[i] = shift ? se[i - 1] : place ? e : se[i];
+                    sv[i] = shift ? sv[i - 1] : place ? sg : sv[i];
+                } else {
+                    sk[i] = place ? key : sk[i];
+                    se[i] = place ? e : se[i];
+                    sv[i] = place ? sg : sv[i];
                 }
             }
-            if (t < static_cast<size_t>(p.N)) {
-                p.rinv[t] = rinv;
-                float sum = 0.f;
+        }
+        if (t < static_cast<size_t>(p.N)) {
+            p.rinv[t] = rinv;
+            float sum = 0.f;
 #pragma unroll
-                for (int j = 0; j < kMaxTopK; ++j)
-                    if (j < k) sum += sv[j];
-                const float den = sum + p.eps;
-                const int hc = static_cast<int>(t / p.chunk_tokens) - t0 / p.chunk_tokens;
+            for (int j = 0; j < kMaxTopK; ++j)
+                if (j < p.k) sum += sv[j];
+            const float den = sum + p.eps;
+            const int hc = static_cast<int>(t / p.chunk_tokens) - t0 / p.chunk_tokens;
 #pragma unroll
-                for (int j = 0; j < kMaxTopK; ++j) {
-                    if (j < k) {
-                        p.idx[t * k + j] = se[j];
-                        p.wts[t * k + j] = p.scale * (sv[j] / den);
-                        atomicAdd(&hist[hc * E + se[j]], 1);
-                    }
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (j < p.k) {
+                    p.idx[t * p.k + j] = se[j];
+                    p.wts[t * p.k + j] = p.scale * (sv[j] / den);
+                    atomicAdd(&hist[hc * E + se[j]], 1);
                 }
             }
         }
     }
 
+    // the other CTAs keep their partial sums until rank 0 has read them
+    if (KS > 1) cg::this_cluster().sync();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -323,6 +372,28 @@ int launch_split_router(const float *wg, void *w3, int E, int d, cudaStream_t s)
     return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+template <int KS>
+int launch_ks(const CUtensorMap &xm, const CUtensorMap &w3_map, const RouteParams &p, int ns,
+              size_t smem, int tiles, cudaStream_t s) {
+    auto kern = route_tc_kernel<KS>;
+    if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(KS * tiles);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = KS;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = KS > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kern, xm, w3_map, p, ns) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int launch_route_tc(const RouteParams &p, const CUtensorMap &w3_map, cudaStream_t s) {
     if (p.N <= 0) return MOE_OK;
     if (p.chunk_tokens % 32 != 0) return MOE_ERR_INVALID_ARG;
@@ -331,9 +402,19 @@ int launch_route_tc(const RouteParams &p, const CUtensorMap &w3_map, cudaStream_
     if (rc != MOE_OK) return rc;
     const int ns = stages_for(p.E);
     const size_t smem = smem_bytes(p.E, ns);
-    if (ensure_smem(route_tc_kernel, smem) != MOE_OK) return MOE_ERR_CUDA;
-    return launch_k(route_tc_kernel, dim3((p.N + TM - 1) / TM), dim3(kThreads), smem, s, xm,
-                    w3_map, p, ns);
+    thread_local int n_sm = 0, n_sm_dev = -1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dev != n_sm_dev) {
+        if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        n_sm_dev = dev;
+    }
+    // split K over a CTA pair while the pairs still fit in one wave (one CTA
+    // per SM): the per-CTA pipeline latency, not bandwidth, bounds this kernel
+    const int tiles = (p.N + TM - 1) / TM;
+    if (2 * tiles <= n_sm) return launch_ks<2>(xm, w3_map, p, ns, smem, tiles, s);
+    return launch_ks<1>(xm, w3_map, p, ns, smem, tiles, s);
 }
 
 }  // namespace moe
