@@ -125,7 +125,7 @@ def test_one_expert_takes_every_token():
     assert res["counts"][3] == 1000 and res["counts"].sum() == 1000
 
 
-@pytest.mark.parametrize("n", [1, 7, 129])
+@pytest.mark.parametrize("n", [1, 7, 64, 65, 129])
 def test_small_batches_decode_shapes(n):
     w = W.DECODE.scaled(n_tokens=n)
     m, x, layer, out, r = run(w, max_tokens=256)
