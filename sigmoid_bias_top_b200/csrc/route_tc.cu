@@ -19,10 +19,11 @@
 // l_e = rinv * (D1_e + (D2_e + D3_e)) carries only fp32 accumulation
 // rounding, the same order of error as the SIMT fp32 dot product.
 //
-// One CTA per 128 tokens, or a cluster of two splitting K when the pairs fit
-// in one wave (each takes half of the stages; the second leaves its partial
-// dot products and sums of squares in its shared memory, the first reads
-// them through DSMEM after a cluster barrier and adds them in rank order).
+// One CTA per 128 tokens, or a cluster of four or two splitting K when the
+// clusters fit in one wave (each takes its share of the stages; the others
+// leave their partial dot products and sums of squares in shared memory, the
+// first reads them through DSMEM after a cluster barrier and adds them in
+// rank order).
 // Per CTA (192 threads): warp 0 issues the TMA loads of the
 // x tile (128 rows x 64) and of [B1; B2; B3] (3E rows x 64) per stage; warp 1
 // allocates TMEM and issues tcgen05.mma; warps 2..5 (thread = token = TMEM
@@ -31,9 +32,9 @@
 // done with it), then read the 3E accumulator columns of their token and
 // leave the partial dot products in shared memory. In the first CTA the same
 // threads add the cluster's partials (rank order), form the logits, compute
-// the sigmoids eight experts at a time and select the top k with a
-// branch-free insertion in ascending expert order (ties keep the lower index),
-// then write the weights and the expert counts of the token's dispatch chunk.
+// the sigmoids eight experts at a time and select the top k in k rounds of
+// arg-max over the keys in shared memory (ties keep the lower index), then
+// write the weights and the expert counts of the token's dispatch chunk.
 // All waits are bounded (1 s) and report MOE_ERR_DEVICE_TIMEOUT.
 #include <cooperative_groups.h>
 
@@ -250,9 +251,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float ss = ssp[r];
         for (int h = 1; h < KS; ++h) ss += cg::this_cluster().map_shared_rank(ssp, h)[r];
         const float rinv = 1.0f / sqrtf(ss / static_cast<float>(p.d) + p.eps);
-        // sigmoid scores in place of the partials, eight experts at a time
-        // (independent exp / divide chains); then a rolled selection pass
+        // sigmoid scores in place of the partials and the biased-score keys
+        // beside them, eight experts at a time (independent exp / divide
+        // chains)
         float *sc = part;
+        uint32_t *kk = reinterpret_cast<uint32_t *>(
+            smem + ((static_cast<size_t>(E) * TM * 4 + TM * 4 + 1023) & ~size_t(1023)));  // [E][TM]
 #pragma unroll 1
         for (int c0 = 0; c0 < E; c0 += 8) {
             float dsum[8];
@@ -264,37 +268,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < 8; ++j) dsum[j] += peer[(c0 + j) * TM + r];
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) sc[(c0 + j) * TM + r] = 1.0f / (1.0f + expf(-rinv * dsum[j]));
+            for (int j = 0; j < 8; ++j) {
+                const float sg = 1.0f / (1.0f + expf(-rinv * dsum[j]));
+                const float cb = sg + bias_s[c0 + j];
+                sc[(c0 + j) * TM + r] = sg;
+                kk[(c0 + j) * TM + r] = (cb == cb) ? float_key(cb) : 1u;  // NaN ranks lowest
+            }
         }
-        uint32_t sk[kMaxTopK];
+        // k rounds of arg-max over the keys (0 = taken): eight partial maxima
+        // over the experts e = u mod 8 in ascending order (strictly greater
+        // keeps the lower expert), combined by larger key, then lower expert
         int se[kMaxTopK];
         float sv[kMaxTopK];
-        // the best kMaxTopK in descending order (k <= kMaxTopK: the first
-        // k entries are the top k); fixed length keeps the list in registers
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) { sk[j] = 0u; se[j] = 0; sv[j] = 0.f; }
-#pragma unroll 1
-        for (int e = 0; e < E; ++e) {
-            const float sg = sc[e * TM + r];
-            const float cb = sg + bias_s[e];
-            const uint32_t key = (cb == cb) ? float_key(cb) : 1u;  // NaN ranks lowest
-            // branch-free insertion: slot i takes the old slot i-1 if the
-            // new key beats it, else the new key if it beats the old slot
-            // i, else keeps its own (an equal key stays behind the earlier,
-            // lower expert); every slot reads only old values
+        for (int j = 0; j < kMaxTopK; ++j) {
+            se[j] = 0;
+            sv[j] = 0.f;
+            if (j < p.k) {
+                uint32_t bk[8];
+                int be[8];
 #pragma unroll
-            for (int i = kMaxTopK - 1; i >= 0; --i) {
-                const bool shift = i > 0 && sk[i > 0 ? i - 1 : 0] < key;
-                const bool place = !shift && sk[i] < key;
-                if (i > 0) {
-                    sk[i] = shift ? sk[i - 1] : place ? key : sk[i];
-                    se[i] = shift ? se[i - 1] : place ? e : se[i];
-                    sv[i] = shift ? sv[i - 1] : place ? sg : sv[i];
-                } else {
-                    sk[i] = place ? key : sk[i];
-                    se[i] = place ? e : se[i];
-                    sv[i] = place ? sg : sv[i];
+                for (int u = 0; u < 8; ++u) { bk[u] = 0u; be[u] = E; }
+#pragma unroll 2
+                for (int e0 = 0; e0 < E; e0 += 8) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t v = kk[(e0 + u) * TM + r];
+                        if (v > bk[u]) { bk[u] = v; be[u] = e0 + u; }
+                    }
                 }
+                uint32_t K = bk[0];
+                int B = be[0];
+#pragma unroll
+                for (int u = 1; u < 8; ++u)
+                    if (bk[u] > K || (bk[u] == K && be[u] < B)) { K = bk[u]; B = be[u]; }
+                // k <= E: an untaken expert remains, so B < E
+                se[j] = B;
+                sv[j] = sc[B * TM + r];
+                kk[B * TM + r] = 0u;
             }
         }
         if (t < static_cast<size_t>(p.N)) {
@@ -410,9 +421,11 @@ int launch_route_tc(const RouteParams &p, const CUtensorMap &w3_map, cudaStream_
             return MOE_ERR_CUDA;
         n_sm_dev = dev;
     }
-    // split K over a CTA pair while the pairs still fit in one wave (one CTA
-    // per SM): the per-CTA pipeline latency, not bandwidth, bounds this kernel
+    // split K over a cluster of 4 or 2 CTAs while the clusters still fit in
+    // one wave (one CTA per SM): the per-CTA pipeline latency, not bandwidth,
+    // bounds this kernel
     const int tiles = (p.N + TM - 1) / TM;
+    if (4 * tiles <= n_sm) return launch_ks<4>(xm, w3_map, p, ns, smem, tiles, s);
     if (2 * tiles <= n_sm) return launch_ks<2>(xm, w3_map, p, ns, smem, tiles, s);
     return launch_ks<1>(xm, w3_map, p, ns, smem, tiles, s);
 }
