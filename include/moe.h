@@ -74,7 +74,12 @@ typedef struct moe_ctx moe_ctx;
  *   MOE_F32: d % 4 == 0, any d_ff >= 1;
  *   MOE_BF16: d % 64 == 0, d_ff % 64 == 0 (tensor-core tiles).
  * On success *out receives the context; on failure *out is set to NULL and
- * nothing stays allocated. Synchronous. */
+ * nothing stays allocated. Synchronous.
+ * The kernels are chosen per forward from the batch size; two environment
+ * variables, read here, force the choice between kernels that compute the
+ * same result (for testing and tuning): MOE_TC_PAIR=0|1 (bf16 expert GEMMs
+ * on single CTAs or on CTA pairs) and MOE_ROUTE_TC=0|1 (SIMT or tensor-core
+ * router for bf16 inputs). */
 int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
                const moe_weights *w, int max_tokens, moe_ctx **out);
 
