@@ -37,7 +37,8 @@ from sigmoid_bias_top_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (d2048,E64,top4,I1536) + % of HBM / bf16 TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DEFAULT_STEPS = {"decode": 2000, "prefill": 200, "skewed": 100, "stacked": 20, "tiny": 2000}
+DEFAULT_STEPS = {"decode": 2000, "prefill": 200, "skewed": 100, "stacked": 20, "tiny": 2000,
+                 "verify": 1000}
 ROTATE = 4  # distinct weight copies cycled through (each step reads >= 1 GB > L2)
 
 

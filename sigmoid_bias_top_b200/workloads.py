@@ -1,7 +1,7 @@
 """Seeded synthetic inputs for the sigmoid-bias top-k MoE feed-forward block.
 
 This module only draws random tensors of the shapes and distributions of the
-five workloads; it contains none of the layer's arithmetic (no norm, no
+workloads; it contains none of the layer's arithmetic (no norm, no
 routing, no expert math), so that the CUDA path and the CPU oracle can both be
 fed from it without sharing any computation.
 
@@ -91,9 +91,20 @@ STACKED = Workload(
     n_experts=64, top_k=4, d_ff=1536, dtype="bf16", seed=5, n_layers=38,
     gain_jitter=0.02, router_std=0.02, bias_kind="uniform", bias_halfwidth=0.05)
 
+# Speculative-decoding verify step: the drafter of "LFM2.5-24B-A2B-DSpark ist
+# live auf Hugging Face" (orcarouter.ai, section "Was ist eigentlich im
+# Repository?") proposes blocks of 9 tokens, so the target verifies 9 + 1
+# tokens per sequence at once; 32 sequences give 320 tokens per step, whose
+# expert union is wider than a 32-token decode step's (section "Die fehlende
+# Mac-Nummer ist die interessante Auslassung.").
+VERIFY = Workload(
+    name="verify_B32x10_N320_d2048_E64_k4_I1536", n_tokens=320, d=2048, n_experts=64,
+    top_k=4, d_ff=1536, dtype="bf16", seed=6, gain_jitter=0.02, router_std=0.02,
+    bias_kind="uniform", bias_halfwidth=0.05)
+
 WORKLOADS: Dict[str, Workload] = {
     "tiny": TINY_F32, "decode": DECODE, "prefill": PREFILL, "skewed": SKEWED,
-    "stacked": STACKED,
+    "stacked": STACKED, "verify": VERIFY,
 }
 
 

@@ -53,6 +53,15 @@ def test_decode_full():
     assert (res["counts"] > 0).sum() >= 45
 
 
+def test_verify_sampled():
+    """The 320-token speculative verify step (fused expert kernel, all experts)."""
+    w = W.VERIFY
+    m, x, layer, out, r = run(w)
+    assert m.launches_per_forward(w.n_tokens) == 4
+    res = full_check(w, x, layer, out, r, tokens="sample")
+    assert (res["counts"] > 0).sum() >= 62
+
+
 def test_prefill_sampled():
     w = W.PREFILL
     m, x, layer, out, r = run(w)

@@ -61,3 +61,15 @@ def test_generator_is_seeded():
     assert not torch.equal(l0["router_w"], l1["router_w"])
     assert torch.equal(W.make_layer(W.TINY_F32, 0, with_experts=False)["router_w"],
                        l0["router_w"])
+
+
+def test_verify_widens_the_expert_union():
+    """320 verify tokens (32 sequences x 10) activate (nearly) every expert,
+    more than the 32-token decode step."""
+    w = W.VERIFY
+    layer = W.make_layer(w, with_experts=False)
+    r = _route(w, layer, W.make_x(w))
+    active = np.unique(r["idx"]).size
+    wd = W.DECODE
+    rd = _route(wd, W.make_layer(wd, with_experts=False), W.make_x(wd))
+    assert active >= 62 and active > np.unique(rd["idx"]).size, active
