@@ -329,3 +329,35 @@ def test_tc_and_simt_routers_agree(monkeypatch):
     same = (res[0][0] == res[1][0]).all(dim=1)
     assert same.float().mean().item() > 0.999
     torch.testing.assert_close(res[0][1][same], res[1][1][same], rtol=1e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("n_experts,top_k,n", [(256, 8, 300), (128, 4, 64), (256, 4, 4096)])
+def test_many_experts(n_experts, top_k, n):
+    """Up to the largest expert count (256) and top-k (8): the SIMT routers'
+    expert blocks, a 256-column dispatch histogram, the fused expert kernel
+    (N*k <= 32*E) and the single-CTA GEMMs (4096 tokens x 4 > 32 * 256)."""
+    w = SMALL_BF16.scaled(n_experts=n_experts, top_k=top_k, d=256, d_ff=128, n_tokens=n,
+                          router_std=0.05)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r, tokens="sample" if n > 512 else None)
+
+
+@pytest.mark.parametrize("route_tc", ["0", "1"])
+def test_wide_rows(monkeypatch, route_tc):
+    """d = 8192 through the cluster router (its row slices near the shared-
+    memory limit) and through the tensor-core router (128 K stages split over
+    a cluster of four)."""
+    monkeypatch.setenv("MOE_ROUTE_TC", route_tc)
+    w = SMALL_BF16.scaled(n_experts=16, top_k=4, d=8192, d_ff=128, n_tokens=96)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r)
+
+
+def test_fp32_widest_rows():
+    """The largest supported width, d = 32768, in fp32: the large router's
+    d-chunked tiles, a 128 KB gain vector in the dispatch's shared memory,
+    the SIMT expert GEMMs."""
+    w = W.TINY_F32.scaled(n_tokens=20, d=32768, d_ff=16, n_experts=8, top_k=2,
+                          router_std=1.0 / 181.0, gate_up_std=1.0 / 181.0, down_std=0.25)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r)
