@@ -77,8 +77,8 @@ typedef struct moe_ctx moe_ctx;
  * nothing stays allocated. Synchronous.
  * The kernels are chosen per forward from the batch size; two environment
  * variables, read here, force the choice between kernels that compute the
- * same result (for testing and tuning): MOE_TC_PAIR=0|1 (bf16 expert GEMMs
- * on single CTAs or on CTA pairs) and MOE_ROUTE_TC=0|1 (SIMT or tensor-core
+ * same result (for testing and tuning): MOE_TC_PAIR=0 (bf16 expert GEMMs
+ * on single CTAs instead of the default CTA pairs) and MOE_ROUTE_TC=0|1 (SIMT or tensor-core
  * router for bf16 inputs). */
 int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
                const moe_weights *w, int max_tokens, moe_ctx **out);

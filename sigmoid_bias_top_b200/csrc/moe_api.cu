@@ -54,7 +54,7 @@ struct moe_ctx {
     void *decode_maps;   // tensor maps of the fused small-batch kernel
     int32_t *sched;      // [1 + E] its work counter and per-expert completion counts
     bool use_tc;
-    int pair_mode;       // CTA-pair GEMMs: -1 by load, 0 never, 1 whenever not fused
+    int pair_mode;       // CTA-pair GEMMs: 0 never, else (default) whenever not fused
 
     int last_n;
     bool last_fused;  // the last forward used the fused small-batch expert kernel
@@ -272,12 +272,14 @@ static bool use_route_tc(const moe_ctx *h, int N) {
     return h->route_tc_mode == 1 || N >= kRouteTcMinTokens;
 }
 
-// bf16 GEMMs on CTA pairs (256 weight rows x up to 256 tokens) once the mean
-// load fills a token tile.
-static bool use_pair_gemms(const moe_ctx *h, int N) {
-    if (!h->use_tc || h->pair_mode == 0) return false;
-    if (h->pair_mode == 1) return true;
-    return static_cast<long long>(N) * h->k >= static_cast<long long>(kTcPairTileM) * h->E;
+// bf16 GEMMs on CTA pairs (256 weight rows x up to 256 tokens) for every
+// batch the fused expert kernel does not take. Their token tiles pad each
+// expert's rows to 16, where the single-CTA GEMMs pad them to a 128-row M
+// tile, so the pairs are as fast or faster at every batch size measured
+// (640 to 8192 tokens at E = 64, k = 4: 1% at 640, 17% at 3072); the
+// single-CTA GEMMs stay behind MOE_TC_PAIR=0 as an independent second path.
+static bool use_pair_gemms(const moe_ctx *h) {
+    return h->use_tc && h->pair_mode != 0;
 }
 
 // Adds the durations of up to `count` (all if < 0) recorded forwards, oldest
@@ -326,7 +328,7 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     int nchunk = 1, chunk_tokens = N;
     chunk_plan(N, h->k, h->max_chunks, &nchunk, &chunk_tokens);
     const bool fused = use_fused_experts(h, N);
-    const bool pair = !fused && use_pair_gemms(h, N);
+    const bool pair = !fused && use_pair_gemms(h);
     const int tile_m = !h->use_tc ? kSimtTileM : pair ? kTcPairTileM : kTcTileM;
 
     MOE_MARK();

@@ -255,11 +255,13 @@ def test_fp32_large_batch_tiled_router():
     full_check(w, x, layer, out, r, tokens="sample")
 
 
-def test_pair_gemms_ragged(monkeypatch):
-    """The CTA-pair GEMMs (256-row tiles, forced on) on ragged shapes: d and I
-    not multiples of the tile widths, experts whose rows end in the leader's
-    half of a pair tile, and empty experts."""
-    monkeypatch.setenv("MOE_TC_PAIR", "1")
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_grouped_gemms_ragged(monkeypatch, pair):
+    """The CTA-pair GEMMs (256 weight rows per pair tile) and the single-CTA
+    GEMMs (128-token tiles) on ragged shapes: d and I not multiples of the
+    tile widths, experts whose rows end in the leader's half of a pair tile,
+    and empty experts."""
+    monkeypatch.setenv("MOE_TC_PAIR", pair)
     m, x, layer, out, r = run(SMALL_BF16)
     full_check(SMALL_BF16, x, layer, out, r)
     w = SMALL_BF16.scaled(n_experts=8, top_k=1, d=256, d_ff=256, n_tokens=1000)
@@ -331,11 +333,14 @@ def test_tc_and_simt_routers_agree(monkeypatch):
     torch.testing.assert_close(res[0][1][same], res[1][1][same], rtol=1e-5, atol=1e-7)
 
 
-@pytest.mark.parametrize("n_experts,top_k,n", [(256, 8, 300), (128, 4, 64), (256, 4, 4096)])
-def test_many_experts(n_experts, top_k, n):
+@pytest.mark.parametrize("n_experts,top_k,n,pair", [(256, 8, 300, "1"), (128, 4, 64, "1"),
+                                                    (256, 4, 4096, "1"), (256, 4, 4096, "0")])
+def test_many_experts(monkeypatch, n_experts, top_k, n, pair):
     """Up to the largest expert count (256) and top-k (8): the SIMT routers'
     expert blocks, a 256-column dispatch histogram, the fused expert kernel
-    (N*k <= 32*E) and the single-CTA GEMMs (4096 tokens x 4 > 32 * 256)."""
+    (N*k <= 32*E), and both the CTA-pair and the single-CTA GEMMs
+    (4096 tokens x 4 > 32 * 256, 16 rows per expert on average)."""
+    monkeypatch.setenv("MOE_TC_PAIR", pair)
     w = SMALL_BF16.scaled(n_experts=n_experts, top_k=top_k, d=256, d_ff=128, n_tokens=n,
                           router_std=0.05)
     m, x, layer, out, r = run(w)
