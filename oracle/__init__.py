@@ -18,12 +18,13 @@ import torch
 
 from ._build import build
 
-F32, BF16, F64 = 0, 1, 2
+F32, BF16, F64, E4M3 = 0, 1, 2, 3
 
 MUTATIONS = {
     "none": 0, "biased_weights": 1, "softmax": 2, "bias_before_act": 3,
     "no_eps": 4, "no_gain": 5, "silu_on_up": 6, "tie_high": 7,
     "no_residual": 8, "mean_not_sum": 9, "slot_swap": 10, "down_transposed": 11,
+    "fp8_scale_transposed": 12, "fp8_no_act_quant": 13, "fp8_no_max": 14,
 }
 
 _lib = None
@@ -38,11 +39,15 @@ def lib():
         L.oracle_rmsnorm.argtypes = [I, I, D, P, I, P, P, I]
         L.oracle_route.argtypes = [I, I, I, I, D, D, P, I, P, P, P, P, P, P, P, I]
         L.oracle_forward.argtypes = [I, P, I, I, I, I, I, D, D, P, I, P, P, P, P, P, I,
-                                     P, P, P, P, I]
+                                     P, P, P, P, P, P, I]
+        L.oracle_expert.argtypes = [I, I, I, P, P, P, I, P, P, I, P, I]
+        L.oracle_quant.argtypes = [I, I, P, P, P, P, I]
+        L.oracle_e4m3.argtypes = [I, P, P, P, P]
         L.oracle_dispatch.argtypes = [I, I, I, P, P, P, P]
         L.oracle_set_threads.argtypes = [I]
-        for f in (L.oracle_rmsnorm, L.oracle_route, L.oracle_forward,
-                  L.oracle_dispatch, L.oracle_set_threads, L.oracle_num_mutations):
+        for f in (L.oracle_rmsnorm, L.oracle_route, L.oracle_forward, L.oracle_expert,
+                  L.oracle_quant, L.oracle_e4m3, L.oracle_dispatch, L.oracle_set_threads,
+                  L.oracle_num_mutations):
             f.restype = I
         _lib = L
     return _lib
@@ -62,6 +67,8 @@ def _raw(t: torch.Tensor):
         return t, t.data_ptr(), BF16
     if t.dtype == torch.float64:
         return t, t.data_ptr(), F64
+    if t.dtype == torch.float8_e4m3fn:
+        return t, t.data_ptr(), E4M3
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -102,11 +109,23 @@ def route(x, layer, k, eps, routed_scale=1.0, mutation=0):
     return {"idx": idx, "w": w, "s": s, "margin": margin}
 
 
+def _scales(layer, wdt):
+    """(keep-alive list, gate/up scale pointer, down scale pointer): the FP8_BLOCK
+    block scales for e4m3 weights, null pointers otherwise."""
+    if wdt != E4M3:
+        return [], None, None
+    sg, sd = _f32(layer["w_gate_up_scale"]), _f32(layer["w_down_scale"])
+    return [sg, sd], sg.data_ptr(), sd.data_ptr()
+
+
 def forward(x, layer, k, eps, routed_scale=1.0, tokens=None, forced=None, mutation=0):
     """Block output (x + MoE(RMSNorm(x))) in f64 for the listed tokens (all if None).
 
     forced: optional int array [n, k] of expert indices (slot order) to use
     instead of the oracle's own selection for those tokens.
+    e4m3 expert weights (torch.float8_e4m3fn) select the FP8_BLOCK experts;
+    the layer then also holds "w_gate_up_scale" [E][2I/128][d/128] and
+    "w_down_scale" [E][d/128][I/128] (float32).
     Returns dict(out[n,d] f64, idx[n,k], w[n,k], tokens[n]).
     """
     xk, xp, xdt = _raw(x)
@@ -114,6 +133,7 @@ def forward(x, layer, k, eps, routed_scale=1.0, tokens=None, forced=None, mutati
     wgu, wgp, wdt = _raw(layer["w_gate_up"])
     wd, wdp, wdt2 = _raw(layer["w_down"])
     assert wdt == wdt2
+    keep, sgp, sdp = _scales(layer, wdt)
     N, d = xk.shape
     E = rw.shape[0]
     I = wgu.shape[1] // 2
@@ -131,9 +151,57 @@ def forward(x, layer, k, eps, routed_scale=1.0, tokens=None, forced=None, mutati
     w = np.zeros((n, k), np.float64)
     _check(lib().oracle_forward(n, tokens.ctypes.data, N, d, E, k, I, eps, routed_scale,
                                 xp, xdt, g.data_ptr(), rw.data_ptr(), b.data_ptr(),
-                                wgp, wdp, wdt, fptr, out.ctypes.data, idx.ctypes.data,
-                                w.ctypes.data, mutation), "oracle_forward")
+                                wgp, wdp, wdt, sgp, sdp, fptr, out.ctypes.data,
+                                idx.ctypes.data, w.ctypes.data, mutation), "oracle_forward")
+    del keep
     return {"out": out, "idx": idx, "w": w, "tokens": tokens}
+
+
+def expert(xin, layer, e, mutation=0) -> np.ndarray:
+    """Expert e of the layer alone on input rows xin[n][d] (f64): y[n][d] f64.
+    For e4m3 weights the rows are quantised per group of 128 first."""
+    xin = np.ascontiguousarray(np.asarray(xin, dtype=np.float64))
+    wgu, wgp, wdt = _raw(layer["w_gate_up"])
+    wd, wdp, _ = _raw(layer["w_down"])
+    keep, sgp, sdp = _scales(layer, wdt)
+    n, d = xin.shape
+    I = wgu.shape[1] // 2
+    y = np.zeros((n, d), np.float64)
+    _check(lib().oracle_expert(n, d, I, xin.ctypes.data, wgp, wdp, wdt, sgp, sdp, int(e),
+                               y.ctypes.data, mutation), "oracle_expert")
+    del keep
+    return y
+
+
+def quant(v, mutation=0):
+    """FP8_BLOCK activation quantisation of rows v[n][m] in groups of 128:
+    dict(codes uint8 [n][m], scales f32 [n][ceil(m/128)], deq f64 [n][m])."""
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    n, m = v.shape
+    ng = (m + 127) // 128
+    codes = np.zeros((n, m), np.uint8)
+    scales = np.zeros((n, ng), np.float32)
+    deq = np.zeros((n, m), np.float64)
+    _check(lib().oracle_quant(n, m, v.ctypes.data, codes.ctypes.data, scales.ctypes.data,
+                              deq.ctypes.data, mutation), "oracle_quant")
+    return {"codes": codes, "scales": scales, "deq": deq}
+
+
+def e4m3_encode(f) -> np.ndarray:
+    """e4m3 codes (uint8) of float32 values: nearest, ties to even, saturating."""
+    f = np.ascontiguousarray(np.asarray(f, dtype=np.float32))
+    codes = np.zeros(f.shape, np.uint8)
+    _check(lib().oracle_e4m3(f.size, f.ctypes.data, codes.ctypes.data, None, None), "oracle_e4m3")
+    return codes
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """The value (f64) of each e4m3 code."""
+    codes = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    v = np.zeros(codes.shape, np.float64)
+    _check(lib().oracle_e4m3(codes.size, None, None, codes.ctypes.data, v.ctypes.data),
+           "oracle_e4m3")
+    return v
 
 
 def dispatch(idx: np.ndarray, n_experts: int):

@@ -31,6 +31,20 @@
  * the gated MLP is down( silu(gate x) * (up x) ) with gate rows first in the
  * packed matrix; the combine sums slots in slot order and adds the residual.
  *
+ * FP8_BLOCK experts, from "LFM2.5-24B-A2B" (same site, German page, section
+ * "Quantisierung"): expert weights are stored as FP8 statically in 128x128
+ * blocks, activations are quantised to FP8 dynamically per group of 128; the
+ * router stays unquantised. Readings taken: the FP8 format is e4m3 with no
+ * infinities (largest finite 448), decoded from its definition; a weight is
+ * its code's value times the fp32 scale of its 128x128 block ([row/128]
+ * [col/128] of each matrix); both expert inputs (the normalised row before
+ * gate/up, SiLU(gate)*up before down) are quantised per token in groups of
+ * 128 consecutive columns with s = amax/448 and code = e4m3(v/s) rounded to
+ * nearest even (saturating at 448), an all-zero group giving s = 0 and zero
+ * codes. That code decision is taken in fp32 like the kernel's: v is rounded
+ * to float first and amax, s and v/s are float operations. Everything else
+ * stays exact double arithmetic on the decoded values.
+ *
  * Planted mistakes (the `mutation` argument) exist only so that the tests can
  * show that each plausible error would be caught by a pin; 0 = the method.
  */
@@ -42,7 +56,10 @@
 #include <omp.h>
 #endif
 
-enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2, OR_E4M3 = 3 };
+
+/* FP8_BLOCK: weight blocks of FP8_B x FP8_B, activation groups of FP8_B. */
+enum { FP8_B = 128 };
 
 enum {
     MUT_NONE = 0,
@@ -57,8 +74,71 @@ enum {
     MUT_MEAN_NOT_SUM = 9,     /* RMS uses sum of squares without the 1/d       */
     MUT_SLOT_SWAP = 10,       /* slots ordered ascending instead of descending */
     MUT_DOWN_TRANSPOSED = 11, /* down matrix read as [I][d]                    */
-    MUT_COUNT = 12
+    MUT_FP8_SCALE_T = 12,     /* weight block scales read as [col/128][row/128] */
+    MUT_FP8_NO_ACT_QUANT = 13,/* SiLU(gate)*up not quantised before down       */
+    MUT_FP8_NO_MAX = 14,      /* activation scale amax instead of amax/448     */
+    MUT_COUNT = 15
 };
+
+/* Value of an e4m3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; exponent 0 is subnormal; S.1111.111 is NaN; no infinities). */
+static double e4m3_value(uint8_t c)
+{
+    int e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+    return (c & 0x80) ? -v : v;
+}
+
+/* e4m3 code of a float, rounded to nearest with ties to even, saturating to
+ * +-448. The spacing of e4m3 values is 2^-9 below 2^-6 and 2^(E-3) in the
+ * binade [2^E, 2^(E+1)); a / spacing is exact (a power-of-two division) and
+ * rint() rounds it to the nearest integer, ties to even. */
+static uint8_t e4m3_encode(float f)
+{
+    uint8_t sign = signbit(f) ? 0x80 : 0;
+    double a = fabs((double)f);
+    if (a != a) return 0x7F;
+    if (a >= 448.0) return sign | 0x7E;
+    double q;
+    if (a < ldexp(1.0, -6)) {
+        q = ldexp(1.0, -9);
+    } else {
+        int ex;
+        frexp(a, &ex);              /* a in [2^(ex-1), 2^ex) */
+        q = ldexp(1.0, ex - 1 - 3);
+    }
+    double v = rint(a / q) * q;     /* the nearest e4m3 magnitude */
+    if (v >= 448.0) return sign | 0x7E;
+    if (v < ldexp(1.0, -6)) return sign | (uint8_t)(v / ldexp(1.0, -9));
+    int ex;
+    double fr = frexp(v, &ex);      /* v = fr * 2^ex, fr in [0.5, 1) */
+    int mant = (int)(fr * 16.0) - 8;  /* (8 + mant) / 16 = fr */
+    return sign | (uint8_t)(((ex - 1 + 7) << 3) | mant);
+}
+
+/* Dynamic FP8 quantisation of n values in groups of FP8_B (the last group
+ * may be shorter): codes, per-group scales and the dequantised values
+ * (code value * scale, exact in double) replacing v. codes/scales may be
+ * NULL. */
+static void quant_groups(int n, double *v, uint8_t *codes, float *scales, int mutation)
+{
+    for (int g0 = 0; g0 < n; g0 += FP8_B) {
+        int g1 = g0 + FP8_B < n ? g0 + FP8_B : n;
+        float amax = 0.0f;
+        for (int j = g0; j < g1; ++j) {
+            float a = fabsf((float)v[j]);
+            if (a > amax) amax = a;
+        }
+        float sc = (mutation == MUT_FP8_NO_MAX) ? amax : amax / 448.0f;
+        if (scales) scales[g0 / FP8_B] = sc;
+        for (int j = g0; j < g1; ++j) {
+            uint8_t c = (sc > 0.0f) ? e4m3_encode((float)v[j] / sc) : 0;
+            if (codes) codes[j] = c;
+            v[j] = e4m3_value(c) * (double)sc;
+        }
+    }
+}
 
 static double ld(const void *p, int dtype, size_t i)
 {
@@ -69,7 +149,22 @@ static double ld(const void *p, int dtype, size_t i)
         memcpy(&f, &u, sizeof f);
         return (double)f;
     }
+    if (dtype == OR_E4M3) return e4m3_value(((const uint8_t *)p)[i]);
     return ((const double *)p)[i];
+}
+
+/* Element (r, c) of a [rows][cols] expert matrix starting at element `base`
+ * of w: the stored value, times its 128x128 block's scale when sc != NULL
+ * (sc points at this matrix's [rows/128][cols/128] scales). */
+static double wval(const void *w, int wdt, size_t base, int cols, int rows, int r, int c,
+                   const float *sc, int mutation)
+{
+    double v = ld(w, wdt, base + (size_t)r * cols + c);
+    if (!sc) return v;
+    int rb = r / FP8_B, cb = c / FP8_B;
+    int nrb = (rows + FP8_B - 1) / FP8_B, ncb = (cols + FP8_B - 1) / FP8_B;
+    size_t bi = (mutation == MUT_FP8_SCALE_T) ? (size_t)cb * nrb + rb : (size_t)rb * ncb + cb;
+    return v * (double)sc[bi];
 }
 
 /* Pre-FFN RMSNorm of one row. */
@@ -213,24 +308,73 @@ int oracle_route(int N, int d, int E, int k, double eps, double scale,
     return 0;
 }
 
+/* One gated SiLU expert e on the row xin[d] (read only): y[d] =
+ * down( silu(gate xin) * (up xin) ). For e4m3 weights (FP8_BLOCK) the
+ * weights carry their block scales (sgu, sdn: all experts' scales,
+ * [E][2I/128][d/128] and [E][d/128][I/128]) and both inputs are quantised
+ * per group of 128 first. Scratch: xq[d], gt/up/a[I]. */
+static void expert_mlp(int d, int I, const double *xin, const void *w_gate_up,
+                       const void *w_down, int wdt, const float *sgu, const float *sdn,
+                       size_t e, double *xq, double *gt, double *up, double *a, double *y,
+                       int mutation)
+{
+    const int fp8 = (wdt == OR_E4M3);
+    const size_t ngu = (size_t)((2 * I + FP8_B - 1) / FP8_B) * ((d + FP8_B - 1) / FP8_B);
+    const size_t ndn = (size_t)((d + FP8_B - 1) / FP8_B) * ((I + FP8_B - 1) / FP8_B);
+    const float *sg = fp8 ? sgu + e * ngu : NULL;
+    const float *sd = fp8 ? sdn + e * ndn : NULL;
+    memcpy(xq, xin, sizeof(double) * (size_t)d);
+    if (fp8) quant_groups(d, xq, NULL, NULL, mutation);
+    size_t gbase = e * (size_t)(2 * I) * (size_t)d;
+    for (int f = 0; f < I; ++f) {
+        double g = 0.0, u = 0.0;
+        for (int j = 0; j < d; ++j) {
+            g += wval(w_gate_up, wdt, gbase, d, 2 * I, f, j, sg, mutation) * xq[j];
+            u += wval(w_gate_up, wdt, gbase, d, 2 * I, I + f, j, sg, mutation) * xq[j];
+        }
+        gt[f] = g;
+        up[f] = u;
+    }
+    for (int f = 0; f < I; ++f)
+        a[f] = (mutation == MUT_SILU_ON_UP) ? up[f] * sigmoid(up[f]) * gt[f]
+                                             : gt[f] * sigmoid(gt[f]) * up[f];
+    if (fp8 && mutation != MUT_FP8_NO_ACT_QUANT) quant_groups(I, a, NULL, NULL, mutation);
+    size_t dbase = e * (size_t)d * (size_t)I;
+    for (int j = 0; j < d; ++j) {
+        double acc = 0.0;
+        for (int f = 0; f < I; ++f) {
+            double wv = (mutation == MUT_DOWN_TRANSPOSED)
+                            ? ld(w_down, wdt, dbase + (size_t)f * d + j)
+                            : wval(w_down, wdt, dbase, I, d, j, f, sd, mutation);
+            acc += wv * a[f];
+        }
+        y[j] = acc;
+    }
+}
+
 /* Full block output for a subset of tokens: out[n][d] (double) for the rows
  * tokens[0..n-1] of x. forced (may be NULL) gives each listed token's
  * selection [n][k] in slot order, used in place of the oracle's own choice;
- * idx_out/w_out (may be NULL) receive the selection and weights used. */
+ * idx_out/w_out (may be NULL) receive the selection and weights used.
+ * wdt == e4m3 selects the FP8_BLOCK experts with block scales sgu/sdn. */
 int oracle_forward(int n, const int64_t *tokens, int N, int d, int E, int k, int I,
                    double eps, double scale, const void *x, int xdt,
                    const float *gain, const float *router_w, const float *bias,
                    const void *w_gate_up, const void *w_down, int wdt,
+                   const float *sgu, const float *sdn,
                    const int32_t *forced, double *out, int32_t *idx_out,
                    double *w_out, int mutation)
 {
     if (n < 0 || N < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || I <= 0) return -1;
+    if (wdt == OR_E4M3 && (!sgu || !sdn)) return -1;
     for (int i = 0; i < n; ++i)
         if (tokens[i] < 0 || tokens[i] >= N) return -2;
     int bad = 0;
 #pragma omp parallel
     {
         double *xn = (double *)malloc(sizeof(double) * (size_t)d);
+        double *xq = (double *)malloc(sizeof(double) * (size_t)d);
+        double *y = (double *)malloc(sizeof(double) * (size_t)d);
         double *s = (double *)malloc(sizeof(double) * (size_t)E);
         double *c = (double *)malloc(sizeof(double) * (size_t)E);
         double *gt = (double *)malloc(sizeof(double) * (size_t)I);
@@ -257,37 +401,61 @@ int oracle_forward(int n, const int64_t *tokens, int N, int d, int E, int k, int
             for (int j = 0; j < d; ++j)
                 o[j] = (mutation == MUT_NO_RESIDUAL) ? 0.0 : ld(x, xdt, t * (size_t)d + j);
             for (int slot = 0; slot < k; ++slot) {
-                size_t e = (size_t)sel[slot];
-                size_t gbase = e * (size_t)(2 * I) * (size_t)d;
-                for (int f = 0; f < I; ++f) {
-                    double g = 0.0, u = 0.0;
-                    size_t rg = gbase + (size_t)f * d, ru = gbase + (size_t)(I + f) * d;
-                    for (int j = 0; j < d; ++j) {
-                        g += ld(w_gate_up, wdt, rg + j) * xn[j];
-                        u += ld(w_gate_up, wdt, ru + j) * xn[j];
-                    }
-                    gt[f] = g;
-                    up[f] = u;
-                }
-                for (int f = 0; f < I; ++f)
-                    a[f] = (mutation == MUT_SILU_ON_UP) ? up[f] * sigmoid(up[f]) * gt[f]
-                                                         : gt[f] * sigmoid(gt[f]) * up[f];
-                size_t dbase = e * (size_t)d * (size_t)I;
-                for (int j = 0; j < d; ++j) {
-                    double y = 0.0;
-                    for (int f = 0; f < I; ++f) {
-                        size_t off = (mutation == MUT_DOWN_TRANSPOSED)
-                                         ? dbase + (size_t)f * d + j
-                                         : dbase + (size_t)j * I + f;
-                        y += ld(w_down, wdt, off) * a[f];
-                    }
-                    o[j] += w[slot] * y;
-                }
+                expert_mlp(d, I, xn, w_gate_up, w_down, wdt, sgu, sdn, (size_t)sel[slot],
+                           xq, gt, up, a, y, mutation);
+                for (int j = 0; j < d; ++j) o[j] += w[slot] * y[j];
             }
         }
-        free(xn); free(s); free(c); free(gt); free(up); free(a); free(sel); free(w);
+        free(xn); free(xq); free(y); free(s); free(c); free(gt); free(up); free(a);
+        free(sel); free(w);
     }
     return bad ? -3 : 0;
+}
+
+/* Expert e alone on n input rows xin[n][d]: y[n][d] (the step each selected
+ * slot takes inside oracle_forward). */
+int oracle_expert(int n, int d, int I, const double *xin, const void *w_gate_up,
+                  const void *w_down, int wdt, const float *sgu, const float *sdn, int e,
+                  double *y, int mutation)
+{
+    if (n < 0 || d <= 0 || I <= 0 || e < 0) return -1;
+    if (wdt == OR_E4M3 && (!sgu || !sdn)) return -1;
+    double *xq = (double *)malloc(sizeof(double) * (size_t)d);
+    double *gt = (double *)malloc(sizeof(double) * (size_t)I);
+    double *up = (double *)malloc(sizeof(double) * (size_t)I);
+    double *a = (double *)malloc(sizeof(double) * (size_t)I);
+    for (int i = 0; i < n; ++i)
+        expert_mlp(d, I, xin + (size_t)i * d, w_gate_up, w_down, wdt, sgu, sdn, (size_t)e,
+                   xq, gt, up, a, y + (size_t)i * d, mutation);
+    free(xq); free(gt); free(up); free(a);
+    return 0;
+}
+
+/* FP8_BLOCK quantisation of rows v[n_rows][n] in groups of 128: codes
+ * [n_rows][n], scales [n_rows][ceil(n/128)], dequantised values deq[n_rows][n]. */
+int oracle_quant(int n_rows, int n, const double *v, uint8_t *codes, float *scales,
+                 double *deq, int mutation)
+{
+    if (n_rows < 0 || n <= 0) return -1;
+    const int ng = (n + FP8_B - 1) / FP8_B;
+    for (int r = 0; r < n_rows; ++r) {
+        memcpy(deq + (size_t)r * n, v + (size_t)r * n, sizeof(double) * (size_t)n);
+        quant_groups(n, deq + (size_t)r * n, codes + (size_t)r * n, scales + (size_t)r * ng,
+                     mutation);
+    }
+    return 0;
+}
+
+/* e4m3 code of each float (round to nearest even, saturating), and the value
+ * of each code: the format conversions alone, for the pins. */
+int oracle_e4m3(int n, const float *f, uint8_t *codes, const uint8_t *in_codes, double *values)
+{
+    if (n < 0) return -1;
+    for (int i = 0; i < n; ++i) {
+        if (f && codes) codes[i] = e4m3_encode(f[i]);
+        if (in_codes && values) values[i] = e4m3_value(in_codes[i]);
+    }
+    return 0;
 }
 
 /* Grouping of the N*k assignments by expert: counts[E], offsets[E+1]

@@ -219,7 +219,175 @@ def pin_identical_experts(mut):
     np.testing.assert_allclose(res["out"], want.numpy(), rtol=1e-12, atol=1e-12)
 
 
+# ---------------------------------------------------------------- FP8_BLOCK
+# "LFM2.5-24B-A2B" (flozi.net, German page, section "Quantisierung"): weights
+# FP8 static in 128x128 blocks, activations FP8 dynamic per group of 128.
+
+E4M3 = torch.float8_e4m3fn
+
+
+def fp8_layer(E, d, I, seed, bias_scale=0.5):
+    """A layer with e4m3 expert weights and per-block fp32 scales: codes of
+    normal draws spread over the e4m3 range, scales around 1/(16 sqrt(K))."""
+    base = rand_layer(E, d, I, seed, bias_scale=bias_scale)
+    g = torch.Generator().manual_seed(seed + 7)
+    return dict(
+        base,
+        w_gate_up=(torch.randn(E, 2 * I, d, generator=g) * 16).clamp(-448, 448).to(E4M3),
+        w_down=(torch.randn(E, d, I, generator=g) * 16).clamp(-448, 448).to(E4M3),
+        w_gate_up_scale=((0.5 + torch.rand(E, -(-2 * I // 128), -(-d // 128), generator=g))
+                         / (16 * math.sqrt(d))).float(),
+        w_down_scale=((0.5 + torch.rand(E, -(-d // 128), -(-I // 128), generator=g))
+                      / (16 * math.sqrt(I))).float())
+
+
+def dequant_weights(layer):
+    """float64 weights = code value x block scale (torch's e4m3 decoding)."""
+    def deq(codes, sc):
+        full = sc.double().repeat_interleave(128, 1).repeat_interleave(128, 2)
+        return codes.double() * full[:, :codes.shape[1], :codes.shape[2]]
+    return dict(layer, w_gate_up=deq(layer["w_gate_up"], layer["w_gate_up_scale"]),
+                w_down=deq(layer["w_down"], layer["w_down_scale"]))
+
+
+def pin_e4m3_codec(mut):
+    """The oracle's e4m3 decoding of all 256 codes and its encoding (nearest,
+    ties to even, saturating) agree with torch's float8_e4m3fn conversions,
+    on random values and on every midpoint between neighbouring codes."""
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes).view(E4M3).double().numpy()
+    got = oracle.e4m3_value(codes)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan) and np.array_equal(got[~nan], want[~nan])
+    pos = np.sort(want[:127])                      # 0 .. 448
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(np.float32)  # exact in float
+    g = torch.Generator().manual_seed(5)
+    vals = np.concatenate([mids, -mids, pos.astype(np.float32),
+                           (torch.randn(20000, generator=g) * 50).clamp(-460, 460).numpy(),
+                           (torch.randn(5000, generator=g) * 0.01).numpy()]).astype(np.float32)
+    ref = torch.from_numpy(vals).to(E4M3).view(torch.uint8).numpy()
+    got = oracle.e4m3_encode(vals)
+    # torch writes -0 for negative values that round to zero; both are zero
+    same = (got == ref) | ((got & 0x7F) == 0) & ((ref & 0x7F) == 0)
+    assert same.all(), vals[~same][:5]
+
+
+def pin_fp8_quant(mut):
+    """Group quantisation: closed forms (a group at its amax maps to 448, a
+    power-of-two amax gives exact codes, all-zero groups give zeros), groups
+    of 128 quantised independently, and the rounding bound of e4m3 on random
+    rows (relative 2^-4 for normal codes, 2^-10 s below)."""
+    c = 0.125
+    row = np.zeros(256)
+    row[:6] = [448 * c, c, 0.5 * c, 1.0625 * c, -3 * c, 0.0]   # group 0: amax 448c
+    row[128:130] = [0.3, 0.3]                                  # group 1: amax 0.3
+    q = oracle.quant(row[None], mutation=mut)
+    assert q["scales"][0, 0] == np.float32(c)
+    np.testing.assert_array_equal(q["deq"][0, :6], [448 * c, c, 0.5 * c, c, -3 * c, 0.0])
+    assert q["codes"][0, 0] == 0x7E and q["codes"][0, 128] == 0x7E
+    assert q["scales"][0, 1] == np.float32(np.float32(0.3) / np.float32(448))
+    z = oracle.quant(np.zeros((1, 130)), mutation=mut)
+    assert not z["codes"].any() and not z["scales"].any() and not z["deq"].any()
+    g = torch.Generator().manual_seed(6)
+    v = (torch.randn(16, 384, generator=g) * torch.rand(16, 1, generator=g) * 3).double().numpy()
+    q = oracle.quant(v, mutation=mut)
+    s = np.repeat(q["scales"].astype(np.float64), 128, axis=1)
+    amax = np.abs(v).reshape(16, 3, 128).max(2).repeat(128, 1)
+    np.testing.assert_allclose(s, amax / 448, rtol=2e-7)
+    err = np.abs(q["deq"] - v)
+    assert (err <= np.maximum(np.abs(v) / 16, s * 2.0 ** -10) * (1 + 1e-6) + 1e-300).all()
+
+
+def pin_fp8_expert_blocks(mut):
+    """One expert with permutation weights, in closed form: gate row f holds
+    code 1.0 and up row f code 2.0 at column (f + 128) mod 256, down is the
+    identity; the 128x128 block scales all differ. Then G[f] = sg * xq[p(f)],
+    U[f] = 2 su * xq[p(f)], y[j] = sd * Q(silu(G) U)[j], where xq = Q(x) and
+    Q is the group quantisation (pinned by pin_fp8_quant), and sg, su, sd are
+    the scales of the blocks the nonzero codes sit in."""
+    d = I = 256
+    perm = (np.arange(I) + 128) % d
+    wgu = np.zeros((1, 2 * I, d), np.float32)
+    wgu[0, np.arange(I), perm] = 1.0
+    wgu[0, I + np.arange(I), perm] = 2.0
+    wd = np.eye(d, dtype=np.float32)[None]
+    sgu = np.array([[[0.5, 0.25], [2.0, 4.0], [1.0, 0.125], [8.0, 0.5]]], np.float32)
+    sdn = np.array([[[2.0, 8.0], [0.25, 4.0]]], np.float32)
+    layer = {"w_gate_up": torch.from_numpy(wgu).to(E4M3), "w_down": torch.from_numpy(wd).to(E4M3),
+             "w_gate_up_scale": torch.from_numpy(sgu), "w_down_scale": torch.from_numpy(sdn)}
+    g = torch.Generator().manual_seed(8)
+    x = (torch.randn(3, d, generator=g) * 0.7).double().numpy()
+    y = oracle.expert(x, layer, 0, mutation=mut)
+    xq = oracle.quant(x)["deq"]
+    rb = np.arange(I) // 128
+    G = sgu[0, rb, 1 - rb] * xq[:, perm]
+    U = 2 * sgu[0, 2 + rb, 1 - rb] * xq[:, perm]
+    a = G * (1.0 / (1.0 + np.exp(-G))) * U
+    want = sdn[0, rb, rb] * oracle.quant(a)["deq"]
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-300)
+
+
+def pin_fp8_forward_error_bound(mut):
+    """The FP8_BLOCK forward against the unquantised forward (pinned above) on
+    the same, dequantised weights: the difference comes only from quantising
+    the two expert inputs and stays inside its interval bound: per element
+    |xq - xn| <= max(|xn|/16, s 2^-10) (plus the float rounding of xn),
+    propagated through |Wg|, |Wu|, the SiLU's slope (below 1.1), the second
+    quantisation and |Wd|, and weighted by the mixture weights."""
+    E, d, I, k = 6, 256, 128, 2
+    layer = fp8_layer(E, d, I, seed=51)
+    ref = dequant_weights(layer)
+    x = rand_x(12, d, 51)
+    got = oracle.forward(x, layer, k=k, eps=EPS, mutation=mut)
+    base = oracle.forward(x, ref, k=k, eps=EPS, forced=got["idx"])
+    xn = oracle.rmsnorm(x, layer["norm_gain"], EPS)
+    ex = np.maximum(np.abs(xn) / 16, np.abs(xn).reshape(12, 2, 128).max(2).repeat(128, 1)
+                    / 448 * 2.0 ** -10) + np.abs(xn) * 2.0 ** -23
+    bound = np.zeros((12, d))
+    for t in range(12):
+        for j, e in enumerate(got["idx"][t]):
+            Wg, Wu = ref["w_gate_up"][e, :I].numpy(), ref["w_gate_up"][e, I:].numpy()
+            Wd = ref["w_down"][e].numpy()
+            G0, U0 = Wg @ xn[t], Wu @ xn[t]
+            eG, eU = np.abs(Wg) @ ex[t], np.abs(Wu) @ ex[t]
+            a0 = G0 / (1 + np.exp(-G0)) * U0
+            da = 1.1 * eG * (np.abs(U0) + eU) + np.abs(G0 / (1 + np.exp(-G0))) * eU
+            amax = np.abs(a0) + da
+            sa = amax.reshape(1, 128).max(1).repeat(128) / 448
+            ea = np.maximum(amax / 16, sa * 2.0 ** -10) + amax * 2.0 ** -23
+            bound[t] += got["w"][t, j] * (np.abs(Wd) @ (da + ea))
+    diff = np.abs(got["out"] - base["out"])
+    assert (diff <= bound * 1.001 + 1e-12).all(), (diff / np.maximum(bound, 1e-30)).max()
+    assert diff.max() > 0  # the quantisation does change the result
+
+
+def pin_fp8_scale_code_trade(mut):
+    """A block's scale and its codes trade a power of two exactly: doubling
+    the scale of gate/up block (1, 0) of expert 2 while halving the codes
+    inside that block (every code chosen with an exactly halvable value)
+    leaves the output unchanged to the last bit."""
+    E, d, I, k = 3, 256, 128, 3
+    layer = fp8_layer(E, d, I, seed=61)
+    v = layer["w_gate_up"].float()
+    v = torch.where(v.abs() < 2.0 ** -5, torch.full_like(v, 0.25), v)  # normal, halvable
+    layer["w_gate_up"] = v.to(E4M3)
+    x = rand_x(4, d, 61)
+    o0 = oracle.forward(x, layer, k=k, eps=EPS, mutation=mut)["out"]
+    l2 = dict(layer)
+    wgu = layer["w_gate_up"].float().clone()
+    wgu[2, 128:256, 0:128] /= 2
+    l2["w_gate_up"] = wgu.to(E4M3)
+    sc = layer["w_gate_up_scale"].clone()
+    sc[2, 1, 0] *= 2
+    l2["w_gate_up_scale"] = sc
+    assert torch.equal(l2["w_gate_up"].float()[2, 128:256, :128] * 2,
+                       layer["w_gate_up"].float()[2, 128:256, :128])
+    o1 = oracle.forward(x, l2, k=k, eps=EPS, mutation=mut)["out"]
+    np.testing.assert_array_equal(o0, o1)
+
+
 PINS = [pin_five_candidate, pin_rmsnorm, pin_router_sigmoid, pin_weights_sum_below_one,
         pin_k1, pin_tie_break, pin_brute_force_subsets, pin_zero_bias_is_logit_topk,
         pin_bias_shift_invariance, pin_all_selected_bias_invariance,
-        pin_zero_down_is_identity, pin_identical_experts]
+        pin_zero_down_is_identity, pin_identical_experts, pin_e4m3_codec, pin_fp8_quant,
+        pin_fp8_expert_blocks, pin_fp8_forward_error_bound, pin_fp8_scale_code_trade]
