@@ -36,8 +36,17 @@ extern "C" {
 #endif
 
 /* Storage type of x, out and the expert matrices. The RMSNorm gain, router
- * matrix and expert bias are always fp32 (the router stays unquantised). */
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+ * matrix and expert bias are always fp32 (the router stays unquantised).
+ * MOE_FP8_BLOCK is the FP8 checkpoint's scheme ("LFM2.5-24B-A2B", flozi.net,
+ * German page, section "Quantisierung": weights FP8 static in 128x128
+ * blocks, activations FP8 dynamic per group of 128): x and out are bf16, the
+ * expert matrices are e4m3 codes (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, no infinities, largest finite 448) with one fp32 scale per
+ * 128x128 block, weight = code value * block scale. Inside the forward each
+ * token's input to gate/up and its SiLU(gate)*up row are quantised in groups
+ * of 128 columns: s = max|v| / 448, code = e4m3(v / s) rounded to nearest
+ * even with saturation (s = 0 and zero codes for an all-zero group). */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_FP8_BLOCK = 2 } moe_dtype;
 
 typedef enum {
     MOE_OK = 0,
@@ -62,6 +71,10 @@ typedef struct {
     const void  *w_gate_up;    /* [E][2I][d] rows 0..I-1 gate, rows I..2I-1 up        */
     const void  *w_down;       /* [E][d][I]  down projection                          */
     float        routed_scale; /* multiplies the normalised weights (1 in the page)   */
+    /* MOE_FP8_BLOCK only (ignored otherwise): fp32 scales of the 128x128 blocks,
+     * block (rb, cb) covering rows rb*128.. and columns cb*128.. of a matrix. */
+    const float *w_gate_up_scale; /* [E][2I/128][d/128]                               */
+    const float *w_down_scale;    /* [E][d/128][I/128]                                */
 } moe_weights;
 
 typedef struct moe_ctx moe_ctx;
@@ -72,7 +85,8 @@ typedef struct moe_ctx moe_ctx;
  * top_k = k, eps serves both the RMSNorm and the weight normalisation.
  * Supported: 1 <= top_k <= min(n_experts, 8), n_experts <= 256,
  *   MOE_F32: d % 4 == 0, any d_ff >= 1;
- *   MOE_BF16: d % 64 == 0, d_ff % 64 == 0 (tensor-core tiles).
+ *   MOE_BF16: d % 64 == 0, d_ff % 64 == 0 (tensor-core tiles);
+ *   MOE_FP8_BLOCK: d % 128 == 0, d_ff % 128 == 0 (whole scale blocks).
  * On success *out receives the context; on failure *out is set to NULL and
  * nothing stays allocated. Synchronous.
  * The kernels are chosen per forward from the batch size; two environment
@@ -83,7 +97,8 @@ typedef struct moe_ctx moe_ctx;
 int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
                const moe_weights *w, int max_tokens, moe_ctx **out);
 
-/* out[N][d] = x + MoE(RMSNorm(x)) for x[N][d] (device, dtype of the weights).
+/* out[N][d] = x + MoE(RMSNorm(x)) for x[N][d] (device, dtype of the weights;
+ * bf16 for MOE_FP8_BLOCK).
  * out == x (in place) is allowed; other overlap is not. Asynchronous on
  * `stream` (a cudaStream_t, NULL = legacy default stream): no host sync, no
  * allocation, a fixed sequence of kernel launches, so it can be captured in a
@@ -112,6 +127,13 @@ int moe_status(moe_ctx *h);
 int moe_debug_routing(moe_ctx *h, int32_t *idx, float *w, int32_t *perm,
                       int32_t *offsets, void *stream);
 
+/* MOE_FP8_BLOCK layers: device-to-device copy of the last forward's grouped,
+ * quantised expert inputs into caller buffers (either may be NULL):
+ * codes[N*k][d] e4m3 (row r is the normalised row of assignment perm[r]) and
+ * scales[N*k][d/128] fp32 group scales. MOE_ERR_INVALID_ARG for other dtypes.
+ * Asynchronous on stream. */
+int moe_debug_fp8_rows(moe_ctx *h, uint8_t *codes, float *scales, void *stream);
+
 /* Per-kernel timing. moe_profile(h, 1) starts (or restarts) profiling: each
  * forward then records CUDA events between its launches on its stream (a ring
  * of 1024 forwards; older entries are folded into running sums as it wraps).
@@ -123,7 +145,8 @@ int moe_profile(moe_ctx *h, int enable);
 int moe_kernel_times(moe_ctx *h, float *ms, int n);
 /* Name of kernel i of the last forward's launch sequence (static string), or
  * NULL: route, dispatch, gate_up, down, combine; or route, dispatch, experts,
- * combine when the batch was small enough for the fused expert kernel. */
+ * combine when the batch was small enough for the fused expert kernel (and
+ * always for MOE_FP8_BLOCK layers). */
 const char *moe_kernel_name(moe_ctx *h, int i);
 
 /* Number of kernel launches one forward makes for n_tokens tokens. */

@@ -18,7 +18,7 @@ from typing import Dict, List, Optional
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
-MOE_F32, MOE_BF16 = 0, 1
+MOE_F32, MOE_BF16, MOE_FP8_BLOCK = 0, 1, 2
 ERRORS = {
     0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
     -3: "MOE_ERR_ALIGNMENT", -4: "MOE_ERR_TOO_MANY_TOKENS", -5: "MOE_ERR_OOM",
@@ -37,7 +37,8 @@ class MoeWeights(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("norm_gain", ctypes.c_void_p),
                 ("router_w", ctypes.c_void_p), ("expert_bias", ctypes.c_void_p),
                 ("w_gate_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
-                ("routed_scale", ctypes.c_float)]
+                ("routed_scale", ctypes.c_float), ("w_gate_up_scale", ctypes.c_void_p),
+                ("w_down_scale", ctypes.c_void_p)]
 
 
 _lib = None
@@ -59,6 +60,7 @@ def lib() -> ctypes.CDLL:
         L.moe_destroy.argtypes = [P]
         L.moe_status.argtypes = [P]
         L.moe_debug_routing.argtypes = [P, P, P, P, P, P]
+        L.moe_debug_fp8_rows.argtypes = [P, P, P, P]
         L.moe_profile.argtypes = [P, I]
         L.moe_kernel_times.argtypes = [P, ctypes.POINTER(F), I]
         L.moe_kernel_name.argtypes = [P, I]
@@ -70,7 +72,8 @@ def lib() -> ctypes.CDLL:
         L.moe_strerror.argtypes = [I]
         L.moe_strerror.restype = ctypes.c_char_p
         for f in (L.moe_create, L.moe_forward, L.moe_forward_host, L.moe_destroy,
-                  L.moe_status, L.moe_debug_routing, L.moe_profile, L.moe_kernel_times,
+                  L.moe_status, L.moe_debug_routing, L.moe_debug_fp8_rows, L.moe_profile,
+                  L.moe_kernel_times,
                   L.moe_launches_per_forward, L.moe_selftest_timeout):
             f.restype = I
         _lib = L
@@ -120,6 +123,9 @@ class MoeLayer:
 
     layer: dict with norm_gain [d] f32, router_w [E,d] f32, bias [E] f32,
     w_gate_up [E,2I,d] and w_down [E,d,I] (both f32 or bf16), on one CUDA device.
+    FP8_BLOCK layers hold e4m3 (torch.float8_e4m3fn) expert matrices plus
+    w_gate_up_scale [E,2I/128,d/128] and w_down_scale [E,d/128,I/128] (f32);
+    their x and out are bf16.
     """
 
     def __init__(self, layer: Dict, top_k: int, eps: float = 1e-6,
@@ -128,24 +134,30 @@ class MoeLayer:
         wgu, wd = layer["w_gate_up"], layer["w_down"]
         E, twoI, d = wgu.shape
         I = twoI // 2
+        names = ["norm_gain", "router_w", "bias", "w_gate_up", "w_down"]
         if wgu.dtype == torch.bfloat16:
             dt = MOE_BF16
         elif wgu.dtype == torch.float32:
             dt = MOE_F32
+        elif wgu.dtype == torch.float8_e4m3fn:
+            dt = MOE_FP8_BLOCK
+            names += ["w_gate_up_scale", "w_down_scale"]
         else:
-            raise TypeError(f"expert weights must be f32 or bf16, got {wgu.dtype}")
-        self._keep = {n: layer[n].contiguous() for n in
-                      ("norm_gain", "router_w", "bias", "w_gate_up", "w_down")}
+            raise TypeError(f"expert weights must be f32, bf16 or e4m3, got {wgu.dtype}")
+        self._keep = {n: layer[n].contiguous() for n in names}
         for n, t in self._keep.items():
             if not t.is_cuda:
                 raise ValueError(f"{n} must be a CUDA tensor")
         self.d, self.E, self.I, self.k = d, E, I, top_k
         self.dtype = wgu.dtype
+        self.fp8 = dt == MOE_FP8_BLOCK
         self.max_tokens = max_tokens
         k = self._keep
         self._w = MoeWeights(dt, k["norm_gain"].data_ptr(), k["router_w"].data_ptr(),
                              k["bias"].data_ptr(), k["w_gate_up"].data_ptr(),
-                             k["w_down"].data_ptr(), routed_scale)
+                             k["w_down"].data_ptr(), routed_scale,
+                             k["w_gate_up_scale"].data_ptr() if self.fp8 else None,
+                             k["w_down_scale"].data_ptr() if self.fp8 else None)
         h = ctypes.c_void_p()
         with torch.cuda.device(wgu.device):
             _check(lib().moe_create(d, E, I, top_k, eps, ctypes.byref(self._w), max_tokens,
@@ -182,6 +194,18 @@ class MoeLayer:
                                        offsets.data_ptr(), _stream_ptr(stream)),
                "moe_debug_routing")
         return {"idx": idx, "w": w, "perm": perm, "offsets": offsets}
+
+    def debug_fp8_rows(self, n_tokens: int, stream=None):
+        """FP8_BLOCK layers: the last forward's grouped e4m3 input rows (uint8
+        codes [n*k, d], in the order of debug_routing's perm) and their group
+        scales [n*k, d/128] f32, as device tensors."""
+        import torch
+        rows = n_tokens * self.k
+        codes = torch.empty(rows, self.d, dtype=torch.uint8, device=self.device)
+        scales = torch.empty(rows, self.d // 128, dtype=torch.float32, device=self.device)
+        _check(lib().moe_debug_fp8_rows(self._h, codes.data_ptr(), scales.data_ptr(),
+                                        _stream_ptr(stream)), "moe_debug_fp8_rows")
+        return {"codes": codes, "scales": scales}
 
     def status(self) -> int:
         return lib().moe_status(self._h)

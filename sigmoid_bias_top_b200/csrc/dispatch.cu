@@ -25,7 +25,14 @@
 //      assignment, one warp per row: xp[row] = x[t] * rinv[t] * gain, the same
 //      fp32 products as the router's input, rounded once to the storage type.
 // The grouped rows let the gate/up GEMM load contiguous 128-row TMA boxes.
-#include "moe_internal.cuh"
+// For FP8_BLOCK layers ("LFM2.5-24B-A2B", German page, section
+// "Quantisierung": activations FP8, dynamic per group of 128) step 3 writes
+// e4m3 codes instead: each group of 128 normalised values (16 lanes) takes
+// s = amax / 448 and codes e4m3(v / s), nearest-even and saturating, with the
+// scale stored beside the codes.
+#include <cuda_fp8.h>
+
+#include "moe_fp8.cuh"
 
 namespace moe {
 namespace {
@@ -62,7 +69,30 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int n, int *warp_sums
     return incl - (tid < n ? v : 0);
 }
 
-__global__ void __launch_bounds__(kThreads, 4) dispatch_kernel(DispatchParams p) {
+// One group of 8 normalised values per lane, 16 lanes per group of 128: the
+// group's scale (shared by the half-warp) and the lane's 8 e4m3 codes.
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float *scale) {
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float s = __fdiv_rn(m, 448.f);
+    uint32_t w[2] = {0u, 0u};
+    if (s > 0.f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // byte i of the 8 = value i
+            const uint32_t c = __nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3);
+            w[i >> 2] |= c << (8 * (i & 3));
+        }
+    }
+    *scale = s;
+    return make_uint2(w[0], w[1]);
+}
+
+template <bool kQuant>
+__global__ void __launch_bounds__(kThreads, 4)
+    dispatch_kernel(DispatchParams p, uint8_t *xq, float *xs) {
     extern __shared__ int4 smem_v[];
     const int E = p.E, nchunk = p.nchunk, k = p.k, d = p.d;
     float *gs = reinterpret_cast<float *>(smem_v);      // [d] RMSNorm gain
@@ -167,6 +197,53 @@ __global__ void __launch_bounds__(kThreads, 4) dispatch_kernel(DispatchParams p)
     __syncthreads();
 
     // 3. normalised rows, one warp per row, 16-byte vectors, 8 loads in flight
+    if constexpr (kQuant) {
+        // bf16 input; d % 128 == 0, so each half-warp's 16 vectors (128
+        // values) are one quantisation group and are all in or all out of the row
+        const int vpr = d / 8;
+        const int gpr = d / kFp8Block;
+        const uint4 *xv = static_cast<const uint4 *>(p.x);
+        constexpr int U = 4;
+        for (int i = rep + warp * p.replicas; i < na; i += kWarps * p.replicas) {
+            const int pos = pos_s[i];
+            if (pos < 0) continue;
+            const int t = (a0 + i) / k;
+            const float r = p.rinv[t];
+            const uint4 *src = xv + static_cast<size_t>(t) * vpr;
+            uint2 *dst = reinterpret_cast<uint2 *>(xq + static_cast<size_t>(pos) * d);
+            for (int v0 = 0; v0 < vpr; v0 += 32 * U) {
+                uint4 raw[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    raw[u] = v < vpr ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    const bool in = v < vpr;
+                    const float *g = gs + (in ? v : 0) * 8;
+                    const float4 g0 = *reinterpret_cast<const float4 *>(g);
+                    const float4 g1 = *reinterpret_cast<const float4 *>(g + 4);
+                    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+                    float xnv[8];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        xnv[2 * h] = bf16_to_f32(w[h] & 0xFFFFu) * r * gg[2 * h];
+                        xnv[2 * h + 1] = bf16_to_f32(w[h] >> 16) * r * gg[2 * h + 1];
+                    }
+                    float sc;
+                    const uint2 codes = quant8(xnv, &sc);  // every lane takes part
+                    if (in) {
+                        dst[v] = codes;
+                        if ((lane & 15) == 0) xs[static_cast<size_t>(pos) * gpr + v / 16] = sc;
+                    }
+                }
+            }
+        }
+        return;
+    }
     const int vpr = d * p.elem_bytes / 16;  // vectors per row
     const int epv = 16 / p.elem_bytes;      // elements per vector
     const uint4 *xv = static_cast<const uint4 *>(p.x);
@@ -226,9 +303,11 @@ size_t dispatch_smem(int nchunk, int E, int chunk_assign, int d) {
             static_cast<size_t>(kWarps) * E + static_cast<size_t>(chunk_assign)) * 4;
 }
 
-int launch_dispatch(const DispatchParams &p, cudaStream_t s) {
+namespace {
+template <bool kQuant>
+int launch_dispatch_t(const DispatchParams &p, uint8_t *xq, float *xs, cudaStream_t s) {
     const size_t smem = dispatch_smem(p.nchunk, p.E, p.chunk_tokens * p.k, p.d);
-    if (ensure_smem(dispatch_kernel, smem) != MOE_OK) return MOE_ERR_CUDA;
+    if (ensure_smem(dispatch_kernel<kQuant>, smem) != MOE_OK) return MOE_ERR_CUDA;
     // All CTAs resident at once: a second wave of a few CTAs would repeat the
     // whole prologue (histogram, ranking) after the first wave's copies.
     thread_local size_t last_smem = 0;
@@ -237,7 +316,8 @@ int launch_dispatch(const DispatchParams &p, cudaStream_t s) {
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (smem != last_smem || dev != last_dev) {
         int per_sm = 0, n_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_kernel, kThreads, smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_kernel<kQuant>, kThreads,
+                                                          smem) !=
                 cudaSuccess ||
             cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -248,7 +328,17 @@ int launch_dispatch(const DispatchParams &p, cudaStream_t s) {
     DispatchParams q = p;
     const int fit = resident / p.nchunk;
     q.replicas = fit < 1 ? 1 : fit < p.replicas ? fit : p.replicas;
-    return launch_k(dispatch_kernel, dim3(q.nchunk * q.replicas), dim3(kThreads), smem, s, q);
+    return launch_k(dispatch_kernel<kQuant>, dim3(q.nchunk * q.replicas), dim3(kThreads), smem, s,
+                    q, xq, xs);
+}
+}  // namespace
+
+int launch_dispatch(const DispatchParams &p, cudaStream_t s) {
+    return launch_dispatch_t<false>(p, nullptr, nullptr, s);
+}
+
+int launch_dispatch_fp8(const DispatchParams &p, uint8_t *xq, float *xs, cudaStream_t s) {
+    return launch_dispatch_t<true>(p, xq, xs, s);
 }
 
 }  // namespace moe

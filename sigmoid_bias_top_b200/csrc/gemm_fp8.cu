@@ -1,0 +1,542 @@
+// gemm_fp8.cu -- FP8_BLOCK experts: both expert contractions of a batch in ONE
+// persistent kernel, e4m3 weights as the tensor-core M operand ("swap-AB").
+//
+// The gated SiLU expert of "LFM2.5-24B-A2B: Biased Routing, Short Convolutions
+// and Ten KV Caches" (flozi.net, English page, section "The router has two
+// different scores") with the FP8_BLOCK storage of the FP8 checkpoint
+// ("LFM2.5-24B-A2B", German page, section "Quantisierung": weights FP8 in
+// static 128x128 blocks, activations FP8 dynamic per group of 128).
+//
+// Work decomposition as in the bf16 small-batch kernel: an item is one
+// 128-row weight tile (gate/up item (e, ft): gate rows ft*128.. and the
+// matching up rows of expert e, K = d; down item (e, nt): rows nt*128.. of
+// Wd_e, K = I), claimed from one atomic counter, gate/up items first; a down
+// item of expert e waits until its I/128 gate/up items have published their
+// act rows. Each item runs in passes of up to 64 tokens.
+//
+// What FP8_BLOCK changes: a stage is one K block of 128 (128 e4m3 = one
+// 128-byte swizzle row), and every block has its own scale on both operands
+// (weight block scale sw, token group scale sa), so the tensor cores cannot
+// accumulate across blocks. Each K block's MMAs (kind::f8f6f4, M128, N32/64,
+// K32) start a fresh accumulator in one of four rotating TMEM buffers; the
+// epilogue warps load it (tcgen05.ld) and add partial * sw * sa[token] into
+// fp32 registers, while the tensor cores already fill the next buffer. At
+// the end of a pass:
+//   gate/up: a = SiLU(gate) * up per (token, row); the item's 128 rows are
+//     exactly one activation group of 128, so the group maximum is a max over
+//     the 128 epilogue threads (warp butterflies, then four warps through
+//     shared memory, met at an mbarrier), s = amax / 448 and the codes
+//     e4m3(a / s) (nearest-even, saturating) go to aq with s in as;
+//   down: y = the fp32 sum, rounded once to bf16.
+// Roles per CTA (192 threads): warp 0 lane 0 claims items and issues TMA;
+// warp 1 owns TMEM (512 columns) and one thread issues the MMAs; warps 2..5
+// are the epilogue. All waits are bounded (1 s) and report
+// MOE_ERR_DEVICE_TIMEOUT; on time-out the kernel drains its own copies and
+// MMAs, frees TMEM and returns.
+#include <cuda_fp8.h>
+
+#include <new>
+
+#include "moe_fp8.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int WM = 128;              // weight rows per item (MMA M)
+constexpr int TT = 32;               // tokens per token tile
+constexpr int MAXT = 2;              // token tiles per pass (N = 32 or 64)
+constexpr int NP = TT * MAXT;        // tokens per pass
+constexpr int BK = kFp8Block;        // K per stage: one scale block, 128 bytes per row
+constexpr int UK = 32;               // K per tcgen05.mma kind::f8f6f4
+constexpr int STAGES = 5;
+constexpr int A_BYTES = WM * BK;                         // 16 KB weight tile
+constexpr int B_TILE = TT * BK;                          // 4 KB token tile
+constexpr int STAGE_BYTES = 2 * A_BYTES + MAXT * B_TILE; // 40 KB
+constexpr int BUF_COLS = 2 * NP;     // TMEM columns per K-block buffer: gate 0..63, up 64..127
+constexpr int NBUF = 4;
+constexpr int TMEM_COLS = NBUF * BUF_COLS;  // 512
+constexpr int RING = 4;
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+struct Ctl {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[NBUF];
+    uint64_t tempty[NBUF];
+    uint64_t ufull[RING];
+    uint64_t uempty[RING];
+    uint64_t pub;        // every epilogue thread's act rows of an item are stored
+    uint64_t red_bar[2]; // the four epilogue warps' column maxima are in red[b]
+    uint64_t drain;
+    float red[2][4][NP]; // per epilogue warp, per token column: max |a| over its 32 rows
+    int ring_item[RING];
+    int ring_pass[RING];
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, int *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_wait(bar, parity, globaltimer_ns() + kWaitNs)) return true;
+    set_status(status, kStatusTimeout);
+    atomicExch(&ctl->abort, 1);
+    return false;
+}
+
+__device__ __forceinline__ bool aborted(Ctl *ctl) {
+    return *reinterpret_cast<volatile int *>(&ctl->abort) != 0;
+}
+
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+struct Unit {
+    bool gate_up;
+    int e, tile;         // expert, weight tile (ft or nt)
+    int row0, rows;      // grouped token rows of this pass
+    int ntt;             // token tiles (1 or 2)
+    bool last_pass;
+};
+
+__device__ __forceinline__ Unit decode(int item, int pass, int n_gu_tiles, int n_dn_tiles, int E,
+                                       const int32_t *offs) {
+    Unit u;
+    const int n_gu = E * n_gu_tiles;
+    u.gate_up = item < n_gu;
+    const int local = u.gate_up ? item : item - n_gu;
+    const int per = u.gate_up ? n_gu_tiles : n_dn_tiles;
+    u.e = local / per;
+    u.tile = local - u.e * per;
+    const int beg = offs[u.e], cnt = offs[u.e + 1] - beg;
+    u.row0 = beg + pass * NP;
+    u.rows = min(NP, cnt - pass * NP);
+    u.ntt = (u.rows + TT - 1) / TT;
+    u.last_pass = (pass + 1) * NP >= cnt;
+    return u;
+}
+
+struct Fp8Maps {
+    CUtensorMap w_gate_up;  // e4m3 [E*2I][d] box 128 x 128
+    CUtensorMap w_down;     // e4m3 [E*d][I]  box 128 x 128
+    CUtensorMap xq;         // e4m3 [rows][d] box 128 x 32
+    CUtensorMap aq;         // e4m3 [rows][I] box 128 x 32
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_experts_kernel(const __grid_constant__ Fp8Maps maps, Fp8ExpertParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + STAGES * STAGE_BYTES);
+    int32_t *offs = reinterpret_cast<int32_t *>(ctl + 1);  // [E+1]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int n_gu_tiles = p.I / WM;
+    const int n_dn_tiles = p.d / WM;
+    const int total = E * (n_gu_tiles + n_dn_tiles);
+    int *next_item = p.sched;     // claimed-item counter
+    int *done = p.sched + 1;      // [E] finished gate/up items per expert
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], 128);
+        }
+        for (int r = 0; r < RING; ++r) {
+            mbar_init(&ctl->ufull[r], 1);
+            mbar_init(&ctl->uempty[r], 1 + 128);  // the MMA thread and every epilogue thread
+        }
+        mbar_init(&ctl->pub, 128);
+        mbar_init(&ctl->red_bar[0], 128);
+        mbar_init(&ctl->red_bar[1], 128);
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&maps.w_gate_up);
+        tma_prefetch_desc(&maps.w_down);
+        tma_prefetch_desc(&maps.xq);
+        tma_prefetch_desc(&maps.aq);
+    }
+    pdl_trigger();
+    pdl_wait();
+    for (int i = threadIdx.x; i <= E; i += kThreads) offs[i] = p.offsets[i];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------- producer -------------------------
+            int s = 0;
+            uint32_t ph = 0;
+            int useq = 0;
+            bool issued[STAGES];
+            uint32_t issued_parity[STAGES];
+            for (int i = 0; i < STAGES; ++i) issued[i] = false;
+            bool ok = true;
+            while (ok && !aborted(ctl)) {
+                const int item = atomicAdd(next_item, 1);
+                const bool stop = item >= total;
+                int npass = 0;
+                Unit u0;
+                if (!stop) {
+                    u0 = decode(item, 0, n_gu_tiles, n_dn_tiles, E, offs);
+                    const int cnt = offs[u0.e + 1] - offs[u0.e];
+                    if (cnt <= 0) continue;  // expert without tokens: nothing to do
+                    npass = (cnt + NP - 1) / NP;
+                    if (!u0.gate_up) {
+                        // the expert's act rows must be complete: all its gate/up items
+                        const uint64_t dl = globaltimer_ns() + kWaitNs;
+                        uint32_t it = 0;
+                        while (ld_acquire(done + u0.e) < n_gu_tiles) {
+                            if ((++it & 255u) == 0 && globaltimer_ns() > dl) {
+                                set_status(p.status, kStatusTimeout);
+                                atomicExch(&ctl->abort, 1);
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!ok) break;
+                        fence_proxy_async_global();  // aq was written by generic stores
+                    }
+                }
+                for (int pass = 0; pass < (stop ? 1 : npass); ++pass) {
+                    const int slot = useq % RING;
+                    if (!wait_bar(&ctl->uempty[slot], ((useq / RING) & 1u) ^ 1u, ctl, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    ctl->ring_item[slot] = stop ? -1 : item;
+                    ctl->ring_pass[slot] = pass;
+                    mbar_arrive(&ctl->ufull[slot]);
+                    ++useq;
+                    if (stop) break;
+                    const Unit u = decode(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
+                    const int nk = (u.gate_up ? p.d : p.I) / BK;
+                    const uint32_t bytes = (u.gate_up ? 2 * A_BYTES : A_BYTES) + u.ntt * B_TILE;
+                    for (int kb = 0; kb < nk; ++kb) {
+                        if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) { ok = false; break; }
+                        uint8_t *sa = smem + s * STAGE_BYTES;
+                        uint8_t *sb = sa + 2 * A_BYTES;
+                        mbar_arrive_expect_tx(&ctl->full[s], bytes);
+                        if (u.gate_up) {
+                            const int rg = u.e * 2 * p.I + u.tile * WM;
+                            tma_load_2d(sa, &maps.w_gate_up, kb * BK, rg, &ctl->full[s]);
+                            tma_load_2d(sa + A_BYTES, &maps.w_gate_up, kb * BK, rg + p.I, &ctl->full[s]);
+                            for (int t = 0; t < u.ntt; ++t)
+                                tma_load_2d(sb + t * B_TILE, &maps.xq, kb * BK, u.row0 + t * TT, &ctl->full[s]);
+                        } else {
+                            tma_load_2d(sa, &maps.w_down, kb * BK, u.e * p.d + u.tile * WM, &ctl->full[s]);
+                            for (int t = 0; t < u.ntt; ++t)
+                                tma_load_2d(sb + t * B_TILE, &maps.aq, kb * BK, u.row0 + t * TT, &ctl->full[s]);
+                        }
+                        issued[s] = true;
+                        issued_parity[s] = ph;
+                        if (++s == STAGES) { s = 0; ph ^= 1u; }
+                    }
+                    if (!ok) break;
+                }
+                if (stop) break;
+            }
+            if (!ok || aborted(ctl)) {
+                // make the other roles leave, then let our own copies land
+                atomicExch(&ctl->abort, 1);
+                const uint64_t dl = globaltimer_ns() + kWaitNs;
+                for (int i = 0; i < STAGES; ++i)
+                    if (issued[i]) mbar_wait(&ctl->full[i], issued_parity[i], dl);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // --------------------------- MMA ----------------------------
+            int s = 0;
+            uint32_t ph = 0;
+            int useq = 0;
+            uint32_t nblk = 0;  // K blocks issued: buffer nblk % NBUF
+            bool any = false, ok = true;
+            while (ok && !aborted(ctl)) {
+                const int slot = useq % RING;
+                if (!wait_bar(&ctl->ufull[slot], (useq / RING) & 1u, ctl, p.status)) break;
+                const int item = ctl->ring_item[slot], pass = ctl->ring_pass[slot];
+                mbar_arrive(&ctl->uempty[slot]);
+                ++useq;
+                if (item < 0) break;
+                const Unit u = decode(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
+                const uint32_t idesc = idesc_e4m3_f32(WM, TT * u.ntt);
+                const int nk = (u.gate_up ? p.d : p.I) / BK;
+                for (int kb = 0; kb < nk; ++kb) {
+                    const int buf = static_cast<int>(nblk % NBUF);
+                    const uint32_t use = nblk / NBUF;
+                    if (!wait_bar(&ctl->tempty[buf], (use & 1u) ^ 1u, ctl, p.status)) { ok = false; break; }
+                    if (!wait_bar(&ctl->full[s], ph, ctl, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * BUF_COLS);
+                    const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b0 = a0 + 2 * A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / UK; ++kk) {
+                        const uint32_t acc = kk != 0 ? 1u : 0u;  // a fresh sum per K block
+                        const uint64_t bd = sw128_kmajor_desc(b0 + kk * UK);
+                        umma_e4m3(d0, sw128_kmajor_desc(a0 + kk * UK), bd, idesc, acc);
+                        if (u.gate_up)  // up rows into columns NP..: same tokens, second weight tile
+                            umma_e4m3(d0 + NP, sw128_kmajor_desc(a0 + A_BYTES + kk * UK), bd, idesc, acc);
+                    }
+                    any = true;
+                    umma_commit(&ctl->empty[s]);
+                    umma_commit(&ctl->tfull[buf]);
+                    ++nblk;
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (any) {
+                umma_commit(&ctl->drain);
+                mbar_wait(&ctl->drain, 0, globaltimer_ns() + kWaitNs);
+            }
+        }
+    } else {
+        // ------------------------- epilogue -------------------------
+        // thread <-> TMEM lane = weight row: warp w reads lanes 32*(w%4)..+31
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const int ngd = p.d / kFp8Block, ngi = p.I / kFp8Block;
+        int useq = 0;
+        uint32_t nblk = 0;
+        uint32_t npub = 0, nred = 0;  // phases of ctl->pub and ctl->red_bar
+        bool ok = true;
+        while (ok && !aborted(ctl)) {
+            const int slot = useq % RING;
+            if (!wait_bar(&ctl->ufull[slot], (useq / RING) & 1u, ctl, p.status)) break;
+            const int item = ctl->ring_item[slot], pass = ctl->ring_pass[slot];
+            mbar_arrive(&ctl->uempty[slot]);
+            ++useq;
+            if (item < 0) break;
+            const Unit u = decode(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
+            const int nk = (u.gate_up ? p.d : p.I) / BK;
+            // weight block scales of this item: row blocks of the gate and up
+            // tiles (gate/up) or of the Wd tile (down), one per K block
+            const float *swg = u.gate_up
+                ? p.sgu + (static_cast<size_t>(u.e) * (2 * n_gu_tiles) + u.tile) * ngd
+                : p.sdn + (static_cast<size_t>(u.e) * n_dn_tiles + u.tile) * ngi;
+            const float *swu = u.gate_up
+                ? p.sgu + (static_cast<size_t>(u.e) * (2 * n_gu_tiles) + n_gu_tiles + u.tile) * ngd
+                : swg;
+            const int ng = u.gate_up ? ngd : ngi;
+            float accg[NP], accu[NP];
+#pragma unroll
+            for (int c = 0; c < NP; ++c) { accg[c] = 0.f; accu[c] = 0.f; }
+            for (int kb = 0; kb < nk; ++kb) {
+                // token group scales of this K block: lane c holds column c (+32)
+                float sa[MAXT];
+#pragma unroll
+                for (int t = 0; t < MAXT; ++t) {
+                    const int c = t * TT + lane;
+                    sa[t] = 0.f;
+                    if (c < u.rows) {
+                        const size_t gi = static_cast<size_t>(u.row0 + c) * ng + kb;
+                        sa[t] = u.gate_up ? p.xs[gi] : __ldcg(p.as + gi);
+                    }
+                }
+                const float wg = __ldg(swg + kb);
+                const float wu = u.gate_up ? __ldg(swu + kb) : 0.f;
+                const int buf = static_cast<int>(nblk % NBUF);
+                const uint32_t use = nblk / NBUF;
+                ++nblk;
+                if (!wait_bar(&ctl->tfull[buf], use & 1u, ctl, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t t0 = tmem_base + static_cast<uint32_t>(buf * BUF_COLS) +
+                                    (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+                for (int t = 0; t < MAXT; ++t) {
+                    if (t < u.ntt) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t g[16], v[16];
+                            tmem_ld_32x32b_x16(t0 + t * TT + h * 16, g);
+                            if (u.gate_up) tmem_ld_32x32b_x16(t0 + NP + t * TT + h * 16, v);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                const float sc = __shfl_sync(0xffffffffu, sa[t], h * 16 + c);
+                                const int col = t * TT + h * 16 + c;
+                                accg[col] = fmaf(__uint_as_float(g[c]), sc * wg, accg[col]);
+                                if (u.gate_up)
+                                    accu[col] = fmaf(__uint_as_float(v[c]), sc * wu, accu[col]);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&ctl->tempty[buf]);
+            }
+            if (!ok) break;
+
+            if (!u.gate_up) {
+                __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.y);
+                const int f = u.tile * WM + r;
+#pragma unroll
+                for (int c = 0; c < NP; ++c)
+                    if (c < u.rows)
+                        y[static_cast<size_t>(u.row0 + c) * p.d + f] = __float2bfloat16_rn(accg[c]);
+                continue;
+            }
+
+            // a = SiLU(gate) * up; group maximum per token column over the 128 rows
+            float mine[MAXT];
+#pragma unroll
+            for (int c = 0; c < NP; ++c) {
+                const float gv = accg[c];
+                accg[c] = gv / (1.0f + expf(-gv)) * accu[c];
+            }
+#pragma unroll
+            for (int t = 0; t < MAXT; ++t) {
+                mine[t] = 0.f;
+                if (t < u.ntt) {
+#pragma unroll
+                    for (int c = 0; c < TT; ++c) {
+                        float m = fabsf(accg[t * TT + c]);
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        if (lane == c) mine[t] = m;
+                    }
+                }
+            }
+            const int rb = static_cast<int>(nred & 1u);
+#pragma unroll
+            for (int t = 0; t < MAXT; ++t) ctl->red[rb][q][t * TT + lane] = mine[t];
+            mbar_arrive(&ctl->red_bar[rb]);
+            if (!wait_bar(&ctl->red_bar[rb], (nred >> 1) & 1u, ctl, p.status)) break;
+            ++nred;
+            float sg[MAXT];  // lane c: the scale of column c (+32)
+#pragma unroll
+            for (int t = 0; t < MAXT; ++t) {
+                const int c = t * TT + lane;
+                const float m = fmaxf(fmaxf(ctl->red[rb][0][c], ctl->red[rb][1][c]),
+                                      fmaxf(ctl->red[rb][2][c], ctl->red[rb][3][c]));
+                sg[t] = __fdiv_rn(m, 448.f);
+                if (q == 0 && c < u.rows)
+                    p.as[static_cast<size_t>(u.row0 + c) * ngi + u.tile] = sg[t];
+            }
+            const int f = u.tile * WM + r;
+#pragma unroll
+            for (int t = 0; t < MAXT; ++t) {
+                if (t < u.ntt) {
+#pragma unroll
+                    for (int c = 0; c < TT; ++c) {
+                        const float sc = __shfl_sync(0xffffffffu, sg[t], c);
+                        const int col = t * TT + c;
+                        if (col < u.rows) {
+                            const uint8_t code = sc > 0.f
+                                ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(
+                                      __fdiv_rn(accg[col], sc), __NV_SATFINITE, __NV_E4M3))
+                                : static_cast<uint8_t>(0);
+                            p.aq[static_cast<size_t>(u.row0 + col) * p.I + f] = code;
+                        }
+                    }
+                }
+            }
+            if (u.last_pass) {
+                // publish the expert's act rows to the down items of other CTAs:
+                // every thread fences its stores (also towards the async proxy
+                // that the TMA reads use) and arrives; one thread waits for all
+                // 128 (bounded) and releases the per-expert counter
+                fence_proxy_async_global();
+                __threadfence();
+                mbar_arrive(&ctl->pub);
+                if (r == 0) {
+                    if (wait_bar(&ctl->pub, npub & 1u, ctl, p.status)) {
+                        __threadfence();
+                        atomicAdd(done + u.e, 1);
+                    }
+                }
+                ++npub;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+size_t smem_bytes(int E) { return 1024 + STAGES * STAGE_BYTES + sizeof(Ctl) + (E + 1) * 4; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// 2-D map of a row-major [rows][cols] byte matrix, box 128 bytes x box_rows,
+// 128-byte swizzle, zero fill outside.
+int encode_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = reinterpret_cast<EncodeTiledFn>(fn)(
+        m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+struct Fp8MapsHolder {
+    Fp8Maps m;
+};
+
+int fp8_build_maps(void **holder, const void *xq, const void *aq, const void *wgu,
+                   const void *wd, int rows_cap, int E, int d, int I) {
+    Fp8MapsHolder *h = new (std::nothrow) Fp8MapsHolder;
+    if (!h) return MOE_ERR_OOM;
+    int rc;
+    if ((rc = encode_u8(&h->m.w_gate_up, wgu, static_cast<uint64_t>(E) * 2 * I, d, WM)) != MOE_OK ||
+        (rc = encode_u8(&h->m.w_down, wd, static_cast<uint64_t>(E) * d, I, WM)) != MOE_OK ||
+        (rc = encode_u8(&h->m.xq, xq, rows_cap, d, TT)) != MOE_OK ||
+        (rc = encode_u8(&h->m.aq, aq, rows_cap, I, TT)) != MOE_OK) {
+        delete h;
+        return rc;
+    }
+    *holder = h;
+    return MOE_OK;
+}
+
+void fp8_free_maps(void *holder) { delete static_cast<Fp8MapsHolder *>(holder); }
+
+int launch_fp8_experts(const void *holder, const Fp8ExpertParams &p, int n_sm, cudaStream_t s) {
+    const Fp8MapsHolder *h = static_cast<const Fp8MapsHolder *>(holder);
+    const size_t smem = smem_bytes(p.E);
+    if (ensure_smem(fp8_experts_kernel, smem) != MOE_OK) return MOE_ERR_CUDA;
+    return launch_k(fp8_experts_kernel, dim3(n_sm), dim3(kThreads), smem, s, h->m, p);
+}
+
+}  // namespace moe

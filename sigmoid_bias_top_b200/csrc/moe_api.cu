@@ -14,7 +14,8 @@
 //               load reaches 256 rows per expert; SIMT for fp32)
 //   4 down      grouped GEMM
 // (bf16 batches of at most 32 rows per expert on average fuse 3 and 4 into one
-// persistent kernel.)
+// persistent kernel. FP8_BLOCK layers always do: their dispatch writes e4m3
+// rows with group scales and one persistent kernel runs both contractions.)
 //   5 combine   out = x + sum_j w_j y_j in fixed slot order
 #include <stdio.h>
 #include <stdlib.h>
@@ -24,7 +25,7 @@
 #include <unordered_map>
 #include <vector>
 
-#include "moe_internal.cuh"
+#include "moe_fp8.cuh"
 
 using namespace moe;
 
@@ -35,9 +36,16 @@ constexpr int kRingForwards = 1024;
 
 struct moe_ctx {
     int d, E, I, k, dtype, max_tokens, device, n_sm;
+    int xdtype;   // storage type of x and out: bf16 for FP8_BLOCK layers, else dtype
     float eps, scale;
     moe_weights w;
-    size_t elem;  // bytes per element of x / experts
+    size_t elem;  // bytes per element of x / out
+
+    // FP8_BLOCK layers: e4m3 rows and group scales (carved from xp and act)
+    bool fp8;
+    void *fp8_maps;
+    uint8_t *xq, *aq;
+    float *xs, *as;
 
     void *ws;  // one allocation, carved below
     void *xp, *act, *y, *x_stage, *out_stage;
@@ -116,11 +124,13 @@ extern "C" const char *moe_strerror(int code) {
 }
 
 static int check_shapes(int d, int E, int I, int k, int dtype, int max_tokens) {
-    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (dtype != MOE_F32 && dtype != MOE_BF16 && dtype != MOE_FP8_BLOCK) return MOE_ERR_INVALID_ARG;
     if (d <= 0 || E <= 0 || I <= 0 || k <= 0 || max_tokens <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (E > kMaxExperts || k > kMaxTopK || k > E) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (d % 4 != 0 || d > 32768) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (dtype == MOE_BF16 && (d % 64 != 0 || I % 64 != 0)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (dtype == MOE_FP8_BLOCK && (d % kFp8Block != 0 || I % kFp8Block != 0))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
     // 32-bit row indices and TMA coordinates
     if (static_cast<long long>(max_tokens) * k >= (1LL << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (static_cast<long long>(E) * 2 * I >= (1LL << 30) ||
@@ -142,6 +152,10 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     if (!aligned16(w->norm_gain) || !aligned16(w->router_w) || !aligned16(w->w_gate_up) ||
         !aligned16(w->w_down))
         return MOE_ERR_ALIGNMENT;
+    if (w->dtype == MOE_FP8_BLOCK) {
+        if (!w->w_gate_up_scale || !w->w_down_scale) return MOE_ERR_INVALID_ARG;
+        if (!aligned16(w->w_gate_up_scale) || !aligned16(w->w_down_scale)) return MOE_ERR_ALIGNMENT;
+    }
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_NO_DEVICE;
@@ -154,7 +168,9 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->d = d; h->E = n_experts; h->I = d_ff; h->k = top_k; h->dtype = w->dtype;
     h->max_tokens = max_tokens; h->device = dev; h->n_sm = prop.multiProcessorCount;
     h->eps = eps; h->scale = w->routed_scale; h->w = *w;
-    h->elem = (w->dtype == MOE_F32) ? 4 : 2;
+    h->fp8 = (w->dtype == MOE_FP8_BLOCK);
+    h->xdtype = h->fp8 ? MOE_BF16 : w->dtype;
+    h->elem = (h->xdtype == MOE_F32) ? 4 : 2;
     h->use_tc = (w->dtype == MOE_BF16);
     h->rows_cap = max_tokens * top_k;
     {
@@ -166,7 +182,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         e = getenv("MOE_ROUTE_TC");
         h->route_tc_mode = (e && e[0] == '0') ? 0 : (e && e[0] == '1') ? 1 : -1;
     }
-    h->route_tc = h->use_tc && route_tc_ok(d, n_experts);
+    h->route_tc = (h->use_tc || h->fp8) && route_tc_ok(d, n_experts);
 
     h->e_pad = (n_experts + 63) / 64 * 64;
     h->max_chunks = 16384 / n_experts < 256 ? 16384 / n_experts : 256;
@@ -223,6 +239,12 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->sched = reinterpret_cast<int32_t *>(b + off[16]);
     h->status = reinterpret_cast<int *>(b + off[17]);
     h->router_w3 = b + off[18];
+    if (h->fp8) {  // codes then scales, inside the (2-byte element) xp and act blocks
+        h->xq = static_cast<uint8_t *>(h->xp);
+        h->xs = reinterpret_cast<float *>(h->xq + R * d);
+        h->aq = static_cast<uint8_t *>(h->act);
+        h->as = reinterpret_cast<float *>(h->aq + R * d_ff);
+    }
     if (cudaMemset(h->ws, 0, total) != cudaSuccess) {
         cudaFree(h->ws);
         delete h;
@@ -246,6 +268,20 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
             rc = tc_encode_2d(&h->w3_map, h->router_w3, 3 * static_cast<uint64_t>(n_experts), d,
                               3 * n_experts);
         if (rc != MOE_OK) {
+            if (h->decode_maps) decode_free_maps(h->decode_maps);
+            cudaFree(h->ws);
+            delete h;
+            return rc;
+        }
+    }
+    if (h->fp8) {
+        rc = fp8_build_maps(&h->fp8_maps, h->xq, h->aq, w->w_gate_up, w->w_down, h->rows_cap,
+                            n_experts, d, d_ff);
+        if (rc == MOE_OK && h->route_tc)
+            rc = tc_encode_2d(&h->w3_map, h->router_w3, 3 * static_cast<uint64_t>(n_experts), d,
+                              3 * n_experts);
+        if (rc != MOE_OK) {
+            if (h->fp8_maps) fp8_free_maps(h->fp8_maps);
             cudaFree(h->ws);
             delete h;
             return rc;
@@ -260,6 +296,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
 // kDecodeRowsPerExpert grouped rows per expert; larger batches use the two
 // row-tiled grouped GEMMs.
 static bool use_fused_experts(const moe_ctx *h, int N) {
+    if (h->fp8) return true;
     return h->use_tc && static_cast<long long>(N) * h->k <=
                             static_cast<long long>(kDecodeRowsPerExpert) * h->E;
 }
@@ -342,7 +379,7 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     if (use_route_tc(h, N))
         MOE_TRY(launch_route_tc(rp, h->w3_map, s));
     else
-        MOE_TRY(launch_route(rp, h->dtype, kind, tt, s));
+        MOE_TRY(launch_route(rp, h->xdtype, kind, tt, s));
     MOE_MARK();
 
     DispatchParams dp;
@@ -357,7 +394,10 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     // several CTAs per chunk share the row copies: about four CTAs per SM in all
     dp.replicas = (4 * h->n_sm + nchunk - 1) / nchunk;
     if (dp.replicas > 64) dp.replicas = 64;
-    MOE_TRY(launch_dispatch(dp, s));
+    if (h->fp8)
+        MOE_TRY(launch_dispatch_fp8(dp, h->xq, h->xs, s));
+    else
+        MOE_TRY(launch_dispatch(dp, s));
     MOE_MARK();
 
     GroupedParams gp;
@@ -365,7 +405,14 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     gp.E = h->E; gp.d = h->d; gp.I = h->I; gp.k = h->k; gp.rows_cap = h->rows_cap;
     const int max_mtiles = (N * h->k + tile_m - 1) / tile_m + h->E;
 
-    if (fused) {
+    if (h->fp8) {
+        Fp8ExpertParams fp;
+        fp.offsets = h->offsets; fp.sgu = h->w.w_gate_up_scale; fp.sdn = h->w.w_down_scale;
+        fp.xs = h->xs; fp.aq = h->aq; fp.as = h->as; fp.y = h->y; fp.sched = h->sched;
+        fp.status = h->status; fp.E = h->E; fp.d = h->d; fp.I = h->I;
+        MOE_TRY(launch_fp8_experts(h->fp8_maps, fp, h->n_sm, s));
+        MOE_MARK();
+    } else if (fused) {
         DecodeParams fp;
         fp.offsets = h->offsets; fp.act = h->act; fp.y = h->y; fp.sched = h->sched;
         fp.status = h->status; fp.E = h->E; fp.d = h->d; fp.I = h->I;
@@ -395,7 +442,7 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     cp.x = x; cp.y = h->y; cp.wts = h->wts; cp.inv = h->inv; cp.out = out; cp.status = h->status;
     cp.chunk_hist = h->chunk_hist; cp.chunk_hist_n = nchunk * h->E;
     cp.N = N; cp.d = h->d; cp.k = h->k;
-    MOE_TRY(launch_combine(cp, h->dtype, s));
+    MOE_TRY(launch_combine(cp, h->xdtype, s));
     MOE_MARK();
 #undef MOE_MARK
 #undef MOE_TRY
@@ -449,6 +496,7 @@ extern "C" int moe_destroy(moe_ctx *h) {
     if (cudaDeviceSynchronize() != cudaSuccess) rc = MOE_ERR_CUDA;
     free_ring(h);
     if (h->decode_maps) decode_free_maps(h->decode_maps);
+    if (h->fp8_maps) fp8_free_maps(h->fp8_maps);
     if (cudaFree(h->ws) != cudaSuccess) rc = MOE_ERR_CUDA;
     delete h;
     return rc;
@@ -482,6 +530,20 @@ extern "C" int moe_debug_routing(moe_ctx *h, int32_t *idx, float *w, int32_t *pe
     return MOE_OK;
 }
 
+extern "C" int moe_debug_fp8_rows(moe_ctx *h, uint8_t *codes, float *scales, void *stream) {
+    if (!h || !h->fp8) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t rows = static_cast<size_t>(h->last_n) * h->k;
+    if (codes && rows &&
+        cudaMemcpyAsync(codes, h->xq, rows * h->d, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (scales && rows &&
+        cudaMemcpyAsync(scales, h->xs, rows * (h->d / kFp8Block) * 4, cudaMemcpyDeviceToDevice,
+                        s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 extern "C" int moe_profile(moe_ctx *h, int enable) {
     if (!h) return MOE_ERR_INVALID_ARG;
     if (enable && h->ring.empty()) {
@@ -490,7 +552,6 @@ extern "C" int moe_profile(moe_ctx *h, int enable) {
             if (cudaEventCreate(&h->ring[i]) != cudaSuccess) {
                 h->ring.resize(i);
                 free_ring(h);
-    if (h->decode_maps) decode_free_maps(h->decode_maps);
                 return MOE_ERR_CUDA;
             }
         }

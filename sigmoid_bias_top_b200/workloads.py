@@ -17,6 +17,15 @@ Tensor layout (what the C ABI consumes):
   bias       [E]           f32           expert bias (selection only)
   w_gate_up  [E, 2I, d]    f32 or bf16   rows 0..I-1 = gate, rows I..2I-1 = up
   w_down     [E, d, I]     f32 or bf16   down projection
+FP8_BLOCK workloads (dtype "fp8"; the FP8 checkpoint of "LFM2.5-24B-A2B",
+German page, section "Quantisierung") keep x bf16 and store the expert
+matrices as e4m3 codes (torch.float8_e4m3fn) with fp32 block scales:
+  w_gate_up_scale [E, 2I/128, d/128]   w_down_scale [E, d/128, I/128]
+The codes are normal draws of standard deviation fp8_code_std cast to e4m3
+(saturating at 448) and every block scale is std / fp8_code_std times a
+uniform factor in (0.9, 1.1), so that code * scale has the std of the bf16
+workloads' weights; for N(0, std) blocks of 128 x 128 values a static
+amax / 448 scale would put the codes at about this spread.
 Distribution parameters written "N(0, v)" with v a fraction of the width
 (1/256, 1/192) are variances; "N(0, 0.02)" is a standard deviation, the usual
 initializer-range convention.
@@ -38,7 +47,7 @@ class Workload:
     n_experts: int
     top_k: int
     d_ff: int
-    dtype: str                      # "f32" or "bf16": x, out and expert weights
+    dtype: str                      # "f32", "bf16" (x, out, experts) or "fp8" (bf16 x)
     eps: float = 1e-6
     routed_scale: float = 1.0
     n_layers: int = 1
@@ -56,9 +65,11 @@ class Workload:
     zipf_scale: float = 0.08
     zipf_tail: int = 4
     zipf_tail_drop: float = 0.15
+    fp8_code_std: float = 109.0
 
     @property
     def torch_dtype(self) -> torch.dtype:
+        """Storage type of x and out."""
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
 
     def scaled(self, **kw) -> "Workload":
@@ -102,9 +113,14 @@ VERIFY = Workload(
     top_k=4, d_ff=1536, dtype="bf16", seed=6, gain_jitter=0.02, router_std=0.02,
     bias_kind="uniform", bias_halfwidth=0.05)
 
+# The decode and prefill steps with the FP8 checkpoint's FP8_BLOCK experts.
+DECODE_FP8 = DECODE.scaled(name="decode_fp8_N32_d2048_E64_k4_I1536", dtype="fp8", seed=7)
+PREFILL_FP8 = PREFILL.scaled(name="prefill_fp8_N8192_d2048_E64_k4_I1536", dtype="fp8", seed=8)
+
 WORKLOADS: Dict[str, Workload] = {
     "tiny": TINY_F32, "decode": DECODE, "prefill": PREFILL, "skewed": SKEWED,
-    "stacked": STACKED, "verify": VERIFY,
+    "stacked": STACKED, "verify": VERIFY, "decode_fp8": DECODE_FP8,
+    "prefill_fp8": PREFILL_FP8,
 }
 
 
@@ -159,7 +175,18 @@ def make_layer(w: Workload, layer: int = 0, device="cpu",
         raise ValueError(w.bias_kind)
     out = {"norm_gain": gain.contiguous(), "router_w": router_w.contiguous(),
            "bias": bias.contiguous()}
-    if with_experts:
+    if with_experts and w.dtype == "fp8":
+        cs = w.fp8_code_std
+        for name, shape, std in (("w_gate_up", (E, 2 * I, d), w.gate_up_std),
+                                 ("w_down", (E, d, I), w.down_std)):
+            codes = (torch.randn(shape, generator=g, device=device, dtype=torch.float32) * cs)
+            out[name] = codes.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).contiguous()
+            del codes
+            blocks = (E, -(-shape[1] // 128), -(-shape[2] // 128))
+            out[name + "_scale"] = ((0.9 + 0.2 * torch.rand(blocks, generator=g, device=device,
+                                                             dtype=torch.float32))
+                                    * (std / cs)).contiguous()
+    elif with_experts:
         out["w_gate_up"] = _normal((E, 2 * I, d), w.gate_up_std, g, device, dt).contiguous()
         out["w_down"] = _normal((E, d, I), w.down_std, g, device, dt).contiguous()
     return out

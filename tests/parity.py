@@ -12,8 +12,17 @@ Rules (the tolerances the tests assert):
   * the dispatch permutation and offsets equal the oracle's counting sort of
     the GPU's own selection, exactly;
   * mixture weights agree to 1e-5 relative (fp32 sigmoid vs fp64);
-  * outputs: per token ||o_gpu - o_ref|| / ||o_ref|| <= 1e-2 for bf16 storage,
-    1e-5 for fp32 storage.
+  * outputs: per token ||o_gpu - o_ref|| / ||o_ref|| <= 1e-2 for bf16 storage
+    (FP8_BLOCK layers store x and out as bf16 too), 1e-5 for fp32 storage;
+  * FP8_BLOCK layers also bound the MoE part alone: per token
+    ||(o_gpu - x) - (o_ref - x)|| / ||o_ref - x|| <= 2e-2 + 2^-8 ||o_ref|| /
+    ||o_ref - x||. The oracle applies the same e4m3 quantisation, so what
+    remains is fp32 summation order, the bf16 rounding of the expert outputs,
+    the rare e4m3 code that rounds the other way because the two sides' fp32
+    inputs differ in the last bits (one code step is 1/16 of one value out of
+    128), and the bf16 rounding of out itself, at most 2^-8 of |out| per
+    element, which the second term admits (it dominates when the MoE part is
+    small beside the residual).
 """
 from __future__ import annotations
 
@@ -24,7 +33,8 @@ import oracle
 
 MARGIN = 1e-3
 ORDER_GAP = 1e-5   # selected experts closer than this may swap slots under fp32 rounding
-TOL = {"bf16": 1e-2, "f32": 1e-5}
+TOL = {"bf16": 1e-2, "f32": 1e-5, "fp8": 1e-2}
+DELTA_TOL = {"fp8": 2e-2}
 W_RTOL = 1e-5
 
 
@@ -88,6 +98,12 @@ def check_outputs(x_cpu, layer_cpu, k, eps, scale, out_gpu, idx, tokens, dtype):
     worst = int(np.argmax(err))
     assert err.max() <= tol, (f"max rel-L2 {err.max():.3e} > {tol} at token {tokens[worst]}; "
                               f"MoE-delta rel err {delta_err[worst]:.3e}")
+    if dtype in DELTA_TOL:
+        dn = np.maximum(np.linalg.norm(ref["out"] - x, axis=1), 1e-30)
+        allowed = DELTA_TOL[dtype] + 2.0 ** -8 * np.linalg.norm(ref["out"], axis=1) / dn
+        wd = int(np.argmax(delta_err / allowed))
+        assert np.all(delta_err <= allowed), (
+            f"MoE-delta rel-L2 {delta_err[wd]:.3e} > {allowed[wd]:.3e} at token {tokens[wd]}")
     return float(err.max()), float(delta_err.max())
 
 

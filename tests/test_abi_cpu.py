@@ -63,6 +63,14 @@ def test_create_validates_before_touching_the_device():
     assert _create(2048, 64, 1536, 4, _weights(dtype=7))[0] == -1
     assert _create(2048, 64, 1536, 4, _weights(ptr=258))[0] == -3  # misaligned
     assert _create(2048, 64, 1536, 4, _weights(ptr=0))[0] == -1    # null
+    # FP8_BLOCK: whole 128 x 128 scale blocks, both scale arrays given and aligned
+    f8 = _weights(dtype=sb.MOE_FP8_BLOCK)
+    assert _create(2048, 64, 1536, 4, f8)[0] == -1               # no block scales
+    f8.w_gate_up_scale, f8.w_down_scale = 256, 256
+    assert _create(2112, 64, 1536, 4, f8)[0] == -2               # d % 128
+    assert _create(2048, 64, 1600, 4, f8)[0] == -2               # I % 128
+    f8.w_down_scale = 260
+    assert _create(2048, 64, 1536, 4, f8)[0] == -3               # misaligned scales
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")

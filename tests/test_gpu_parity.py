@@ -366,3 +366,97 @@ def test_fp32_widest_rows():
                           router_std=1.0 / 181.0, gate_up_std=1.0 / 181.0, down_std=0.25)
     m, x, layer, out, r = run(w)
     full_check(w, x, layer, out, r)
+
+
+# ---------------------------------------------------------------- FP8_BLOCK
+# The FP8 checkpoint's experts ("LFM2.5-24B-A2B", flozi.net, German page,
+# section "Quantisierung"): e4m3 weights in 128x128 blocks, activations
+# quantised per group of 128 inside the forward.
+
+def fp8_small(**kw):
+    """Small FP8_BLOCK shapes with weights of std 1/sqrt(K), so that the MoE
+    part of out is as large as the residual and its error is measurable."""
+    d, I = kw["d"], kw["d_ff"]
+    return W.DECODE_FP8.scaled(router_std=0.05, gate_up_std=d ** -0.5, down_std=I ** -0.5, **kw)
+
+
+def test_fp8_decode_full():
+    """The 32-token decode step with FP8_BLOCK experts, every token."""
+    w = W.DECODE_FP8
+    m, x, layer, out, r = run(w)
+    assert m.launches_per_forward(w.n_tokens) == 4
+    res = full_check(w, x, layer, out, r)
+    assert (res["counts"] > 0).sum() >= 45
+
+
+@pytest.mark.parametrize("n_experts,top_k,d,d_ff,n", [(8, 2, 256, 256, 100), (16, 4, 384, 640, 333),
+                                                      (4, 4, 128, 128, 1)])
+def test_fp8_ragged(n_experts, top_k, d, d_ff, n):
+    """Ragged FP8_BLOCK shapes: passes of 64 tokens with ragged tails, several
+    K blocks of both contractions, k = E, a single token."""
+    w = fp8_small(n_experts=n_experts, top_k=top_k, d=d, d_ff=d_ff, n_tokens=n)
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r)
+
+
+def test_fp8_one_expert_takes_all():
+    """One expert receives all 700 tokens (11 passes of 64 per item, the
+    others empty): the act rows of many passes before the down items."""
+    w = fp8_small(n_experts=8, top_k=1, d=256, d_ff=384, n_tokens=700)
+    layer = W.make_layer(w, 0, DEV)
+    layer["bias"] = torch.zeros_like(layer["bias"])
+    layer["bias"][5] = 5.0
+    m, x, layer, out, r = run(w, layer=layer)
+    res = full_check(w, x, layer, out, r)
+    assert res["counts"][5] == 700
+
+
+def test_fp8_quantised_rows_match_the_oracle():
+    """The dispatch's e4m3 rows: each grouped row holds the codes and group
+    scales of its token's normalised row (oracle RMSNorm, quantised by the
+    oracle). Scales agree to fp32 rounding; a code may differ only by one
+    step, where v / s lies within a hair of a rounding midpoint."""
+    import oracle
+    w = W.DECODE_FP8.scaled(n_tokens=96)
+    m, x, layer, out, r = run(w)
+    q = m.debug_fp8_rows(w.n_tokens)
+    torch.cuda.synchronize()
+    perm = r["perm"].cpu().numpy()
+    tok = perm // w.top_k
+    xn = oracle.rmsnorm(x.cpu(), layer["norm_gain"].cpu(), w.eps)
+    ref = oracle.quant(xn[tok])
+    np.testing.assert_allclose(q["scales"].cpu().numpy(), ref["scales"], rtol=2e-6)
+    codes = q["codes"].cpu().numpy()
+    same = codes == ref["codes"]
+    assert same.mean() > 0.999, same.mean()
+    vals_g = oracle.e4m3_value(codes[~same])
+    vals_r = oracle.e4m3_value(ref["codes"][~same])
+    s = np.repeat(ref["scales"], 128, axis=1)[~same]
+    v = xn[tok][~same] / s
+    # both neighbours of v: the two codes bracket v and v sits near their midpoint
+    assert np.all(np.minimum(vals_g, vals_r) <= v + 1e-6 * np.abs(v)), "code not adjacent"
+    assert np.all(np.maximum(vals_g, vals_r) >= v - 1e-6 * np.abs(v)), "code not adjacent"
+    mid = (vals_g + vals_r) / 2
+    assert np.all(np.abs(v - mid) <= 1e-5 * np.abs(v) + 1e-12), "flip away from a midpoint"
+
+
+def test_fp8_prefill_sampled():
+    """8192 tokens with FP8_BLOCK experts (about 512 rows per expert: eight
+    passes per weight tile) on sampled tokens."""
+    w = W.PREFILL_FP8
+    m, x, layer, out, r = run(w)
+    full_check(w, x, layer, out, r, tokens="sample")
+
+
+def test_fp8_deterministic_and_in_place():
+    w = W.DECODE_FP8.scaled(n_tokens=200)
+    layer = W.make_layer(w, 0, DEV)
+    x = W.make_x(w, DEV)
+    m = MoeLayer(layer, w.top_k, w.eps, max_tokens=w.n_tokens)
+    a = m(x)
+    b = m(x)
+    xi = x.clone()
+    m(xi, out=xi)
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    assert torch.equal(a, b) and torch.equal(a, xi)
