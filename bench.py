@@ -38,7 +38,7 @@ from sigmoid_bias_top_b200 import workloads as W  # noqa: E402
 METRIC = "MoE-layer tokens/s (d2048,E64,top4,I1536) + % of HBM / bf16 TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DEFAULT_STEPS = {"decode": 2000, "prefill": 200, "skewed": 100, "stacked": 20, "tiny": 2000,
-                 "verify": 1000}
+                 "verify": 1000, "decode_fp8": 2000, "prefill_fp8": 100}
 ROTATE = 4  # distinct weight copies cycled through (each step reads >= 1 GB > L2)
 
 
@@ -301,9 +301,13 @@ def run_ours(args, w, world, rank, local):
     U = float(np.mean(active))
     n_assign = N * w.top_k
     bpe = 2 if w.dtype == "bf16" else 4
+    fp8 = w.dtype == "fp8"
+    tc_peak_key = "bf16_tflops_sustained"
     if N * w.top_k / max(U, 1) < 64:  # weight-streaming regime: HBM-bound
         bound = "hbm"
-        if dom == "experts":   # both contractions in one launch
+        if fp8:                # FP8_BLOCK: both contractions in one launch
+            work = A.fp8_experts_bytes(U, n_assign, w.d, w.d_ff)
+        elif dom == "experts":   # both contractions in one launch
             work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + A.down_bytes(U, w.d, w.d_ff, bpe)
                     + 2 * n_assign * (w.d + w.d_ff) * bpe)
         elif dom == "gate_up":
@@ -317,10 +321,16 @@ def run_ours(args, w, world, rank, local):
         unit = "GB/s"
     else:
         bound = "tensor"
-        work = (A.gate_up_flops(n_assign, w.d, w.d_ff) if dom == "gate_up"
-                else A.down_flops(n_assign, w.d, w.d_ff))
+        if dom == "experts":
+            work = A.gate_up_flops(n_assign, w.d, w.d_ff) + A.down_flops(n_assign, w.d, w.d_ff)
+        else:
+            work = (A.gate_up_flops(n_assign, w.d, w.d_ff) if dom == "gate_up"
+                    else A.down_flops(n_assign, w.d, w.d_ff))
         achieved = work / (mean_ms[dom] / 1e3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        if fp8:  # e4m3 dense peak = the measured bf16 peak x the nominal 4.5 / 2.25
+            peak *= 2.0
+            tc_peak_key = "bf16_tflops_sustained x 2 (e4m3 / bf16 nominal ratio)"
         unit = "TFLOP/s"
     traffic = traffic_from_profiles(dom, args.workload)
     launches = mods[0].launches_per_forward(N) * args.steps * (len(mods) if w.n_layers > 1 else 1)
@@ -328,11 +338,13 @@ def run_ours(args, w, world, rank, local):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": w.dtype, "data": "synthetic (seeded; random-init weights of the layer's shapes)",
+        "dtype": "e4m3" if fp8 else w.dtype,
+        "data": "synthetic (seeded; random-init weights of the layer's shapes)",
         "config": {"workload": w.name, "tokens_per_gpu": N, "layers": w.n_layers,
                    "d": w.d, "experts": w.n_experts, "top_k": w.top_k, "d_ff": w.d_ff,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": (f"weights rotate over {n_rot} copies, >= 1 GB read per step (> 126 MB L2)"
+                   "l2": (f"weights rotate over {n_rot} copies; each step streams one copy's "
+                          "active experts, >= 0.5 GB (> 126 MB L2)"
                           if w.n_layers == 1 else "38 distinct layers, 45.9 GB per step (> L2)"),
                    "active_experts_per_layer": U},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
@@ -340,7 +352,7 @@ def run_ours(args, w, world, rank, local):
         "gpu_launches": launches,
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": unit, "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
+                     "peak_source": f"{src} ({'hbm_gbs' if bound == 'hbm' else tc_peak_key})",
                      "work_per_launch": work},
         "kernel_ms": per_layer,
         "clocks": clk,

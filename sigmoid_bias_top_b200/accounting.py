@@ -51,3 +51,23 @@ def gate_up_flops(n_assign: int, d: int, d_ff: int) -> int:
 
 def down_flops(n_assign: int, d: int, d_ff: int) -> int:
     return 2 * n_assign * d * d_ff
+
+
+# FP8_BLOCK experts ("LFM2.5-24B-A2B", German page, section "Quantisierung":
+# weights FP8 in static 128x128 blocks, activations FP8 per group of 128).
+
+def fp8_scale_bytes(active_experts: int, d: int, d_ff: int) -> int:
+    """fp32 block scales of the active experts' gate/up and down matrices."""
+    blocks = (-(-2 * d_ff // 128)) * (-(-d // 128)) + (-(-d // 128)) * (-(-d_ff // 128))
+    return active_experts * blocks * 4
+
+
+def fp8_experts_bytes(active_experts: int, n_assign: int, d: int, d_ff: int) -> int:
+    """Bytes the FP8 expert kernel (both contractions in one launch) must
+    move: e4m3 weights (1 byte each) and their block scales; the grouped e4m3
+    input rows and their group scales read; SiLU(gate)*up codes and scales
+    written and read back; the bf16 expert outputs written."""
+    rows_in = n_assign * (d + 4 * (-(-d // 128)))
+    act = 2 * n_assign * (d_ff + 4 * (-(-d_ff // 128)))
+    return (active_experts * expert_weights(d, d_ff) + fp8_scale_bytes(active_experts, d, d_ff)
+            + rows_in + act + n_assign * d * 2)

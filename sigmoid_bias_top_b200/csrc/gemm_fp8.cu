@@ -24,13 +24,15 @@
 // the end of a pass:
 //   gate/up: a = SiLU(gate) * up per (token, row); the item's 128 rows are
 //     exactly one activation group of 128, so the group maximum is a max over
-//     the 128 epilogue threads (warp butterflies, then four warps through
-//     shared memory, met at an mbarrier), s = amax / 448 and the codes
+//     the 128 TMEM lanes (a warp redux per column, then the four lane
+//     quadrants through shared memory, met at an mbarrier), s = amax / 448 and the codes
 //     e4m3(a / s) (nearest-even, saturating) go to aq with s in as;
 //   down: y = the fp32 sum, rounded once to bf16.
-// Roles per CTA (192 threads): warp 0 lane 0 claims items and issues TMA;
-// warp 1 owns TMEM (512 columns) and one thread issues the MMAs; warps 2..5
-// are the epilogue. All waits are bounded (1 s) and report
+// Roles per CTA (320 threads): warp 0 lane 0 claims items and issues TMA;
+// warp 1 owns TMEM (512 columns) and one thread issues the MMAs; warps 2..9
+// are the epilogue, two per TMEM lane quadrant, each promoting 16 columns of
+// every token tile; the per-column scale products sa * sw of a K block are
+// formed once per lane and read back from shared memory as float4s. All waits are bounded (1 s) and report
 // MOE_ERR_DEVICE_TIMEOUT; on time-out the kernel drains its own copies and
 // MMAs, frees TMEM and returns.
 #include <cuda_fp8.h>
@@ -44,22 +46,35 @@ namespace {
 
 constexpr int WM = 128;              // weight rows per item (MMA M)
 constexpr int TT = 32;               // tokens per token tile
-constexpr int MAXT = 2;              // token tiles per pass (N = 32 or 64)
-constexpr int NP = TT * MAXT;        // tokens per pass
 constexpr int BK = kFp8Block;        // K per stage: one scale block, 128 bytes per row
 constexpr int UK = 32;               // K per tcgen05.mma kind::f8f6f4
 constexpr int STAGES = 5;
-constexpr int A_BYTES = WM * BK;                         // 16 KB weight tile
-constexpr int B_TILE = TT * BK;                          // 4 KB token tile
-constexpr int STAGE_BYTES = 2 * A_BYTES + MAXT * B_TILE; // 40 KB
-constexpr int BUF_COLS = 2 * NP;     // TMEM columns per K-block buffer: gate 0..63, up 64..127
-constexpr int NBUF = 4;
-constexpr int TMEM_COLS = NBUF * BUF_COLS;  // 512
+constexpr int A_BYTES = WM * BK;     // 16 KB weight tile
+constexpr int B_TILE = TT * BK;      // 4 KB token tile
+constexpr int TMEM_COLS = 512;
 constexpr int RING = 4;
-constexpr int kThreads = 192;
+
+// Sizes that follow from MAXT, the token tiles per pass (1 for small batches,
+// 2 otherwise): a K block's partials take 2 * NP TMEM columns (gate, up), so
+// fewer tokens per pass leave more K-block buffers for the tensor cores to
+// run ahead of the epilogue (8 instead of 4).
+template <int MAXT>
+struct Shape {
+    static constexpr int NP = TT * MAXT;                          // tokens per pass
+    static constexpr int STAGE_BYTES = 2 * A_BYTES + MAXT * B_TILE;
+    static constexpr int BUF_COLS = 2 * NP;                       // gate 0..NP-1, up NP..
+    static constexpr int NBUF = TMEM_COLS / BUF_COLS;
+};
+constexpr int kEpiWarps = 8;         // two per TMEM lane quadrant
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int CW = 16;               // columns of each token tile per epilogue warp
+constexpr int TBL_KB = 8;            // K blocks per chunk of the epilogue's scale table
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
+template <int MAXT>
 struct Ctl {
+    static constexpr int NBUF = Shape<MAXT>::NBUF, NP = Shape<MAXT>::NP;
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tfull[NBUF];
@@ -69,29 +84,40 @@ struct Ctl {
     uint64_t pub;        // every epilogue thread's act rows of an item are stored
     uint64_t red_bar[2]; // the four epilogue warps' column maxima are in red[b]
     uint64_t drain;
-    float red[2][4][NP]; // per epilogue warp, per token column: max |a| over its 32 rows
+    float red[2][4][NP]; // per lane quadrant, per token column: max |a| over its 32 rows
+    // per epilogue warp, per K block of the current chunk: sa[col] * sw of
+    // each of the warp's MAXT * CW columns, for gate (0) and up (1)
+    float4 tbl[kEpiWarps][2][TBL_KB][MAXT * CW / 4];
     int ring_item[RING];
     int ring_pass[RING];
     uint32_t tmem_base;
     int abort;
 };
 
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, int *status) {
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *abort_flag,
+                                         int *status) {
     if (mbar_try_wait(bar, parity)) return true;
     if (mbar_wait(bar, parity, globaltimer_ns() + kWaitNs)) return true;
     set_status(status, kStatusTimeout);
-    atomicExch(&ctl->abort, 1);
+    atomicExch(abort_flag, 1);
     return false;
 }
 
-__device__ __forceinline__ bool aborted(Ctl *ctl) {
-    return *reinterpret_cast<volatile int *>(&ctl->abort) != 0;
+__device__ __forceinline__ bool aborted(int *abort_flag) {
+    return *reinterpret_cast<volatile int *>(abort_flag) != 0;
 }
 
 __device__ __forceinline__ int ld_acquire(const int *p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Brings the bytes [p, p + bytes) into L2 (no registers written).
+__device__ __forceinline__ void prefetch_l2(const void *p, int bytes) {
+    const char *c = static_cast<const char *>(p);
+    for (int o = 0; o < bytes; o += 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(c + o));
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -106,8 +132,10 @@ struct Unit {
     bool last_pass;
 };
 
+template <int MAXT>
 __device__ __forceinline__ Unit decode(int item, int pass, int n_gu_tiles, int n_dn_tiles, int E,
                                        const int32_t *offs) {
+    constexpr int NP = Shape<MAXT>::NP;
     Unit u;
     const int n_gu = E * n_gu_tiles;
     u.gate_up = item < n_gu;
@@ -123,6 +151,54 @@ __device__ __forceinline__ Unit decode(int item, int pass, int n_gu_tiles, int n
     return u;
 }
 
+// One epilogue step: NKB consecutive K blocks (TMEM buffers buf, buf+1, ...)
+// of NT token tiles, gate and up (GU) or down only: every partial times its
+// column's scale product from the table row of that K block, added into the
+// fp32 accumulators. Per token tile, the loads of all NKB blocks are issued
+// before one wait.
+template <int MAXT, bool GU, int NT, int NKB>
+__device__ __forceinline__ void promote(uint32_t t0, int buf, const float4 (*tg)[MAXT * CW / 4],
+                                        const float4 (*tu)[MAXT * CW / 4], float (&accg)[NT * CW],
+                                        float (&accu)[NT * CW]) {
+    constexpr int NP = Shape<MAXT>::NP, NBUF = Shape<MAXT>::NBUF, BUF_COLS = Shape<MAXT>::BUF_COLS;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        uint32_t g[NKB][16], v[NKB][16];
+#pragma unroll
+        for (int k = 0; k < NKB; ++k) {
+            const uint32_t tb = t0 + static_cast<uint32_t>(((buf + k) % NBUF) * BUF_COLS);
+            tmem_ld_32x32b_x16(tb + t * TT, g[k]);
+            if (GU) tmem_ld_32x32b_x16(tb + NP + t * TT, v[k]);
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < NKB; ++k)
+#pragma unroll
+            for (int c4 = 0; c4 < CW / 4; ++c4) {
+                const float4 sg = tg[k][t * (CW / 4) + c4];
+                const int c = t * CW + 4 * c4;
+                accg[c + 0] = fmaf(__uint_as_float(g[k][4 * c4 + 0]), sg.x, accg[c + 0]);
+                accg[c + 1] = fmaf(__uint_as_float(g[k][4 * c4 + 1]), sg.y, accg[c + 1]);
+                accg[c + 2] = fmaf(__uint_as_float(g[k][4 * c4 + 2]), sg.z, accg[c + 2]);
+                accg[c + 3] = fmaf(__uint_as_float(g[k][4 * c4 + 3]), sg.w, accg[c + 3]);
+                if (GU) {
+                    const float4 su = tu[k][t * (CW / 4) + c4];
+                    accu[c + 0] = fmaf(__uint_as_float(v[k][4 * c4 + 0]), su.x, accu[c + 0]);
+                    accu[c + 1] = fmaf(__uint_as_float(v[k][4 * c4 + 1]), su.y, accu[c + 1]);
+                    accu[c + 2] = fmaf(__uint_as_float(v[k][4 * c4 + 2]), su.z, accu[c + 2]);
+                    accu[c + 3] = fmaf(__uint_as_float(v[k][4 * c4 + 3]), su.w, accu[c + 3]);
+                }
+            }
+    }
+}
+
+// Per-thread state of an epilogue warp across units.
+struct EpiState {
+    int ew, q, h2, r, lt, lcol;  // warp index, TMEM lane quadrant, column half, row, lane column
+    uint32_t tmem_base;
+    uint32_t nblk, npub, nred;   // K blocks consumed; phases of ctl->pub and ctl->red_bar
+};
+
 struct Fp8Maps {
     CUtensorMap w_gate_up;  // e4m3 [E*2I][d] box 128 x 128
     CUtensorMap w_down;     // e4m3 [E*d][I]  box 128 x 128
@@ -130,12 +206,169 @@ struct Fp8Maps {
     CUtensorMap aq;         // e4m3 [rows][I] box 128 x 32
 };
 
+
+// The epilogue's work on one unit (item, pass) with NT = u.ntt token tiles:
+// the K loop (scale table per chunk of TBL_KB blocks, promotion of every
+// block), then the pass's output: bf16 y rows (down) or the quantised
+// SiLU(gate)*up codes and group scales (gate/up), published after the last
+// pass. Returns false after a timed-out wait (status and abort already set).
+template <int MAXT, int NT>
+__device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp8ExpertParams &p,
+                                         EpiState &st, int n_gu_tiles, int n_dn_tiles,
+                                         int *done) {
+    constexpr int NBUF = Shape<MAXT>::NBUF;
+    const int lane = threadIdx.x & 31;
+    const int ngd = p.d / kFp8Block, ngi = p.I / kFp8Block;
+    const int nk = (u.gate_up ? p.d : p.I) / BK;
+    // weight block scales of this item: row blocks of the gate and up tiles
+    // (gate/up) or of the Wd tile (down), one per K block
+    const float *swg = u.gate_up
+        ? p.sgu + (static_cast<size_t>(u.e) * (2 * n_gu_tiles) + u.tile) * ngd
+        : p.sdn + (static_cast<size_t>(u.e) * n_dn_tiles + u.tile) * ngi;
+    const float *swu = u.gate_up
+        ? p.sgu + (static_cast<size_t>(u.e) * (2 * n_gu_tiles) + n_gu_tiles + u.tile) * ngd
+        : swg;
+    const int ng = u.gate_up ? ngd : ngi;
+    // this lane's column: lanes 16..31 serve the second token tile, which
+    // exists in the two-tile shape only; its group scales (row of xs or as)
+    const bool lserve = st.lt < MAXT;
+    const bool lvalid = st.lt < NT && st.lcol < u.rows;
+    const float *sa_row = (u.gate_up ? p.xs : p.as) +
+                          static_cast<size_t>(u.row0 + (lvalid ? st.lcol : 0)) * ng;
+    float accg[NT * CW], accu[NT * CW];
+#pragma unroll
+    for (int c = 0; c < NT * CW; ++c) { accg[c] = 0.f; accu[c] = 0.f; }
+    const float4 (*tg)[MAXT * CW / 4] = ctl->tbl[st.ew][0];
+    const float4 (*tu)[MAXT * CW / 4] = ctl->tbl[st.ew][1];
+    const uint32_t tq = st.tmem_base + (static_cast<uint32_t>(st.q * 32) << 16) + st.h2 * CW;
+    for (int kb = 0; kb < nk;) {
+        if (kb % TBL_KB == 0) {
+            // the next chunk of the scale table: lane l writes column l's
+            // products for up to TBL_KB K blocks
+            const int n = min(TBL_KB, nk - kb);
+            __syncwarp();  // every lane is done with the previous chunk
+#pragma unroll
+            for (int j = 0; j < TBL_KB; ++j) {
+                float sg = 0.f, su = 0.f;
+                if (j < n) {
+                    const float sa = !lvalid ? 0.f
+                        : u.gate_up ? __ldg(sa_row + kb + j) : __ldcg(sa_row + kb + j);
+                    sg = sa * __ldg(swg + kb + j);
+                    if (u.gate_up) su = sa * __ldg(swu + kb + j);
+                }
+                if (lserve) {
+                    reinterpret_cast<float *>(ctl->tbl[st.ew][0][j])[lane] = sg;
+                    reinterpret_cast<float *>(ctl->tbl[st.ew][1][j])[lane] = su;
+                }
+            }
+            __syncwarp();
+        }
+        // two K blocks per step for one token tile while both lie in this chunk
+        const int nkb = (NT == 1 && kb + 1 < nk && (kb + 1) % TBL_KB != 0) ? 2 : 1;
+        const int buf = static_cast<int>(st.nblk % NBUF);
+        for (int k = 0; k < nkb; ++k)
+            if (!wait_bar(&ctl->tfull[(buf + k) % NBUF], ((st.nblk + k) / NBUF) & 1u, &ctl->abort, p.status))
+                return false;
+        tc_fence_after();
+        const int row = kb % TBL_KB;
+        if (u.gate_up) {
+            if (nkb == 2) promote<MAXT, true, NT, 2>(tq, buf, tg + row, tu + row, accg, accu);
+            else promote<MAXT, true, NT, 1>(tq, buf, tg + row, tu + row, accg, accu);
+        } else {
+            if (nkb == 2) promote<MAXT, false, NT, 2>(tq, buf, tg + row, tu + row, accg, accu);
+            else promote<MAXT, false, NT, 1>(tq, buf, tg + row, tu + row, accg, accu);
+        }
+        tc_fence_before();
+        for (int k = 0; k < nkb; ++k) mbar_arrive(&ctl->tempty[(buf + k) % NBUF]);
+        st.nblk += nkb;
+        kb += nkb;
+    }
+
+    if (!u.gate_up) {
+        __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.y);
+        const int f = u.tile * WM + st.r;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int c = 0; c < CW; ++c) {
+                const int col = t * TT + st.h2 * CW + c;
+                if (col < u.rows)
+                    y[static_cast<size_t>(u.row0 + col) * p.d + f] = __float2bfloat16_rn(accg[t * CW + c]);
+            }
+        return true;
+    }
+
+    // a = SiLU(gate) * up; group maximum per token column over the 128 rows:
+    // a warp maximum over the bits of |a| (non-negative floats order like
+    // their bit patterns), then the four lane quadrants
+#pragma unroll
+    for (int c = 0; c < NT * CW; ++c) {
+        const float gv = accg[c];
+        accg[c] = __fdividef(gv, 1.0f + __expf(-gv)) * accu[c];
+    }
+    float mine = 0.f;  // the warp maximum of column lcol
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+            const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(accg[t * CW + c])));
+            if (lane == t * 16 + c) mine = __uint_as_float(m);
+        }
+    const int rb = static_cast<int>(st.nred & 1u);
+    if (lserve) ctl->red[rb][st.q][st.lcol] = mine;
+    mbar_arrive(&ctl->red_bar[rb]);
+    if (!wait_bar(&ctl->red_bar[rb], (st.nred >> 1) & 1u, &ctl->abort, p.status)) return false;
+    ++st.nred;
+    float sl = 0.f;  // the scale of column lcol
+    if (lserve) {
+        const float amax = fmaxf(fmaxf(ctl->red[rb][0][st.lcol], ctl->red[rb][1][st.lcol]),
+                                 fmaxf(ctl->red[rb][2][st.lcol], ctl->red[rb][3][st.lcol]));
+        sl = __fdiv_rn(amax, 448.f);
+    }
+    if (st.q == 0 && lvalid) p.as[static_cast<size_t>(u.row0 + st.lcol) * ngi + u.tile] = sl;
+    const int f = u.tile * WM + st.r;
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+            const float sc = __shfl_sync(0xffffffffu, sl, t * 16 + c);
+            const int col = t * TT + st.h2 * CW + c;
+            if (col < u.rows) {
+                const uint8_t code = sc > 0.f
+                    ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(accg[t * CW + c], sc),
+                                                                 __NV_SATFINITE, __NV_E4M3))
+                    : static_cast<uint8_t>(0);
+                p.aq[static_cast<size_t>(u.row0 + col) * p.I + f] = code;
+            }
+        }
+    if (u.last_pass) {
+        // publish the expert's act rows to the down items of other CTAs:
+        // every thread fences its stores (also towards the async proxy that
+        // the TMA reads use) and arrives; one thread waits for all (bounded)
+        // and releases the per-expert counter
+        fence_proxy_async_global();
+        __threadfence();
+        mbar_arrive(&ctl->pub);
+        if (st.ew == 0 && lane == 0) {
+            if (wait_bar(&ctl->pub, st.npub & 1u, &ctl->abort, p.status)) {
+                __threadfence();
+                atomicAdd(done + u.e, 1);
+            }
+        }
+        ++st.npub;
+    }
+    return true;
+}
+
+template <int MAXT>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_experts_kernel(const __grid_constant__ Fp8Maps maps, Fp8ExpertParams p) {
+    constexpr int NP = Shape<MAXT>::NP, NBUF = Shape<MAXT>::NBUF;
+    constexpr int BUF_COLS = Shape<MAXT>::BUF_COLS, STAGE_BYTES = Shape<MAXT>::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    Ctl *ctl = reinterpret_cast<Ctl *>(smem + STAGES * STAGE_BYTES);
+    Ctl<MAXT> *ctl = reinterpret_cast<Ctl<MAXT> *>(smem + STAGES * STAGE_BYTES);
     int32_t *offs = reinterpret_cast<int32_t *>(ctl + 1);  // [E+1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -153,15 +386,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], 128);
+            mbar_init(&ctl->tempty[b], kEpiThreads);
         }
         for (int r = 0; r < RING; ++r) {
             mbar_init(&ctl->ufull[r], 1);
-            mbar_init(&ctl->uempty[r], 1 + 128);  // the MMA thread and every epilogue thread
+            mbar_init(&ctl->uempty[r], 1 + kEpiThreads);  // the MMA thread, every epilogue thread
         }
-        mbar_init(&ctl->pub, 128);
-        mbar_init(&ctl->red_bar[0], 128);
-        mbar_init(&ctl->red_bar[1], 128);
+        mbar_init(&ctl->pub, kEpiThreads);
+        mbar_init(&ctl->red_bar[0], kEpiThreads);
+        mbar_init(&ctl->red_bar[1], kEpiThreads);
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_mbar_init();
@@ -194,16 +427,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t issued_parity[STAGES];
             for (int i = 0; i < STAGES; ++i) issued[i] = false;
             bool ok = true;
-            while (ok && !aborted(ctl)) {
+            while (ok && !aborted(&ctl->abort)) {
                 const int item = atomicAdd(next_item, 1);
                 const bool stop = item >= total;
                 int npass = 0;
                 Unit u0;
                 if (!stop) {
-                    u0 = decode(item, 0, n_gu_tiles, n_dn_tiles, E, offs);
+                    u0 = decode<MAXT>(item, 0, n_gu_tiles, n_dn_tiles, E, offs);
                     const int cnt = offs[u0.e + 1] - offs[u0.e];
                     if (cnt <= 0) continue;  // expert without tokens: nothing to do
                     npass = (cnt + NP - 1) / NP;
+                    // the item's weight block scales, for the epilogue units to come
+                    const int ngd = p.d / kFp8Block, ngi = p.I / kFp8Block;
+                    if (u0.gate_up) {
+                        const float *sg = p.sgu + (static_cast<size_t>(u0.e) * (2 * n_gu_tiles) + u0.tile) * ngd;
+                        prefetch_l2(sg, ngd * 4);
+                        prefetch_l2(sg + static_cast<size_t>(n_gu_tiles) * ngd, ngd * 4);
+                    } else {
+                        prefetch_l2(p.sdn + (static_cast<size_t>(u0.e) * n_dn_tiles + u0.tile) * ngi, ngi * 4);
+                    }
                     if (!u0.gate_up) {
                         // the expert's act rows must be complete: all its gate/up items
                         const uint64_t dl = globaltimer_ns() + kWaitNs;
@@ -222,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 for (int pass = 0; pass < (stop ? 1 : npass); ++pass) {
                     const int slot = useq % RING;
-                    if (!wait_bar(&ctl->uempty[slot], ((useq / RING) & 1u) ^ 1u, ctl, p.status)) {
+                    if (!wait_bar(&ctl->uempty[slot], ((useq / RING) & 1u) ^ 1u, &ctl->abort, p.status)) {
                         ok = false;
                         break;
                     }
@@ -231,11 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&ctl->ufull[slot]);
                     ++useq;
                     if (stop) break;
-                    const Unit u = decode(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
+                    const Unit u = decode<MAXT>(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
                     const int nk = (u.gate_up ? p.d : p.I) / BK;
                     const uint32_t bytes = (u.gate_up ? 2 * A_BYTES : A_BYTES) + u.ntt * B_TILE;
                     for (int kb = 0; kb < nk; ++kb) {
-                        if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) { ok = false; break; }
+                        if (!wait_bar(&ctl->empty[s], ph ^ 1u, &ctl->abort, p.status)) { ok = false; break; }
                         uint8_t *sa = smem + s * STAGE_BYTES;
                         uint8_t *sb = sa + 2 * A_BYTES;
                         mbar_arrive_expect_tx(&ctl->full[s], bytes);
@@ -258,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (stop) break;
             }
-            if (!ok || aborted(ctl)) {
+            if (!ok || aborted(&ctl->abort)) {
                 // make the other roles leave, then let our own copies land
                 atomicExch(&ctl->abort, 1);
                 const uint64_t dl = globaltimer_ns() + kWaitNs;
@@ -274,21 +516,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             int useq = 0;
             uint32_t nblk = 0;  // K blocks issued: buffer nblk % NBUF
             bool any = false, ok = true;
-            while (ok && !aborted(ctl)) {
+            while (ok && !aborted(&ctl->abort)) {
                 const int slot = useq % RING;
-                if (!wait_bar(&ctl->ufull[slot], (useq / RING) & 1u, ctl, p.status)) break;
+                if (!wait_bar(&ctl->ufull[slot], (useq / RING) & 1u, &ctl->abort, p.status)) break;
                 const int item = ctl->ring_item[slot], pass = ctl->ring_pass[slot];
                 mbar_arrive(&ctl->uempty[slot]);
                 ++useq;
                 if (item < 0) break;
-                const Unit u = decode(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
+                const Unit u = decode<MAXT>(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
                 const uint32_t idesc = idesc_e4m3_f32(WM, TT * u.ntt);
                 const int nk = (u.gate_up ? p.d : p.I) / BK;
                 for (int kb = 0; kb < nk; ++kb) {
                     const int buf = static_cast<int>(nblk % NBUF);
                     const uint32_t use = nblk / NBUF;
-                    if (!wait_bar(&ctl->tempty[buf], (use & 1u) ^ 1u, ctl, p.status)) { ok = false; break; }
-                    if (!wait_bar(&ctl->full[s], ph, ctl, p.status)) { ok = false; break; }
+                    if (!wait_bar(&ctl->tempty[buf], (use & 1u) ^ 1u, &ctl->abort, p.status)) { ok = false; break; }
+                    if (!wait_bar(&ctl->full[s], ph, &ctl->abort, p.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * BUF_COLS);
                     const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
@@ -315,161 +557,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------- epilogue -------------------------
-        // thread <-> TMEM lane = weight row: warp w reads lanes 32*(w%4)..+31
-        const int q = warp & 3;
-        const int r = q * 32 + lane;
-        const int ngd = p.d / kFp8Block, ngi = p.I / kFp8Block;
+        // thread <-> TMEM lane = weight row: warp w reads lanes 32*(w%4)..+31;
+        // the two warps of a quadrant split every token tile's 32 columns into
+        // halves of CW. Lane l also serves one column for the lane-parallel
+        // work: lcol = tile (l / 16), column h2 * CW + l % 16 of that tile.
+        EpiState st;
+        st.ew = warp - 2;
+        st.q = warp & 3;
+        st.h2 = st.ew >> 2;
+        st.r = st.q * 32 + lane;
+        st.lt = lane >> 4;
+        st.lcol = st.lt * TT + st.h2 * CW + (lane & 15);
+        st.tmem_base = tmem_base;
+        st.nblk = st.npub = st.nred = 0;
         int useq = 0;
-        uint32_t nblk = 0;
-        uint32_t npub = 0, nred = 0;  // phases of ctl->pub and ctl->red_bar
         bool ok = true;
-        while (ok && !aborted(ctl)) {
+        while (ok && !aborted(&ctl->abort)) {
             const int slot = useq % RING;
-            if (!wait_bar(&ctl->ufull[slot], (useq / RING) & 1u, ctl, p.status)) break;
+            if (!wait_bar(&ctl->ufull[slot], (useq / RING) & 1u, &ctl->abort, p.status)) break;
             const int item = ctl->ring_item[slot], pass = ctl->ring_pass[slot];
             mbar_arrive(&ctl->uempty[slot]);
             ++useq;
             if (item < 0) break;
-            const Unit u = decode(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
-            const int nk = (u.gate_up ? p.d : p.I) / BK;
-            // weight block scales of this item: row blocks of the gate and up
-            // tiles (gate/up) or of the Wd tile (down), one per K block
-            const float *swg = u.gate_up
-                ? p.sgu + (static_cast<size_t>(u.e) * (2 * n_gu_tiles) + u.tile) * ngd
-                : p.sdn + (static_cast<size_t>(u.e) * n_dn_tiles + u.tile) * ngi;
-            const float *swu = u.gate_up
-                ? p.sgu + (static_cast<size_t>(u.e) * (2 * n_gu_tiles) + n_gu_tiles + u.tile) * ngd
-                : swg;
-            const int ng = u.gate_up ? ngd : ngi;
-            float accg[NP], accu[NP];
-#pragma unroll
-            for (int c = 0; c < NP; ++c) { accg[c] = 0.f; accu[c] = 0.f; }
-            for (int kb = 0; kb < nk; ++kb) {
-                // token group scales of this K block: lane c holds column c (+32)
-                float sa[MAXT];
-#pragma unroll
-                for (int t = 0; t < MAXT; ++t) {
-                    const int c = t * TT + lane;
-                    sa[t] = 0.f;
-                    if (c < u.rows) {
-                        const size_t gi = static_cast<size_t>(u.row0 + c) * ng + kb;
-                        sa[t] = u.gate_up ? p.xs[gi] : __ldcg(p.as + gi);
-                    }
-                }
-                const float wg = __ldg(swg + kb);
-                const float wu = u.gate_up ? __ldg(swu + kb) : 0.f;
-                const int buf = static_cast<int>(nblk % NBUF);
-                const uint32_t use = nblk / NBUF;
-                ++nblk;
-                if (!wait_bar(&ctl->tfull[buf], use & 1u, ctl, p.status)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t t0 = tmem_base + static_cast<uint32_t>(buf * BUF_COLS) +
-                                    (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll
-                for (int t = 0; t < MAXT; ++t) {
-                    if (t < u.ntt) {
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t g[16], v[16];
-                            tmem_ld_32x32b_x16(t0 + t * TT + h * 16, g);
-                            if (u.gate_up) tmem_ld_32x32b_x16(t0 + NP + t * TT + h * 16, v);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const float sc = __shfl_sync(0xffffffffu, sa[t], h * 16 + c);
-                                const int col = t * TT + h * 16 + c;
-                                accg[col] = fmaf(__uint_as_float(g[c]), sc * wg, accg[col]);
-                                if (u.gate_up)
-                                    accu[col] = fmaf(__uint_as_float(v[c]), sc * wu, accu[col]);
-                            }
-                        }
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&ctl->tempty[buf]);
-            }
-            if (!ok) break;
-
-            if (!u.gate_up) {
-                __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.y);
-                const int f = u.tile * WM + r;
-#pragma unroll
-                for (int c = 0; c < NP; ++c)
-                    if (c < u.rows)
-                        y[static_cast<size_t>(u.row0 + c) * p.d + f] = __float2bfloat16_rn(accg[c]);
-                continue;
-            }
-
-            // a = SiLU(gate) * up; group maximum per token column over the 128 rows
-            float mine[MAXT];
-#pragma unroll
-            for (int c = 0; c < NP; ++c) {
-                const float gv = accg[c];
-                accg[c] = gv / (1.0f + expf(-gv)) * accu[c];
-            }
-#pragma unroll
-            for (int t = 0; t < MAXT; ++t) {
-                mine[t] = 0.f;
-                if (t < u.ntt) {
-#pragma unroll
-                    for (int c = 0; c < TT; ++c) {
-                        float m = fabsf(accg[t * TT + c]);
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                        if (lane == c) mine[t] = m;
-                    }
-                }
-            }
-            const int rb = static_cast<int>(nred & 1u);
-#pragma unroll
-            for (int t = 0; t < MAXT; ++t) ctl->red[rb][q][t * TT + lane] = mine[t];
-            mbar_arrive(&ctl->red_bar[rb]);
-            if (!wait_bar(&ctl->red_bar[rb], (nred >> 1) & 1u, ctl, p.status)) break;
-            ++nred;
-            float sg[MAXT];  // lane c: the scale of column c (+32)
-#pragma unroll
-            for (int t = 0; t < MAXT; ++t) {
-                const int c = t * TT + lane;
-                const float m = fmaxf(fmaxf(ctl->red[rb][0][c], ctl->red[rb][1][c]),
-                                      fmaxf(ctl->red[rb][2][c], ctl->red[rb][3][c]));
-                sg[t] = __fdiv_rn(m, 448.f);
-                if (q == 0 && c < u.rows)
-                    p.as[static_cast<size_t>(u.row0 + c) * ngi + u.tile] = sg[t];
-            }
-            const int f = u.tile * WM + r;
-#pragma unroll
-            for (int t = 0; t < MAXT; ++t) {
-                if (t < u.ntt) {
-#pragma unroll
-                    for (int c = 0; c < TT; ++c) {
-                        const float sc = __shfl_sync(0xffffffffu, sg[t], c);
-                        const int col = t * TT + c;
-                        if (col < u.rows) {
-                            const uint8_t code = sc > 0.f
-                                ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(
-                                      __fdiv_rn(accg[col], sc), __NV_SATFINITE, __NV_E4M3))
-                                : static_cast<uint8_t>(0);
-                            p.aq[static_cast<size_t>(u.row0 + col) * p.I + f] = code;
-                        }
-                    }
-                }
-            }
-            if (u.last_pass) {
-                // publish the expert's act rows to the down items of other CTAs:
-                // every thread fences its stores (also towards the async proxy
-                // that the TMA reads use) and arrives; one thread waits for all
-                // 128 (bounded) and releases the per-expert counter
-                fence_proxy_async_global();
-                __threadfence();
-                mbar_arrive(&ctl->pub);
-                if (r == 0) {
-                    if (wait_bar(&ctl->pub, npub & 1u, ctl, p.status)) {
-                        __threadfence();
-                        atomicAdd(done + u.e, 1);
-                    }
-                }
-                ++npub;
-            }
+            const Unit u = decode<MAXT>(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
+            if (MAXT == 2 && u.ntt == 2)
+                ok = epi_unit<MAXT, MAXT>(u, ctl, p, st, n_gu_tiles, n_dn_tiles, done);
+            else
+                ok = epi_unit<MAXT, 1>(u, ctl, p, st, n_gu_tiles, n_dn_tiles, done);
         }
     }
 
@@ -482,7 +596,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-size_t smem_bytes(int E) { return 1024 + STAGES * STAGE_BYTES + sizeof(Ctl) + (E + 1) * 4; }
+template <int MAXT>
+size_t smem_bytes(int E) {
+    return 1024 + STAGES * Shape<MAXT>::STAGE_BYTES + sizeof(Ctl<MAXT>) + (E + 1) * 4;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -532,11 +649,29 @@ int fp8_build_maps(void **holder, const void *xq, const void *aq, const void *wg
 
 void fp8_free_maps(void *holder) { delete static_cast<Fp8MapsHolder *>(holder); }
 
-int launch_fp8_experts(const void *holder, const Fp8ExpertParams &p, int n_sm, cudaStream_t s) {
+namespace {
+template <int MAXT>
+int launch_t(const Fp8MapsHolder *h, const Fp8ExpertParams &p, int n_sm, cudaStream_t s) {
+    const size_t smem = smem_bytes<MAXT>(p.E);
+    if (ensure_smem(fp8_experts_kernel<MAXT>, smem) != MOE_OK) return MOE_ERR_CUDA;
+    // one CTA must fit an SM (registers and shared memory): checked once per size
+    thread_local size_t checked = 0;
+    if (checked != smem) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8_experts_kernel<MAXT>,
+                                                          kThreads, smem) != cudaSuccess ||
+            per_sm < 1)
+            return MOE_ERR_CUDA;
+        checked = smem;
+    }
+    return launch_k(fp8_experts_kernel<MAXT>, dim3(n_sm), dim3(kThreads), smem, s, h->m, p);
+}
+}  // namespace
+
+int launch_fp8_experts(const void *holder, const Fp8ExpertParams &p, int n_sm, int pass_tokens,
+                       cudaStream_t s) {
     const Fp8MapsHolder *h = static_cast<const Fp8MapsHolder *>(holder);
-    const size_t smem = smem_bytes(p.E);
-    if (ensure_smem(fp8_experts_kernel, smem) != MOE_OK) return MOE_ERR_CUDA;
-    return launch_k(fp8_experts_kernel, dim3(n_sm), dim3(kThreads), smem, s, h->m, p);
+    return pass_tokens <= TT ? launch_t<1>(h, p, n_sm, s) : launch_t<2>(h, p, n_sm, s);
 }
 
 }  // namespace moe

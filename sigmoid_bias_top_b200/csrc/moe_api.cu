@@ -410,7 +410,10 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
         fp.offsets = h->offsets; fp.sgu = h->w.w_gate_up_scale; fp.sdn = h->w.w_down_scale;
         fp.xs = h->xs; fp.aq = h->aq; fp.as = h->as; fp.y = h->y; fp.sched = h->sched;
         fp.status = h->status; fp.E = h->E; fp.d = h->d; fp.I = h->I;
-        MOE_TRY(launch_fp8_experts(h->fp8_maps, fp, h->n_sm, s));
+        // passes of 32 tokens (more TMEM buffers) while the mean load is small
+        const bool small = static_cast<long long>(N) * h->k <=
+                           static_cast<long long>(kDecodeRowsPerExpert) * h->E;
+        MOE_TRY(launch_fp8_experts(h->fp8_maps, fp, h->n_sm, small ? 32 : 64, s));
         MOE_MARK();
     } else if (fused) {
         DecodeParams fp;

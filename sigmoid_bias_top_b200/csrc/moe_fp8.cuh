@@ -37,7 +37,10 @@ int launch_dispatch_fp8(const DispatchParams &p, uint8_t *xq, float *xs, cudaStr
 int fp8_build_maps(void **holder, const void *xq, const void *aq, const void *wgu,
                    const void *wd, int rows_cap, int E, int d, int I);
 void fp8_free_maps(void *holder);
-int launch_fp8_experts(const void *holder, const Fp8ExpertParams &p, int n_sm, cudaStream_t s);
+// pass_tokens: tokens per pass of a weight tile, 32 (small batches: eight
+// TMEM buffers of K-block partials) or 64 (two token tiles, four buffers).
+int launch_fp8_experts(const void *holder, const Fp8ExpertParams &p, int n_sm, int pass_tokens,
+                       cudaStream_t s);
 
 // Instruction descriptor of kind::f8f6f4 with e4m3 A and B (both K-major) and
 // an fp32 accumulator, for an M x N tile (A/B format code 0 = E4M3).

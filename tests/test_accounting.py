@@ -34,3 +34,13 @@ def test_split_counts_add_up():
         8192 * A.expert_flops_per_token(2048, 1536, 4)
     assert A.gate_up_bytes(56, 2048, 1536) + A.down_bytes(56, 2048, 1536) == \
         56 * A.expert_weights(2048, 1536) * 2
+
+
+def test_fp8_bytes():
+    """One byte per e4m3 weight plus one fp32 scale per 128x128 block: the
+    2048 x 1536 expert has 24 x 16 gate/up blocks and 16 x 12 down blocks."""
+    assert A.fp8_scale_bytes(1, 2048, 1536) == (24 * 16 + 16 * 12) * 4
+    w = A.fp8_experts_bytes(56, 0, 2048, 1536)
+    assert w == 56 * (A.expert_weights(2048, 1536) + 2304)
+    assert A.fp8_experts_bytes(56, 128, 2048, 1536) - w == \
+        128 * (2048 + 64) + 2 * 128 * (1536 + 48) + 128 * 2048 * 2
