@@ -30,9 +30,10 @@
 //   down: y = the fp32 sum, rounded once to bf16.
 // Roles per CTA (320 threads): warp 0 lane 0 claims items and issues TMA;
 // warp 1 owns TMEM (512 columns) and one thread issues the MMAs; warps 2..9
-// are the epilogue, two per TMEM lane quadrant, each promoting 16 columns of
-// every token tile; the per-column scale products sa * sw of a K block are
-// formed once per lane and read back from shared memory as float4s. All waits are bounded (1 s) and report
+// are the epilogue, two per TMEM lane quadrant (two teams taking alternate
+// units, or both warps of a quadrant sharing each unit's columns: see Shape);
+// the per-column scale products sa * sw of up to eight K blocks are formed
+// once per lane into a shared-memory table and read back as float4s. All waits are bounded (1 s) and report
 // MOE_ERR_DEVICE_TIMEOUT; on time-out the kernel drains its own copies and
 // MMAs, frees TMEM and returns.
 #include <cuda_fp8.h>
@@ -53,23 +54,33 @@ constexpr int A_BYTES = WM * BK;     // 16 KB weight tile
 constexpr int B_TILE = TT * BK;      // 4 KB token tile
 constexpr int TMEM_COLS = 512;
 constexpr int RING = 4;
+constexpr int kEpiWarps = 8;         // two per TMEM lane quadrant
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int TBL_KB = 8;            // K blocks per chunk of the epilogue's scale table
+constexpr int kThreads = 64 + kEpiThreads;
 
 // Sizes that follow from MAXT, the token tiles per pass (1 for small batches,
 // 2 otherwise): a K block's partials take 2 * NP TMEM columns (gate, up), so
 // fewer tokens per pass leave more K-block buffers for the tensor cores to
 // run ahead of the epilogue (8 instead of 4).
+//
+// The epilogue warps: with one token tile per pass they form two teams of
+// four (one warp per TMEM lane quadrant) that take alternate units, each warp
+// covering all 32 columns, so that one team's end-of-pass work (SiLU,
+// quantisation, publication) and scale loads overlap the other team's K loop;
+// with two tiles the eight warps share every unit, the two warps of a
+// quadrant taking 16 columns of each tile (the registers of a 64-column warp
+// would not fit).
 template <int MAXT>
 struct Shape {
     static constexpr int NP = TT * MAXT;                          // tokens per pass
     static constexpr int STAGE_BYTES = 2 * A_BYTES + MAXT * B_TILE;
     static constexpr int BUF_COLS = 2 * NP;                       // gate 0..NP-1, up NP..
     static constexpr int NBUF = TMEM_COLS / BUF_COLS;
+    static constexpr int TEAMS = MAXT == 1 ? 2 : 1;
+    static constexpr int CWW = MAXT == 1 ? 32 : 16;               // columns per tile per warp
+    static constexpr int TEAM_THREADS = kEpiThreads / TEAMS;
 };
-constexpr int kEpiWarps = 8;         // two per TMEM lane quadrant
-constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int CW = 16;               // columns of each token tile per epilogue warp
-constexpr int TBL_KB = 8;            // K blocks per chunk of the epilogue's scale table
-constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 template <int MAXT>
@@ -81,13 +92,14 @@ struct Ctl {
     uint64_t tempty[NBUF];
     uint64_t ufull[RING];
     uint64_t uempty[RING];
-    uint64_t pub;        // every epilogue thread's act rows of an item are stored
-    uint64_t red_bar[2]; // the four epilogue warps' column maxima are in red[b]
+    static constexpr int TEAMS = Shape<MAXT>::TEAMS, CWW = Shape<MAXT>::CWW;
+    uint64_t pub[TEAMS];        // every thread of a team has stored an item's act rows
+    uint64_t red_bar[TEAMS][2]; // a team's column maxima are in red[team][b]
     uint64_t drain;
-    float red[2][4][NP]; // per lane quadrant, per token column: max |a| over its 32 rows
+    float red[TEAMS][2][4][NP]; // per lane quadrant, per token column: max |a| over its 32 rows
     // per epilogue warp, per K block of the current chunk: sa[col] * sw of
-    // each of the warp's MAXT * CW columns, for gate (0) and up (1)
-    float4 tbl[kEpiWarps][2][TBL_KB][MAXT * CW / 4];
+    // each of the warp's MAXT * CWW columns, for gate (0) and up (1)
+    float4 tbl[kEpiWarps][2][TBL_KB][MAXT * CWW / 4];
     int ring_item[RING];
     int ring_pass[RING];
     uint32_t tmem_base;
@@ -154,47 +166,52 @@ __device__ __forceinline__ Unit decode(int item, int pass, int n_gu_tiles, int n
 // One epilogue step: NKB consecutive K blocks (TMEM buffers buf, buf+1, ...)
 // of NT token tiles, gate and up (GU) or down only: every partial times its
 // column's scale product from the table row of that K block, added into the
-// fp32 accumulators. Per token tile, the loads of all NKB blocks are issued
+// fp32 accumulators. Per 16 columns, the loads of all NKB blocks are issued
 // before one wait.
 template <int MAXT, bool GU, int NT, int NKB>
-__device__ __forceinline__ void promote(uint32_t t0, int buf, const float4 (*tg)[MAXT * CW / 4],
-                                        const float4 (*tu)[MAXT * CW / 4], float (&accg)[NT * CW],
-                                        float (&accu)[NT * CW]) {
+__device__ __forceinline__ void promote(
+    uint32_t t0, int buf, const float4 (*tg)[MAXT * Shape<MAXT>::CWW / 4],
+    const float4 (*tu)[MAXT * Shape<MAXT>::CWW / 4], float (&accg)[NT * Shape<MAXT>::CWW],
+    float (&accu)[NT * Shape<MAXT>::CWW]) {
     constexpr int NP = Shape<MAXT>::NP, NBUF = Shape<MAXT>::NBUF, BUF_COLS = Shape<MAXT>::BUF_COLS;
+    constexpr int CWW = Shape<MAXT>::CWW, NH = CWW / 16;
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        uint32_t g[NKB][16], v[NKB][16];
+    for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int k = 0; k < NKB; ++k) {
-            const uint32_t tb = t0 + static_cast<uint32_t>(((buf + k) % NBUF) * BUF_COLS);
-            tmem_ld_32x32b_x16(tb + t * TT, g[k]);
-            if (GU) tmem_ld_32x32b_x16(tb + NP + t * TT, v[k]);
-        }
-        tmem_ld_wait();
+        for (int h = 0; h < NH; ++h) {  // 16 columns at a time
+            uint32_t g[NKB][16], v[NKB][16];
 #pragma unroll
-        for (int k = 0; k < NKB; ++k)
-#pragma unroll
-            for (int c4 = 0; c4 < CW / 4; ++c4) {
-                const float4 sg = tg[k][t * (CW / 4) + c4];
-                const int c = t * CW + 4 * c4;
-                accg[c + 0] = fmaf(__uint_as_float(g[k][4 * c4 + 0]), sg.x, accg[c + 0]);
-                accg[c + 1] = fmaf(__uint_as_float(g[k][4 * c4 + 1]), sg.y, accg[c + 1]);
-                accg[c + 2] = fmaf(__uint_as_float(g[k][4 * c4 + 2]), sg.z, accg[c + 2]);
-                accg[c + 3] = fmaf(__uint_as_float(g[k][4 * c4 + 3]), sg.w, accg[c + 3]);
-                if (GU) {
-                    const float4 su = tu[k][t * (CW / 4) + c4];
-                    accu[c + 0] = fmaf(__uint_as_float(v[k][4 * c4 + 0]), su.x, accu[c + 0]);
-                    accu[c + 1] = fmaf(__uint_as_float(v[k][4 * c4 + 1]), su.y, accu[c + 1]);
-                    accu[c + 2] = fmaf(__uint_as_float(v[k][4 * c4 + 2]), su.z, accu[c + 2]);
-                    accu[c + 3] = fmaf(__uint_as_float(v[k][4 * c4 + 3]), su.w, accu[c + 3]);
-                }
+            for (int k = 0; k < NKB; ++k) {
+                const uint32_t tb = t0 + static_cast<uint32_t>(((buf + k) % NBUF) * BUF_COLS);
+                tmem_ld_32x32b_x16(tb + t * TT + h * 16, g[k]);
+                if (GU) tmem_ld_32x32b_x16(tb + NP + t * TT + h * 16, v[k]);
             }
-    }
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < NKB; ++k)
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int cc = t * CWW + h * 16 + 4 * c4;  // accumulator / table column
+                    const float4 sg = tg[k][cc / 4];
+                    accg[cc + 0] = fmaf(__uint_as_float(g[k][4 * c4 + 0]), sg.x, accg[cc + 0]);
+                    accg[cc + 1] = fmaf(__uint_as_float(g[k][4 * c4 + 1]), sg.y, accg[cc + 1]);
+                    accg[cc + 2] = fmaf(__uint_as_float(g[k][4 * c4 + 2]), sg.z, accg[cc + 2]);
+                    accg[cc + 3] = fmaf(__uint_as_float(g[k][4 * c4 + 3]), sg.w, accg[cc + 3]);
+                    if (GU) {
+                        const float4 su = tu[k][cc / 4];
+                        accu[cc + 0] = fmaf(__uint_as_float(v[k][4 * c4 + 0]), su.x, accu[cc + 0]);
+                        accu[cc + 1] = fmaf(__uint_as_float(v[k][4 * c4 + 1]), su.y, accu[cc + 1]);
+                        accu[cc + 2] = fmaf(__uint_as_float(v[k][4 * c4 + 2]), su.z, accu[cc + 2]);
+                        accu[cc + 3] = fmaf(__uint_as_float(v[k][4 * c4 + 3]), su.w, accu[cc + 3]);
+                    }
+                }
+        }
 }
 
 // Per-thread state of an epilogue warp across units.
 struct EpiState {
     int ew, q, h2, r, lt, lcol;  // warp index, TMEM lane quadrant, column half, row, lane column
+    int team;
     uint32_t tmem_base;
     uint32_t nblk, npub, nred;   // K blocks consumed; phases of ctl->pub and ctl->red_bar
 };
@@ -216,7 +233,7 @@ template <int MAXT, int NT>
 __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp8ExpertParams &p,
                                          EpiState &st, int n_gu_tiles, int n_dn_tiles,
                                          int *done) {
-    constexpr int NBUF = Shape<MAXT>::NBUF;
+    constexpr int NBUF = Shape<MAXT>::NBUF, CWW = Shape<MAXT>::CWW;
     const int lane = threadIdx.x & 31;
     const int ngd = p.d / kFp8Block, ngi = p.I / kFp8Block;
     const int nk = (u.gate_up ? p.d : p.I) / BK;
@@ -229,18 +246,18 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
         ? p.sgu + (static_cast<size_t>(u.e) * (2 * n_gu_tiles) + n_gu_tiles + u.tile) * ngd
         : swg;
     const int ng = u.gate_up ? ngd : ngi;
-    // this lane's column: lanes 16..31 serve the second token tile, which
-    // exists in the two-tile shape only; its group scales (row of xs or as)
+    // this lane's column (lane / CWW is its token tile, which must exist in
+    // this shape); its group scales (row of xs or as)
     const bool lserve = st.lt < MAXT;
     const bool lvalid = st.lt < NT && st.lcol < u.rows;
     const float *sa_row = (u.gate_up ? p.xs : p.as) +
                           static_cast<size_t>(u.row0 + (lvalid ? st.lcol : 0)) * ng;
-    float accg[NT * CW], accu[NT * CW];
+    float accg[NT * CWW], accu[NT * CWW];
 #pragma unroll
-    for (int c = 0; c < NT * CW; ++c) { accg[c] = 0.f; accu[c] = 0.f; }
-    const float4 (*tg)[MAXT * CW / 4] = ctl->tbl[st.ew][0];
-    const float4 (*tu)[MAXT * CW / 4] = ctl->tbl[st.ew][1];
-    const uint32_t tq = st.tmem_base + (static_cast<uint32_t>(st.q * 32) << 16) + st.h2 * CW;
+    for (int c = 0; c < NT * CWW; ++c) { accg[c] = 0.f; accu[c] = 0.f; }
+    const float4 (*tg)[MAXT * CWW / 4] = ctl->tbl[st.ew][0];
+    const float4 (*tu)[MAXT * CWW / 4] = ctl->tbl[st.ew][1];
+    const uint32_t tq = st.tmem_base + (static_cast<uint32_t>(st.q * 32) << 16) + st.h2 * CWW;
     for (int kb = 0; kb < nk;) {
         if (kb % TBL_KB == 0) {
             // the next chunk of the scale table: lane l writes column l's
@@ -263,8 +280,8 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
             }
             __syncwarp();
         }
-        // two K blocks per step for one token tile while both lie in this chunk
-        const int nkb = (NT == 1 && kb + 1 < nk && (kb + 1) % TBL_KB != 0) ? 2 : 1;
+        // two K blocks per step for one 16-column tile while both lie in this chunk
+        const int nkb = (NT == 1 && CWW == 16 && kb + 1 < nk && (kb + 1) % TBL_KB != 0) ? 2 : 1;
         const int buf = static_cast<int>(st.nblk % NBUF);
         for (int k = 0; k < nkb; ++k)
             if (!wait_bar(&ctl->tfull[(buf + k) % NBUF], ((st.nblk + k) / NBUF) & 1u, &ctl->abort, p.status))
@@ -272,10 +289,10 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
         tc_fence_after();
         const int row = kb % TBL_KB;
         if (u.gate_up) {
-            if (nkb == 2) promote<MAXT, true, NT, 2>(tq, buf, tg + row, tu + row, accg, accu);
+            if (CWW == 16 && nkb == 2) promote<MAXT, true, NT, (CWW == 16 ? 2 : 1)>(tq, buf, tg + row, tu + row, accg, accu);
             else promote<MAXT, true, NT, 1>(tq, buf, tg + row, tu + row, accg, accu);
         } else {
-            if (nkb == 2) promote<MAXT, false, NT, 2>(tq, buf, tg + row, tu + row, accg, accu);
+            if (CWW == 16 && nkb == 2) promote<MAXT, false, NT, (CWW == 16 ? 2 : 1)>(tq, buf, tg + row, tu + row, accg, accu);
             else promote<MAXT, false, NT, 1>(tq, buf, tg + row, tu + row, accg, accu);
         }
         tc_fence_before();
@@ -290,10 +307,10 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
 #pragma unroll
         for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int c = 0; c < CW; ++c) {
-                const int col = t * TT + st.h2 * CW + c;
+            for (int c = 0; c < CWW; ++c) {
+                const int col = t * TT + st.h2 * CWW + c;
                 if (col < u.rows)
-                    y[static_cast<size_t>(u.row0 + col) * p.d + f] = __float2bfloat16_rn(accg[t * CW + c]);
+                    y[static_cast<size_t>(u.row0 + col) * p.d + f] = __float2bfloat16_rn(accg[t * CWW + c]);
             }
         return true;
     }
@@ -302,7 +319,7 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
     // a warp maximum over the bits of |a| (non-negative floats order like
     // their bit patterns), then the four lane quadrants
 #pragma unroll
-    for (int c = 0; c < NT * CW; ++c) {
+    for (int c = 0; c < NT * CWW; ++c) {
         const float gv = accg[c];
         accg[c] = __fdividef(gv, 1.0f + __expf(-gv)) * accu[c];
     }
@@ -310,19 +327,21 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int c = 0; c < CW; ++c) {
-            const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(accg[t * CW + c])));
-            if (lane == t * 16 + c) mine = __uint_as_float(m);
+        for (int c = 0; c < CWW; ++c) {
+            const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(accg[t * CWW + c])));
+            if (lane == t * CWW + c) mine = __uint_as_float(m);
         }
     const int rb = static_cast<int>(st.nred & 1u);
-    if (lserve) ctl->red[rb][st.q][st.lcol] = mine;
-    mbar_arrive(&ctl->red_bar[rb]);
-    if (!wait_bar(&ctl->red_bar[rb], (st.nred >> 1) & 1u, &ctl->abort, p.status)) return false;
+    float (*red)[Shape<MAXT>::NP] = ctl->red[st.team][rb];
+    if (lserve) red[st.q][st.lcol] = mine;
+    mbar_arrive(&ctl->red_bar[st.team][rb]);
+    if (!wait_bar(&ctl->red_bar[st.team][rb], (st.nred >> 1) & 1u, &ctl->abort, p.status))
+        return false;
     ++st.nred;
     float sl = 0.f;  // the scale of column lcol
     if (lserve) {
-        const float amax = fmaxf(fmaxf(ctl->red[rb][0][st.lcol], ctl->red[rb][1][st.lcol]),
-                                 fmaxf(ctl->red[rb][2][st.lcol], ctl->red[rb][3][st.lcol]));
+        const float amax = fmaxf(fmaxf(red[0][st.lcol], red[1][st.lcol]),
+                                 fmaxf(red[2][st.lcol], red[3][st.lcol]));
         sl = __fdiv_rn(amax, 448.f);
     }
     if (st.q == 0 && lvalid) p.as[static_cast<size_t>(u.row0 + st.lcol) * ngi + u.tile] = sl;
@@ -330,12 +349,12 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int c = 0; c < CW; ++c) {
-            const float sc = __shfl_sync(0xffffffffu, sl, t * 16 + c);
-            const int col = t * TT + st.h2 * CW + c;
+        for (int c = 0; c < CWW; ++c) {
+            const float sc = __shfl_sync(0xffffffffu, sl, t * CWW + c);
+            const int col = t * TT + st.h2 * CWW + c;
             if (col < u.rows) {
                 const uint8_t code = sc > 0.f
-                    ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(accg[t * CW + c], sc),
+                    ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(accg[t * CWW + c], sc),
                                                                  __NV_SATFINITE, __NV_E4M3))
                     : static_cast<uint8_t>(0);
                 p.aq[static_cast<size_t>(u.row0 + col) * p.I + f] = code;
@@ -348,9 +367,10 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
         // and releases the per-expert counter
         fence_proxy_async_global();
         __threadfence();
-        mbar_arrive(&ctl->pub);
-        if (st.ew == 0 && lane == 0) {
-            if (wait_bar(&ctl->pub, st.npub & 1u, &ctl->abort, p.status)) {
+        mbar_arrive(&ctl->pub[st.team]);
+        const bool lead = Shape<MAXT>::TEAMS == 2 ? (st.ew & 3) == 0 : st.ew == 0;
+        if (lead && lane == 0) {  // the team's first warp
+            if (wait_bar(&ctl->pub[st.team], st.npub & 1u, &ctl->abort, p.status)) {
                 __threadfence();
                 atomicAdd(done + u.e, 1);
             }
@@ -386,15 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], kEpiThreads);
+            mbar_init(&ctl->tempty[b], Shape<MAXT>::TEAM_THREADS);  // the consuming team
         }
         for (int r = 0; r < RING; ++r) {
             mbar_init(&ctl->ufull[r], 1);
             mbar_init(&ctl->uempty[r], 1 + kEpiThreads);  // the MMA thread, every epilogue thread
         }
-        mbar_init(&ctl->pub, kEpiThreads);
-        mbar_init(&ctl->red_bar[0], kEpiThreads);
-        mbar_init(&ctl->red_bar[1], kEpiThreads);
+        for (int t = 0; t < Shape<MAXT>::TEAMS; ++t) {
+            mbar_init(&ctl->pub[t], Shape<MAXT>::TEAM_THREADS);
+            mbar_init(&ctl->red_bar[t][0], Shape<MAXT>::TEAM_THREADS);
+            mbar_init(&ctl->red_bar[t][1], Shape<MAXT>::TEAM_THREADS);
+        }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_mbar_init();
@@ -557,20 +579,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------- epilogue -------------------------
-        // thread <-> TMEM lane = weight row: warp w reads lanes 32*(w%4)..+31;
-        // the two warps of a quadrant split every token tile's 32 columns into
-        // halves of CW. Lane l also serves one column for the lane-parallel
-        // work: lcol = tile (l / 16), column h2 * CW + l % 16 of that tile.
+        // thread <-> TMEM lane = weight row: warp w reads lanes 32*(w%4)..+31
+        // and CWW columns of each token tile (from column h2 * CWW). Lane l
+        // also serves one column for the lane-parallel work: lcol = tile
+        // l / CWW, column h2 * CWW + l % CWW of that tile.
+        constexpr int TEAMS = Shape<MAXT>::TEAMS, CWW = Shape<MAXT>::CWW;
         EpiState st;
         st.ew = warp - 2;
         st.q = warp & 3;
-        st.h2 = st.ew >> 2;
+        st.team = TEAMS == 2 ? st.ew >> 2 : 0;
+        st.h2 = TEAMS == 2 ? 0 : st.ew >> 2;
         st.r = st.q * 32 + lane;
-        st.lt = lane >> 4;
-        st.lcol = st.lt * TT + st.h2 * CW + (lane & 15);
+        st.lt = lane / CWW;
+        st.lcol = st.lt * TT + st.h2 * CWW + lane % CWW;
         st.tmem_base = tmem_base;
         st.nblk = st.npub = st.nred = 0;
-        int useq = 0;
+        int useq = 0, nunit = 0;
         bool ok = true;
         while (ok && !aborted(&ctl->abort)) {
             const int slot = useq % RING;
@@ -580,6 +604,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++useq;
             if (item < 0) break;
             const Unit u = decode<MAXT>(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
+            if (nunit++ % TEAMS != st.team) {  // the other team's unit: skip its K blocks
+                st.nblk += (u.gate_up ? p.d : p.I) / BK;
+                continue;
+            }
             if (MAXT == 2 && u.ntt == 2)
                 ok = epi_unit<MAXT, MAXT>(u, ctl, p, st, n_gu_tiles, n_dn_tiles, done);
             else
