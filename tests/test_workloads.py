@@ -73,3 +73,21 @@ def test_verify_widens_the_expert_union():
     wd = W.DECODE
     rd = _route(wd, W.make_layer(wd, with_experts=False), W.make_x(wd))
     assert active >= 62 and active > np.unique(rd["idx"]).size, active
+
+
+def test_fp8_layer_draw():
+    """FP8_BLOCK layers: e4m3 expert matrices, one fp32 scale per 128x128
+    block, the dequantised weights at the bf16 workloads' standard deviation,
+    the same router tensors as a draw without experts."""
+    w = W.DECODE_FP8.scaled(n_experts=4, d=256, d_ff=384)
+    layer = W.make_layer(w, 0)
+    assert layer["w_gate_up"].dtype == torch.float8_e4m3fn
+    assert layer["w_down"].dtype == torch.float8_e4m3fn
+    assert tuple(layer["w_gate_up_scale"].shape) == (4, 6, 2)
+    assert tuple(layer["w_down_scale"].shape) == (4, 2, 3)
+    sc = layer["w_gate_up_scale"].repeat_interleave(128, 1).repeat_interleave(128, 2)
+    deq = layer["w_gate_up"].float() * sc
+    assert abs(deq.std().item() - w.gate_up_std) < 0.05 * w.gate_up_std
+    assert not torch.isnan(layer["w_down"].float()).any()
+    r = W.make_layer(w, 0, with_experts=False)
+    assert torch.equal(r["router_w"], layer["router_w"]) and torch.equal(r["bias"], layer["bias"])
