@@ -12,30 +12,31 @@
 // matching up rows of expert e, K = d; down item (e, nt): rows nt*128.. of
 // Wd_e, K = I), claimed from one atomic counter, gate/up items first; a down
 // item of expert e waits until its I/128 gate/up items have published their
-// act rows. Each item runs in passes of up to 64 tokens.
+// act rows. Each item runs in passes of 32 tokens (small batches) or 64.
 //
 // What FP8_BLOCK changes: a stage is one K block of 128 (128 e4m3 = one
 // 128-byte swizzle row), and every block has its own scale on both operands
 // (weight block scale sw, token group scale sa), so the tensor cores cannot
 // accumulate across blocks. Each K block's MMAs (kind::f8f6f4, M128, N32/64,
-// K32) start a fresh accumulator in one of four rotating TMEM buffers; the
-// epilogue warps load it (tcgen05.ld) and add partial * sw * sa[token] into
-// fp32 registers, while the tensor cores already fill the next buffer. At
-// the end of a pass:
+// K32) start a fresh accumulator in one of 8 (32-token passes) or 4 rotating
+// TMEM buffers; the epilogue warps load it (tcgen05.ld) and add
+// partial * sw * sa[token] into fp32 registers, while the tensor cores
+// already fill the next buffers. At the end of a pass:
 //   gate/up: a = SiLU(gate) * up per (token, row); the item's 128 rows are
-//     exactly one activation group of 128, so the group maximum is a max over
-//     the 128 TMEM lanes (a warp redux per column, then the four lane
-//     quadrants through shared memory, met at an mbarrier), s = amax / 448 and the codes
-//     e4m3(a / s) (nearest-even, saturating) go to aq with s in as;
+//     exactly one activation group of 128, so the group maximum is a max
+//     over the 128 TMEM lanes (a warp redux per column, then the four lane
+//     quadrants through shared memory, met at an mbarrier), s = amax / 448
+//     and the codes e4m3(a / s) (nearest-even, saturating) go to aq, s to as;
 //   down: y = the fp32 sum, rounded once to bf16.
-// Roles per CTA (320 threads): warp 0 lane 0 claims items and issues TMA;
-// warp 1 owns TMEM (512 columns) and one thread issues the MMAs; warps 2..9
-// are the epilogue, two per TMEM lane quadrant (two teams taking alternate
-// units, or both warps of a quadrant sharing each unit's columns: see Shape);
-// the per-column scale products sa * sw of up to eight K blocks are formed
-// once per lane into a shared-memory table and read back as float4s. All waits are bounded (1 s) and report
-// MOE_ERR_DEVICE_TIMEOUT; on time-out the kernel drains its own copies and
-// MMAs, frees TMEM and returns.
+// Roles per CTA (320 threads): warp 0 lane 0 claims items and issues TMA
+// (and prefetches the item's block scales into L2); warp 1 owns TMEM (512
+// columns) and one thread issues the MMAs; warps 2..9 are the epilogue, two
+// per TMEM lane quadrant (two teams taking alternate units, or both warps of
+// a quadrant sharing each unit's columns: see Shape); the per-column scale
+// products sa * sw of up to eight K blocks are formed once per lane into a
+// shared-memory table and read back as float4s. All waits are bounded (1 s)
+// and report MOE_ERR_DEVICE_TIMEOUT; on time-out the kernel drains its own
+// copies and MMAs, frees TMEM and returns.
 #include <cuda_fp8.h>
 
 #include <new>
