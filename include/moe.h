@@ -163,7 +163,9 @@ int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream);
  * they may synchronise the device, or under a memory planner that owns all
  * device memory). The page describes no such entry point; it is an interface
  * of this library only. Computes, for x[n_tokens][d] (dtype MOE_F32 or
- * MOE_BF16) and the fp32 norm_gain[d], router_w[E][d], expert_bias[E], the
+ * MOE_BF16: the storage type of x, so MOE_BF16 for the bf16 x of an
+ * MOE_FP8_BLOCK layer, whose router is unquantised; any other dtype gives
+ * MOE_ERR_INVALID_ARG) and the fp32 norm_gain[d], router_w[E][d], expert_bias[E], the
  * same idx[n_tokens][top_k] (int32, slot order) and w[n_tokens][top_k] (fp32)
  * as moe_forward's routing (see moe_debug_routing). All pointers are device
  * pointers owned by the caller; x, norm_gain and router_w 16-byte aligned.

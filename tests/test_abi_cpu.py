@@ -79,6 +79,15 @@ def test_create_without_gpu_reports_no_device():
     assert rc == -9 and not h.value
 
 
+def test_route_noalloc_takes_the_storage_type_of_x():
+    """The no-allocation router takes x's own dtype (f32 or bf16); the
+    FP8_BLOCK layer dtype, which describes expert weights, is refused before
+    any device work."""
+    L = sb.lib()
+    args = (256, 1, 256, 256, 256, 8, 256, 16, 4, 1e-6, 1.0, 256, 256, None)
+    assert L.moe_route_noalloc(args[0], sb.MOE_FP8_BLOCK, *args[2:]) == -1
+
+
 def test_calls_on_null_handle_are_rejected():
     L = sb.lib()
     assert L.moe_forward(None, None, None, 1, None) == -1
