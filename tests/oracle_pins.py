@@ -386,8 +386,44 @@ def pin_fp8_scale_code_trade(mut):
     np.testing.assert_array_equal(o0, o1)
 
 
+def pin_fp8_sign_symmetry(mut):
+    """Quantisation is odd: negating a row flips every code's sign bit (zero
+    codes excepted) and keeps the scales; the dequantised row is negated."""
+    g = torch.Generator().manual_seed(9)
+    v = (torch.randn(4, 256, generator=g) * 2).double().numpy()
+    a, b = oracle.quant(v, mutation=mut), oracle.quant(-v, mutation=mut)
+    np.testing.assert_array_equal(a["scales"], b["scales"])
+    nz = (a["codes"] & 0x7F) != 0
+    np.testing.assert_array_equal(a["codes"][nz] ^ 0x80, b["codes"][nz])
+    np.testing.assert_array_equal(a["deq"], -b["deq"])
+
+
+def pin_fp8_zero_block_scale(mut):
+    """A block scale of zero removes exactly that block: the output equals the
+    one with the block's codes set to zero (both leave the other 127 x 128
+    blocks' products untouched, and a scale read from the wrong block would
+    change a different block)."""
+    E, d, I, k = 2, 256, 128, 2
+    layer = fp8_layer(E, d, I, seed=71)
+    x = rand_x(5, d, 71)
+    a = dict(layer)
+    sc = layer["w_gate_up_scale"].clone()
+    sc[1, 0, 1] = 0.0
+    a["w_gate_up_scale"] = sc
+    b = dict(layer)
+    wgu = layer["w_gate_up"].float().clone()
+    wgu[1, 0:128, 128:256] = 0.0
+    b["w_gate_up"] = wgu.to(E4M3)
+    oa = oracle.forward(x, a, k=k, eps=EPS, mutation=mut)["out"]
+    ob = oracle.forward(x, b, k=k, eps=EPS, mutation=mut)["out"]
+    np.testing.assert_array_equal(oa, ob)
+    o0 = oracle.forward(x, layer, k=k, eps=EPS, mutation=mut)["out"]
+    assert np.abs(oa - o0).max() > 0
+
+
 PINS = [pin_five_candidate, pin_rmsnorm, pin_router_sigmoid, pin_weights_sum_below_one,
         pin_k1, pin_tie_break, pin_brute_force_subsets, pin_zero_bias_is_logit_topk,
         pin_bias_shift_invariance, pin_all_selected_bias_invariance,
         pin_zero_down_is_identity, pin_identical_experts, pin_e4m3_codec, pin_fp8_quant,
-        pin_fp8_expert_blocks, pin_fp8_forward_error_bound, pin_fp8_scale_code_trade]
+        pin_fp8_expert_blocks, pin_fp8_forward_error_bound, pin_fp8_scale_code_trade,
+        pin_fp8_sign_symmetry, pin_fp8_zero_block_scale]
