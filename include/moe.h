@@ -37,9 +37,10 @@ extern "C" {
 
 /* Storage type of x, out and the expert matrices. The RMSNorm gain, router
  * matrix and expert bias are always fp32 (the router stays unquantised).
- * MOE_FP8_BLOCK is the FP8 checkpoint's scheme ("LFM2.5-24B-A2B", flozi.net,
- * German page, section "Quantisierung": weights FP8 static in 128x128
- * blocks, activations FP8 dynamic per group of 128): x and out are bf16, the
+ * MOE_FP8_BLOCK is the FP8 checkpoint's scheme ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
+ * inferencekey.com, section "Für Engineers", paragraph "Quantisierung":
+ * weights FP8 static in 128x128 blocks, activations FP8 dynamic per group of
+ * 128): x and out are bf16, the
  * expert matrices are e4m3 codes (1 sign, 4 exponent bits with bias 7, 3
  * mantissa bits, no infinities, largest finite 448) with one fp32 scale per
  * 128x128 block, weight = code value * block scale. Inside the forward each

@@ -31,8 +31,9 @@
  * the gated MLP is down( silu(gate x) * (up x) ) with gate rows first in the
  * packed matrix; the combine sums slots in slot order and adds the residual.
  *
- * FP8_BLOCK experts, from "LFM2.5-24B-A2B" (same site, German page, section
- * "Quantisierung"): expert weights are stored as FP8 statically in 128x128
+ * FP8_BLOCK experts, from "LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell"
+ * (inferencekey.com, section "Für Engineers", paragraph "Quantisierung"):
+ * expert weights are stored as FP8 statically in 128x128
  * blocks, activations are quantised to FP8 dynamically per group of 128; the
  * router stays unquantised. Readings taken: the FP8 format is e4m3 with no
  * infinities (largest finite 448), decoded from its definition; a weight is

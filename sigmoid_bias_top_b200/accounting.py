@@ -53,7 +53,8 @@ def down_flops(n_assign: int, d: int, d_ff: int) -> int:
     return 2 * n_assign * d * d_ff
 
 
-# FP8_BLOCK experts ("LFM2.5-24B-A2B", German page, section "Quantisierung":
+# FP8_BLOCK experts ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
+# inferencekey.com, section "Für Engineers", paragraph "Quantisierung":
 # weights FP8 in static 128x128 blocks, activations FP8 per group of 128).
 
 def fp8_scale_bytes(active_experts: int, d: int, d_ff: int) -> int:

@@ -25,8 +25,9 @@
 //      assignment, one warp per row: xp[row] = x[t] * rinv[t] * gain, the same
 //      fp32 products as the router's input, rounded once to the storage type.
 // The grouped rows let the gate/up GEMM load contiguous 128-row TMA boxes.
-// For FP8_BLOCK layers ("LFM2.5-24B-A2B", German page, section
-// "Quantisierung": activations FP8, dynamic per group of 128) step 3 writes
+// For FP8_BLOCK layers ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
+// inferencekey.com, section "Für Engineers", paragraph "Quantisierung":
+// activations FP8, dynamic per group of 128) step 3 writes
 // e4m3 codes instead: each group of 128 normalised values (16 lanes) takes
 // s = amax / 448 and codes e4m3(v / s), nearest-even and saturating, with the
 // scale stored beside the codes.

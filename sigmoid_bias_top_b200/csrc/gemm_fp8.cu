@@ -4,8 +4,10 @@
 // The gated SiLU expert of "LFM2.5-24B-A2B: Biased Routing, Short Convolutions
 // and Ten KV Caches" (flozi.net, English page, section "The router has two
 // different scores") with the FP8_BLOCK storage of the FP8 checkpoint
-// ("LFM2.5-24B-A2B", German page, section "Quantisierung": weights FP8 in
-// static 128x128 blocks, activations FP8 dynamic per group of 128).
+// ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
+// inferencekey.com, section "Für Engineers", paragraph "Quantisierung":
+// weights FP8 in static 128x128 blocks, activations FP8 dynamic per group
+// of 128).
 //
 // Work decomposition as in the bf16 small-batch kernel: an item is one
 // 128-row weight tile (gate/up item (e, ft): gate rows ft*128.. and the

@@ -1,7 +1,8 @@
 // moe_fp8.cuh -- the FP8_BLOCK expert path: parameter blocks, launchers and
 // the kind::f8f6f4 tensor-core wrappers.
 //
-// Scheme ("LFM2.5-24B-A2B", flozi.net, German page, section "Quantisierung"):
+// Scheme ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
+// inferencekey.com, section "Für Engineers", paragraph "Quantisierung"):
 // expert weights are stored as FP8 with one scale per 128 x 128 block, and the
 // activations entering each expert matrix are quantised to FP8 per token in
 // groups of 128. Here the FP8 format is e4m3 (largest finite 448); a weight

@@ -17,8 +17,9 @@ Tensor layout (what the C ABI consumes):
   bias       [E]           f32           expert bias (selection only)
   w_gate_up  [E, 2I, d]    f32 or bf16   rows 0..I-1 = gate, rows I..2I-1 = up
   w_down     [E, d, I]     f32 or bf16   down projection
-FP8_BLOCK workloads (dtype "fp8"; the FP8 checkpoint of "LFM2.5-24B-A2B",
-German page, section "Quantisierung") keep x bf16 and store the expert
+FP8_BLOCK workloads (dtype "fp8"; the FP8 checkpoint of "LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
+inferencekey.com, section "Für Engineers", paragraphs "Checkpoint" and
+"Quantisierung") keep x bf16 and store the expert
 matrices as e4m3 codes (torch.float8_e4m3fn) with fp32 block scales:
   w_gate_up_scale [E, 2I/128, d/128]   w_down_scale [E, d/128, I/128]
 The codes are normal draws of standard deviation fp8_code_std cast to e4m3

@@ -220,8 +220,9 @@ def pin_identical_experts(mut):
 
 
 # ---------------------------------------------------------------- FP8_BLOCK
-# "LFM2.5-24B-A2B" (flozi.net, German page, section "Quantisierung"): weights
-# FP8 static in 128x128 blocks, activations FP8 dynamic per group of 128.
+# "LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell" (inferencekey.com,
+# section "Für Engineers", paragraph "Quantisierung"): weights FP8 static in
+# 128x128 blocks, activations FP8 dynamic per group of 128.
 
 E4M3 = torch.float8_e4m3fn
 

@@ -369,8 +369,9 @@ def test_fp32_widest_rows():
 
 
 # ---------------------------------------------------------------- FP8_BLOCK
-# The FP8 checkpoint's experts ("LFM2.5-24B-A2B", flozi.net, German page,
-# section "Quantisierung"): e4m3 weights in 128x128 blocks, activations
+# The FP8 checkpoint's experts ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
+# inferencekey.com, section "Für Engineers", paragraph "Quantisierung"):
+# e4m3 weights in 128x128 blocks, activations
 # quantised per group of 128 inside the forward.
 
 def fp8_small(**kw):
