@@ -33,7 +33,7 @@
 // Roles per CTA (320 threads): warp 0 lane 0 claims items and issues TMA
 // (and prefetches the item's block scales into L2); warp 1 owns TMEM (512
 // columns) and one thread issues the MMAs; warps 2..9 are the epilogue, two
-// per TMEM lane quadrant (two teams taking alternate units, or both warps of
+// per TMEM lane quadrant (two teams taking alternate items, or both warps of
 // a quadrant sharing each unit's columns: see Shape); the per-column scale
 // products sa * sw of up to eight K blocks are formed once per lane into a
 // shared-memory table and read back as float4s. All waits are bounded (1 s)
@@ -68,7 +68,9 @@ constexpr int kThreads = 64 + kEpiThreads;
 // run ahead of the epilogue (8 instead of 4).
 //
 // The epilogue warps: with one token tile per pass they form two teams of
-// four (one warp per TMEM lane quadrant) that take alternate units, each warp
+// four (one warp per TMEM lane quadrant) that take alternate items (all the
+// passes of an item go to the same team, so that the team's fence before
+// publishing the item covers every row it wrote), each warp
 // covering all 32 columns, so that one team's end-of-pass work (SiLU,
 // quantisation, publication) and scale loads overlap the other team's K loop;
 // with two tiles the eight warps share every unit, the two warps of a
@@ -105,6 +107,7 @@ struct Ctl {
     float4 tbl[kEpiWarps][2][TBL_KB][MAXT * CWW / 4];
     int ring_item[RING];
     int ring_pass[RING];
+    int ring_team[RING];  // the epilogue team of the unit's item (all its passes)
     uint32_t tmem_base;
     int abort;
 };
@@ -452,16 +455,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t issued_parity[STAGES];
             for (int i = 0; i < STAGES; ++i) issued[i] = false;
             bool ok = true;
+            int nitem = 0;  // items with tokens claimed by this CTA
             while (ok && !aborted(&ctl->abort)) {
                 const int item = atomicAdd(next_item, 1);
                 const bool stop = item >= total;
-                int npass = 0;
+                int npass = 0, team = 0;
                 Unit u0;
                 if (!stop) {
                     u0 = decode<MAXT>(item, 0, n_gu_tiles, n_dn_tiles, E, offs);
                     const int cnt = offs[u0.e + 1] - offs[u0.e];
                     if (cnt <= 0) continue;  // expert without tokens: nothing to do
                     npass = (cnt + NP - 1) / NP;
+                    // every pass of an item goes to one epilogue team, whose
+                    // fence at the last pass then covers all the item's rows
+                    team = nitem++ % Shape<MAXT>::TEAMS;
                     // the item's weight block scales, for the epilogue units to come
                     const int ngd = p.d / kFp8Block, ngi = p.I / kFp8Block;
                     if (u0.gate_up) {
@@ -495,6 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ctl->ring_item[slot] = stop ? -1 : item;
                     ctl->ring_pass[slot] = pass;
+                    ctl->ring_team[slot] = team;
                     mbar_arrive(&ctl->ufull[slot]);
                     ++useq;
                     if (stop) break;
@@ -597,17 +605,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         st.lcol = st.lt * TT + st.h2 * CWW + lane % CWW;
         st.tmem_base = tmem_base;
         st.nblk = st.npub = st.nred = 0;
-        int useq = 0, nunit = 0;
+        int useq = 0;
         bool ok = true;
         while (ok && !aborted(&ctl->abort)) {
             const int slot = useq % RING;
             if (!wait_bar(&ctl->ufull[slot], (useq / RING) & 1u, &ctl->abort, p.status)) break;
             const int item = ctl->ring_item[slot], pass = ctl->ring_pass[slot];
+            const int team = ctl->ring_team[slot];
             mbar_arrive(&ctl->uempty[slot]);
             ++useq;
             if (item < 0) break;
             const Unit u = decode<MAXT>(item, pass, n_gu_tiles, n_dn_tiles, E, offs);
-            if (nunit++ % TEAMS != st.team) {  // the other team's unit: skip its K blocks
+            if (team != st.team) {  // the other team's unit: skip its K blocks
                 st.nblk += (u.gate_up ? p.d : p.I) / BK;
                 continue;
             }

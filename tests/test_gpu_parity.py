@@ -412,6 +412,19 @@ def test_fp8_one_expert_takes_all():
     assert res["counts"][5] == 700
 
 
+def test_fp8_many_passes_in_the_small_batch_shape():
+    """200 tokens, k = 1, all on one of 8 experts: still the 32-token shape
+    (N*k <= 32*E), so that expert's items run in 7 passes, which must all be
+    published before its down items read the act rows."""
+    w = fp8_small(n_experts=8, top_k=1, d=256, d_ff=256, n_tokens=200)
+    layer = W.make_layer(w, 0, DEV)
+    layer["bias"] = torch.zeros_like(layer["bias"])
+    layer["bias"][2] = 5.0
+    m, x, layer, out, r = run(w, layer=layer)
+    res = full_check(w, x, layer, out, r)
+    assert res["counts"][2] == 200
+
+
 def test_fp8_quantised_rows_match_the_oracle():
     """The dispatch's e4m3 rows: each grouped row holds the codes and group
     scales of its token's normalised row (oracle RMSNorm, quantised by the
