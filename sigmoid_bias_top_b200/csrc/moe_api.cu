@@ -9,9 +9,9 @@
 //               the router matrix split into three bf16 parts)
 //   2 dispatch  per-expert counts, offsets, row-tile prefix, perm / inv
 //   3 gate_up   grouped GEMM over the grouped normalised rows, SiLU(gate)*up
-//               (tcgen05 for bf16: 128-row tiles on single CTAs, or tiles of
-//               256 weight rows x up to 256 tokens on CTA pairs once the mean
-//               load reaches 256 rows per expert; SIMT for fp32)
+//               (tcgen05 for bf16: tiles of 256 weight rows x up to 256
+//               tokens on CTA pairs, or with MOE_TC_PAIR=0 128-token tiles on
+//               single CTAs; SIMT for fp32)
 //   4 down      grouped GEMM
 // (bf16 batches of at most 32 rows per expert on average fuse 3 and 4 into one
 // persistent kernel. FP8_BLOCK layers always do: their dispatch writes e4m3
