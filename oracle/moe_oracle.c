@@ -141,7 +141,7 @@ static void quant_groups(int n, double *v, uint8_t *codes, float *scales, int mu
     }
 }
 
-static double ld(const void *p, int dtype, size_t i)
+static inline __attribute__((always_inline)) double ld(const void *p, int dtype, size_t i)
 {
     if (dtype == OR_F32) return (double)((const float *)p)[i];
     if (dtype == OR_BF16) {
@@ -157,7 +157,8 @@ static double ld(const void *p, int dtype, size_t i)
 /* Element (r, c) of a [rows][cols] expert matrix starting at element `base`
  * of w: the stored value, times its 128x128 block's scale when sc != NULL
  * (sc points at this matrix's [rows/128][cols/128] scales). */
-static double wval(const void *w, int wdt, size_t base, int cols, int rows, int r, int c,
+static inline __attribute__((always_inline)) double wval(const void *w, int wdt, size_t base,
+                                                          int cols, int rows, int r, int c,
                    const float *sc, int mutation)
 {
     double v = ld(w, wdt, base + (size_t)r * cols + c);
