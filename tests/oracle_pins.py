@@ -219,6 +219,20 @@ def pin_identical_experts(mut):
     np.testing.assert_allclose(res["out"], want.numpy(), rtol=1e-12, atol=1e-12)
 
 
+def pin_routed_scale_is_linear(mut):
+    """The routed scale multiplies the normalised weights («Biased Routing»
+    §"The router has two different scores": the factor is 1 for the
+    checkpoint), so out - x scales with it exactly; a scale applied before
+    the normalisation would cancel instead."""
+    E, d, I, k = 6, 16, 8, 3
+    layer = rand_layer(E, d, I, seed=81)
+    x = rand_x(9, d, 81)
+    o1 = oracle.forward(x, layer, k=k, eps=EPS, routed_scale=1.0, mutation=mut)["out"]
+    o3 = oracle.forward(x, layer, k=k, eps=EPS, routed_scale=3.0, mutation=mut)["out"]
+    xd = x.double().numpy()
+    np.testing.assert_allclose(o3 - xd, 3.0 * (o1 - xd), rtol=1e-13, atol=1e-15)
+
+
 # ---------------------------------------------------------------- FP8_BLOCK
 # "LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell" (inferencekey.com,
 # section "Für Engineers", paragraph "Quantisierung"): weights FP8 static in
@@ -425,6 +439,7 @@ def pin_fp8_zero_block_scale(mut):
 PINS = [pin_five_candidate, pin_rmsnorm, pin_router_sigmoid, pin_weights_sum_below_one,
         pin_k1, pin_tie_break, pin_brute_force_subsets, pin_zero_bias_is_logit_topk,
         pin_bias_shift_invariance, pin_all_selected_bias_invariance,
-        pin_zero_down_is_identity, pin_identical_experts, pin_e4m3_codec, pin_fp8_quant,
+        pin_zero_down_is_identity, pin_identical_experts, pin_routed_scale_is_linear,
+        pin_e4m3_codec, pin_fp8_quant,
         pin_fp8_expert_blocks, pin_fp8_forward_error_bound, pin_fp8_scale_code_trade,
         pin_fp8_sign_symmetry, pin_fp8_zero_block_scale]
