@@ -25,6 +25,8 @@ MUTATIONS = {
     "no_eps": 4, "no_gain": 5, "silu_on_up": 6, "tie_high": 7,
     "no_residual": 8, "mean_not_sum": 9, "slot_swap": 10, "down_transposed": 11,
     "fp8_scale_transposed": 12, "fp8_no_act_quant": 13, "fp8_no_max": 14,
+    "margin_zero": 15, "margin_worst_unselected": 16, "margin_on_s": 17,
+    "forced_ignored": 18, "forced_weights_own_choice": 19,
 }
 
 _lib = None

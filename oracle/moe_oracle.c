@@ -78,7 +78,12 @@ enum {
     MUT_FP8_SCALE_T = 12,     /* weight block scales read as [col/128][row/128] */
     MUT_FP8_NO_ACT_QUANT = 13,/* SiLU(gate)*up not quantised before down       */
     MUT_FP8_NO_MAX = 14,      /* activation scale amax instead of amax/448     */
-    MUT_COUNT = 15
+    MUT_MARGIN_ZERO = 15,     /* margin reported as 0 for every token          */
+    MUT_MARGIN_WORST = 16,    /* margin against the WORST unselected expert    */
+    MUT_MARGIN_ON_S = 17,     /* margin on the unbiased s instead of c = s + b */
+    MUT_FORCED_IGNORED = 18,  /* a forced selection is ignored                 */
+    MUT_FORCED_WEIGHTS_OWN = 19, /* forced experts, but weights of the oracle's own choice */
+    MUT_COUNT = 20
 };
 
 /* Value of an e4m3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa
@@ -219,33 +224,44 @@ static double route_one(int d, int E, int k, double eps, double scale,
             c[e] = s[e] + (double)bias[e];
     }
 
+    /* The oracle's own choice: k rounds of arg-max over the biased scores,
+     * then the margin between the last selected and the best unselected. */
     double margin = INFINITY;
-    if (forced) {
-        for (int j = 0; j < k; ++j) sel[j] = forced[j];
-    } else {
-        unsigned char *taken = (unsigned char *)calloc((size_t)E, 1);
-        for (int j = 0; j < k; ++j) {
-            int best = -1;
-            for (int e = 0; e < E; ++e) {
-                if (taken[e]) continue;
-                if (best < 0 || c[e] > c[best] ||
-                    (mutation == MUT_TIE_HIGH && c[e] == c[best]))
-                    best = e;
-            }
-            taken[best] = 1;
-            sel[j] = best;
+    unsigned char *taken = (unsigned char *)calloc((size_t)(unsigned)E, 1);
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || c[e] > c[best] ||
+                (mutation == MUT_TIE_HIGH && c[e] == c[best]))
+                best = e;
         }
-        if (k < E) {
-            int nxt = -1;
-            for (int e = 0; e < E; ++e)
-                if (!taken[e] && (nxt < 0 || c[e] > c[nxt])) nxt = e;
-            margin = c[sel[k - 1]] - c[nxt];
+        taken[best] = 1;
+        sel[j] = best;
+    }
+    if (k < E) {
+        const double *key = (mutation == MUT_MARGIN_ON_S) ? s : c;
+        int nxt = -1;
+        for (int e = 0; e < E; ++e) {
+            if (taken[e]) continue;
+            if (nxt < 0 || (mutation == MUT_MARGIN_WORST ? key[e] < key[nxt] : key[e] > key[nxt]))
+                nxt = e;
         }
-        free(taken);
-        if (mutation == MUT_SLOT_SWAP)
-            for (int j = 0; j < k / 2; ++j) {
-                int32_t t = sel[j]; sel[j] = sel[k - 1 - j]; sel[k - 1 - j] = t;
-            }
+        margin = key[sel[k - 1]] - key[nxt];
+        if (mutation == MUT_MARGIN_ZERO) margin = 0.0;
+    }
+    free(taken);
+    if (mutation == MUT_SLOT_SWAP)
+        for (int j = 0; j < k / 2; ++j) {
+            int32_t t = sel[j]; sel[j] = sel[k - 1 - j]; sel[k - 1 - j] = t;
+        }
+    /* A forced selection (slot order as given) replaces the own choice; the
+     * margin then does not apply. */
+    const int use_forced = forced && mutation != MUT_FORCED_IGNORED;
+    if (use_forced) {
+        margin = INFINITY;
+        if (mutation != MUT_FORCED_WEIGHTS_OWN)
+            for (int j = 0; j < k; ++j) sel[j] = forced[j];
     }
 
     double sum = 0.0;
@@ -256,6 +272,8 @@ static double route_one(int d, int E, int k, double eps, double scale,
         double num = (mutation == MUT_BIASED_WEIGHTS) ? c[sel[j]] : s[sel[j]];
         w[j] = scale * (num / den);
     }
+    if (use_forced && mutation == MUT_FORCED_WEIGHTS_OWN)
+        for (int j = 0; j < k; ++j) sel[j] = forced[j];
     return margin;
 }
 

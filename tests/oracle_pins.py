@@ -233,6 +233,93 @@ def pin_routed_scale_is_linear(mut):
     np.testing.assert_allclose(o3 - xd, 3.0 * (o1 - xd), rtol=1e-13, atol=1e-15)
 
 
+def pin_margin(mut):
+    """The margin c_(k) - c_(k+1) between the last selected and the best
+    unselected biased score, which decides where the GPU selection must be
+    exact. (a) A zero router gives s = 1/2 for every expert, so c = 1/2 + b and
+    the margin is the gap between the k-th and (k+1)-th largest stored biases,
+    exactly; (b) two biases tied at ranks k and k+1 give a margin of exactly
+    0; (c) hand-set logits whose biased order differs from the unbiased one
+    give the gap of the sorted biased scores; (d) random tokens: the gap
+    between ranks k and k+1 of numpy's sort of s + b; (e) k = E gives inf."""
+    d, E = 8, 8
+    b = np.array([0.30, -0.10, 0.25, 0.05, -0.40, 0.125, 0.0, -0.2], np.float32)
+    layer = {"norm_gain": torch.ones(d), "router_w": torch.zeros(E, d),
+             "bias": torch.from_numpy(b)}
+    x = torch.ones(1, d)
+    r = oracle.route(x, layer, k=3, eps=EPS, mutation=mut)
+    assert r["idx"][0].tolist() == [0, 2, 5], r["idx"][0]
+    bd = b.astype(np.float64)
+    want = (0.5 + bd[5]) - (0.5 + bd[3])          # exact in double
+    assert r["margin"][0] == want, (r["margin"][0], want)
+    b2 = b.copy()
+    b2[3] = b2[5]                                   # tie at ranks 3 and 4
+    r = oracle.route(x, dict(layer, bias=torch.from_numpy(b2)), k=3, eps=EPS, mutation=mut)
+    assert r["idx"][0].tolist() == [0, 2, 3] and r["margin"][0] == 0.0, (r["idx"], r["margin"])
+    # (c) logits 1.5, -2.25, 0, 3.75, -0.5, 0.125 with biases that reorder them
+    E6 = 6
+    l = torch.tensor([1.5, -2.25, 0.0, 3.75, -0.5, 0.125], dtype=torch.float64)
+    b6 = torch.tensor([0.0, 0.6, 0.0, -0.5, 0.0, 0.3], dtype=torch.float32)
+    layer6 = {"norm_gain": torch.ones(d), "router_w": (l / d)[:, None].expand(E6, d).float(),
+              "bias": b6}
+    r = oracle.route(x, layer6, k=2, eps=EPS, mutation=mut)
+    c = torch.sigmoid(l / math.sqrt(1 + EPS)).numpy() + b6.double().numpy()
+    # c ~ [0.818, 0.695, 0.5, 0.477, 0.378, 0.831]: experts 5, 0 selected, 1 next
+    assert r["idx"][0].tolist() == [5, 0], r["idx"][0]
+    np.testing.assert_allclose(r["margin"][0], c[0] - c[1], rtol=1e-12, atol=0)
+    # (d) random tokens against a sort
+    E, k = 16, 4
+    layer = rand_layer(E, 32, 4, seed=23, bias_scale=0.2)
+    rr = oracle.route(rand_x(60, 32, 23), layer, k=k, eps=EPS, mutation=mut)
+    cs = -np.sort(-(rr["s"] + layer["bias"].double().numpy()[None, :]), axis=1)
+    np.testing.assert_allclose(rr["margin"], cs[:, k - 1] - cs[:, k], rtol=1e-12, atol=1e-15)
+    # (e) every expert selected: nothing to displace
+    r = oracle.route(x, dict(layer6), k=E6, eps=EPS, mutation=mut)
+    assert np.isinf(r["margin"][0])
+
+
+def pin_forced_selection(mut):
+    """A forced selection replaces the oracle's choice slot by slot, weights
+    included: (a) forcing the oracle's own selection reproduces its output bit
+    for bit; (b) forcing, per token, the three experts with the LOWEST biased
+    scores in ascending order (never the oracle's choice, and not in its slot
+    order) gives idx = the forced slots, w_j = s_f(j) / (sum_j s_f(j) + eps)
+    and out = x + sum_j w_j SwiGLU_f(j)(xn), all written with
+    torch.nn.functional in float64; (c) the forced rows follow the listed
+    tokens, not the token ids."""
+    E, d, I, k = 6, 16, 8, 3
+    layer = rand_layer(E, d, I, seed=29, bias_scale=0.3)
+    x = rand_x(5, d, 29)
+    own = oracle.forward(x, layer, k=k, eps=EPS, mutation=mut)
+    again = oracle.forward(x, layer, k=k, eps=EPS, forced=own["idx"], mutation=mut)
+    assert np.array_equal(again["out"], own["out"]) and np.array_equal(again["idx"], own["idx"])
+    # (b) an independent float64 computation of the forced mixture
+    xd = x.double()
+    xn = F.rms_norm(xd, (d,), weight=layer["norm_gain"].double(), eps=EPS)
+    s = torch.sigmoid(xn @ layer["router_w"].double().T)
+    c = s + layer["bias"].double()[None, :]
+    forced = torch.argsort(c, dim=1)[:, :k].to(torch.int32)   # lowest c, ascending
+    got = oracle.forward(x, layer, k=k, eps=EPS, forced=forced.numpy(), mutation=mut)
+    assert np.array_equal(got["idx"], forced.numpy()), (got["idx"], forced)
+    sf = torch.gather(s, 1, forced.long())
+    w = sf / (sf.sum(1, keepdim=True) + EPS)
+    np.testing.assert_allclose(got["w"], w.numpy(), rtol=1e-13, atol=0)
+    want = xd.clone()
+    for t in range(x.shape[0]):
+        for j in range(k):
+            e = int(forced[t, j])
+            Wg, Wu = layer["w_gate_up"][e, :I].double(), layer["w_gate_up"][e, I:].double()
+            y = F.linear(F.silu(F.linear(xn[t], Wg)) * F.linear(xn[t], Wu),
+                         layer["w_down"][e].double())
+            want[t] += w[t, j] * y
+    np.testing.assert_allclose(got["out"], want.numpy(), rtol=1e-12, atol=1e-12)
+    # (c) a token subset in another order, each with its own forced row
+    toks = np.array([4, 1])
+    sub = oracle.forward(x, layer, k=k, eps=EPS, tokens=toks, forced=forced.numpy()[toks],
+                         mutation=mut)
+    np.testing.assert_array_equal(sub["out"], got["out"][toks])
+
+
 # ---------------------------------------------------------------- FP8_BLOCK
 # "LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell" (inferencekey.com,
 # section "Für Engineers", paragraph "Quantisierung"): weights FP8 static in
@@ -440,6 +527,6 @@ PINS = [pin_five_candidate, pin_rmsnorm, pin_router_sigmoid, pin_weights_sum_bel
         pin_k1, pin_tie_break, pin_brute_force_subsets, pin_zero_bias_is_logit_topk,
         pin_bias_shift_invariance, pin_all_selected_bias_invariance,
         pin_zero_down_is_identity, pin_identical_experts, pin_routed_scale_is_linear,
-        pin_e4m3_codec, pin_fp8_quant,
+        pin_margin, pin_forced_selection, pin_e4m3_codec, pin_fp8_quant,
         pin_fp8_expert_blocks, pin_fp8_forward_error_bound, pin_fp8_scale_code_trade,
         pin_fp8_sign_symmetry, pin_fp8_zero_block_scale]

@@ -14,15 +14,23 @@ Rules (the tolerances the tests assert):
   * mixture weights agree to 1e-5 relative (fp32 sigmoid vs fp64);
   * outputs: per token ||o_gpu - o_ref|| / ||o_ref|| <= 1e-2 for bf16 storage
     (FP8_BLOCK layers store x and out as bf16 too), 1e-5 for fp32 storage;
-  * FP8_BLOCK layers also bound the MoE part alone: per token
-    ||(o_gpu - x) - (o_ref - x)|| / ||o_ref - x|| <= 2e-2 + 2^-8 ||o_ref|| /
-    ||o_ref - x||. The oracle applies the same e4m3 quantisation, so what
-    remains is fp32 summation order, the bf16 rounding of the expert outputs,
-    the rare e4m3 code that rounds the other way because the two sides' fp32
-    inputs differ in the last bits (one code step is 1/16 of one value out of
-    128), and the bf16 rounding of out itself, at most 2^-8 of |out| per
-    element, which the second term admits (it dominates when the MoE part is
-    small beside the residual).
+  * the MoE part alone is bounded too, since the residual x dominates ||out||
+    (on the decode step the MoE part is under a fifth of it, so the bound on
+    out alone would admit a 5% error in the part the kernels compute): per
+    token ||(o_gpu - x) - (o_ref - x)|| / ||o_ref - x|| <= DELTA_TOL + u
+    ||o_ref|| / ||o_ref - x||, where u is the rounding of the stored out
+    (2^-8 of |out| per element for bf16, 2^-24 for fp32), which the second
+    term admits. DELTA_TOL is 1e-2 for bf16 layers (the GPU rounds the
+    normalised rows, SiLU(gate)*up and the expert outputs to bf16, 2^-9
+    relative each), 2e-2 for FP8_BLOCK layers (the oracle applies the same
+    e4m3 quantisation, so what remains is fp32 summation order, the bf16
+    rounding of the expert outputs and the rare e4m3 code that rounds the
+    other way because the two sides' fp32 inputs differ in the last bits: one
+    code step is 1/16 of one value out of 128) and 1e-4 for fp32 layers;
+  * near ties are rare: the number of tokens whose margin is at most 1e-3 is
+    bounded by NEAR_FRAC of the batch plus NEAR_SLACK (the workloads have
+    4-10%), so a margin computed too small cannot move most tokens out of the
+    exact checks.
 """
 from __future__ import annotations
 
@@ -34,7 +42,9 @@ import oracle
 MARGIN = 1e-3
 ORDER_GAP = 1e-5   # selected experts closer than this may swap slots under fp32 rounding
 TOL = {"bf16": 1e-2, "f32": 1e-5, "fp8": 1e-2}
-DELTA_TOL = {"fp8": 2e-2}
+DELTA_TOL = {"bf16": 1e-2, "fp8": 2e-2, "f32": 1e-4}
+OUT_ROUND = {"bf16": 2.0 ** -8, "fp8": 2.0 ** -8, "f32": 2.0 ** -24}
+NEAR_FRAC, NEAR_SLACK = 0.2, 2
 W_RTOL = 1e-5
 
 
@@ -67,6 +77,9 @@ def check_routing(x_cpu, layer_cpu, k, eps, scale, r_gpu):
     c_gpu_sel = np.take_along_axis(c, idx.astype(np.int64), 1)
     assert np.all(np.diff(c_gpu_sel, axis=1) <= ORDER_GAP), "GPU slots not in descending c"
     # near ties: every GPU-selected expert is within MARGIN of the k-th best
+    n_near = int((~clear).sum())
+    assert n_near <= NEAR_FRAC * N + NEAR_SLACK, (
+        f"{n_near} of {N} tokens have margin <= {MARGIN}: more near ties than the inputs allow")
     ck = np.take_along_axis(c, ref["idx"][:, -1:].astype(np.int64), 1)[:, 0]
     for t in np.where(~clear)[0]:
         sel = idx[t]
@@ -76,7 +89,7 @@ def check_routing(x_cpu, layer_cpu, k, eps, scale, r_gpu):
     s_sel = np.take_along_axis(ref["s"], idx.astype(np.int64), 1)
     w_ref = scale * s_sel / (s_sel.sum(1, keepdims=True) + eps)
     np.testing.assert_allclose(w, w_ref, rtol=W_RTOL, atol=1e-7)
-    return ref, idx, int((~clear).sum())
+    return ref, idx, n_near
 
 
 def check_dispatch(idx, n_experts, r_gpu):
@@ -98,12 +111,11 @@ def check_outputs(x_cpu, layer_cpu, k, eps, scale, out_gpu, idx, tokens, dtype):
     worst = int(np.argmax(err))
     assert err.max() <= tol, (f"max rel-L2 {err.max():.3e} > {tol} at token {tokens[worst]}; "
                               f"MoE-delta rel err {delta_err[worst]:.3e}")
-    if dtype in DELTA_TOL:
-        dn = np.maximum(np.linalg.norm(ref["out"] - x, axis=1), 1e-30)
-        allowed = DELTA_TOL[dtype] + 2.0 ** -8 * np.linalg.norm(ref["out"], axis=1) / dn
-        wd = int(np.argmax(delta_err / allowed))
-        assert np.all(delta_err <= allowed), (
-            f"MoE-delta rel-L2 {delta_err[wd]:.3e} > {allowed[wd]:.3e} at token {tokens[wd]}")
+    dn = np.maximum(np.linalg.norm(ref["out"] - x, axis=1), 1e-30)
+    allowed = DELTA_TOL[dtype] + OUT_ROUND[dtype] * np.linalg.norm(ref["out"], axis=1) / dn
+    wd = int(np.argmax(delta_err / allowed))
+    assert np.all(delta_err <= allowed), (
+        f"MoE-delta rel-L2 {delta_err[wd]:.3e} > {allowed[wd]:.3e} at token {tokens[wd]}")
     return float(err.max()), float(delta_err.max())
 
 
