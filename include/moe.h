@@ -171,12 +171,17 @@ int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream);
  * as moe_forward's routing (see moe_debug_routing). All pointers are device
  * pointers owned by the caller; x, norm_gain and router_w 16-byte aligned.
  * Limits of the fixed scratch: n_tokens <= 4096 (else MOE_ERR_TOO_MANY_TOKENS),
- * n_experts <= 64 and d <= 2048 (else MOE_ERR_UNSUPPORTED_SHAPE), d % 4 == 0,
- * 1 <= top_k <= min(n_experts, 8). The scratch is one array compiled into the
- * library, about 1.1 MB on every GPU that loads it, held until the process
- * exits; a device's first call looks its address up (make that first call
- * before any stream capture). Calls share the array: calls that overlap on
- * the GPU race, calls ordered on one stream do not. Asynchronous on stream. */
+ * n_experts <= 64 and d <= 2048 (else MOE_ERR_UNSUPPORTED_SHAPE); shapes as
+ * moe_create takes them: d % 4 == 0 for MOE_F32 x, d % 64 == 0 for MOE_BF16 x,
+ * 1 <= top_k <= min(n_experts, 8) (else MOE_ERR_UNSUPPORTED_SHAPE). The
+ * scratch is one array compiled into the library, about 1.1 MB on every GPU
+ * that loads it, held until the process exits; a device's first call looks
+ * its address up (make that first call before any stream capture). Calls
+ * share the array: calls that overlap on the GPU race, calls ordered on one
+ * stream do not. Asynchronous on stream. Device-side failure: there is no
+ * context and so no moe_status here; if the router's bounded wait for its
+ * input copies runs out (1 s), every idx of the call is set to -1 and every
+ * w to NaN. */
 int moe_route_noalloc(const void *x, int dtype, const float *norm_gain, const float *router_w,
                       const float *expert_bias, int n_tokens, int d, int n_experts, int top_k,
                       float eps, float routed_scale, int32_t *idx, float *w, void *stream);

@@ -104,12 +104,25 @@ def route_noalloc(x, layer: Dict, top_k: int, eps: float = 1e-6, routed_scale: f
     capture, allocator-free serving loops); idx and w may be passed in
     preallocated so that the call itself allocates nothing."""
     import torch
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"x must be float32 or bfloat16, got {x.dtype}")
+    if x.dim() != 2 or not x.is_contiguous() or not x.is_cuda:
+        raise ValueError("x must be a contiguous [n, d] CUDA tensor")
     n, d = x.shape
     E = layer["router_w"].shape[0]
+    for name, want in (("norm_gain", (d,)), ("router_w", (E, d)), ("bias", (E,))):
+        t = layer[name]
+        if (t.dtype != torch.float32 or tuple(t.shape) != want or not t.is_contiguous()
+                or t.device != x.device):
+            raise ValueError(f"{name} must be a contiguous float32 {want} tensor on {x.device}")
     if idx is None:
         idx = torch.empty(n, top_k, dtype=torch.int32, device=x.device)
     if w is None:
         w = torch.empty(n, top_k, dtype=torch.float32, device=x.device)
+    for name, t, dt_ in (("idx", idx, torch.int32), ("w", w, torch.float32)):
+        if (t.dtype != dt_ or tuple(t.shape) != (n, top_k) or not t.is_contiguous()
+                or t.device != x.device):
+            raise ValueError(f"{name} must be a contiguous {dt_} ({n}, {top_k}) tensor on {x.device}")
     dt = MOE_BF16 if x.dtype == torch.bfloat16 else MOE_F32
     _check(lib().moe_route_noalloc(x.data_ptr(), dt, layer["norm_gain"].data_ptr(),
                                    layer["router_w"].data_ptr(), layer["bias"].data_ptr(), n, d, E,

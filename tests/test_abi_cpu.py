@@ -88,6 +88,36 @@ def test_route_noalloc_takes_the_storage_type_of_x():
     assert L.moe_route_noalloc(args[0], sb.MOE_FP8_BLOCK, *args[2:]) == -1
 
 
+def test_route_noalloc_refuses_shapes_before_device_work():
+    """Shapes outside what moe_create takes are refused on the host: bf16 rows
+    need d % 64 == 0 (the router copies whole row groups in 16-byte units),
+    fp32 rows d % 4 == 0; sizes beyond the fixed scratch are refused too."""
+    L = sb.lib()
+
+    def call(dtype, n, d, E, k):
+        return L.moe_route_noalloc(256, dtype, 256, 256, 256, n, d, E, k, 1e-6, 1.0, 256, 256,
+                                   None)
+    assert call(sb.MOE_BF16, 7, 100, 16, 4) == -2       # d % 8 == 4: odd row groups
+    assert call(sb.MOE_BF16, 7, 96, 16, 4) == -2        # d % 64 != 0
+    assert call(sb.MOE_F32, 7, 102, 16, 4) == -2        # d % 4 != 0
+    assert call(sb.MOE_F32, 7, 256, 16, 9) == -2        # k > 8
+    assert call(sb.MOE_F32, 7, 256, 4, 5) == -2         # k > E
+    assert call(sb.MOE_BF16, 4097, 2048, 64, 4) == -4   # beyond the scratch's tokens
+    assert call(sb.MOE_BF16, 8, 4096, 64, 4) == -2      # beyond its width
+    assert call(sb.MOE_BF16, 8, 2048, 128, 4) == -2     # beyond its experts
+    assert call(sb.MOE_BF16, 0, 2048, 64, 4) == 0       # empty batch: nothing to do
+
+
+def test_route_noalloc_binding_checks_tensors():
+    """The Python binding refuses other dtypes and non-contiguous tensors
+    before calling the library."""
+    layer = {"norm_gain": torch.ones(64), "router_w": torch.zeros(8, 64), "bias": torch.zeros(8)}
+    with pytest.raises(TypeError):
+        sb.route_noalloc(torch.zeros(4, 64, dtype=torch.float16), layer, 2)
+    with pytest.raises(ValueError):
+        sb.route_noalloc(torch.zeros(64, 4).t(), layer, 2)
+
+
 def test_calls_on_null_handle_are_rejected():
     L = sb.lib()
     assert L.moe_forward(None, None, None, 1, None) == -1
