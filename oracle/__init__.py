@@ -27,6 +27,8 @@ MUTATIONS = {
     "fp8_scale_transposed": 12, "fp8_no_act_quant": 13, "fp8_no_max": 14,
     "margin_zero": 15, "margin_worst_unselected": 16, "margin_on_s": 17,
     "forced_ignored": 18, "forced_weights_own_choice": 19,
+    "conv_lag_reversed": 20, "conv_centered": 21, "conv_gate_after": 22,
+    "conv_sequence_leak": 23, "conv_uv_swapped": 24,
 }
 
 _lib = None
@@ -47,6 +49,10 @@ def lib():
         L.oracle_e4m3.argtypes = [I, P, P, P, P]
         L.oracle_dispatch.argtypes = [I, I, I, P, P, P, P]
         L.oracle_set_threads.argtypes = [I]
+        L.oracle_dense_ffn.argtypes = [I, I, I, D, P, I, P, P, P, I, P, I]
+        L.oracle_shortconv.argtypes = [I, I, I, D, P, I, P, P, P, I, P, P, P, P, I]
+        L.oracle_dense_ffn.restype = I
+        L.oracle_shortconv.restype = I
         for f in (L.oracle_rmsnorm, L.oracle_route, L.oracle_forward, L.oracle_expert,
                   L.oracle_quant, L.oracle_e4m3, L.oracle_dispatch, L.oracle_set_threads,
                   L.oracle_num_mutations):
@@ -216,3 +222,48 @@ def dispatch(idx: np.ndarray, n_experts: int):
     _check(lib().oracle_dispatch(N, n_experts, k, idx.ctypes.data, counts.ctypes.data,
                                  offsets.ctypes.data, perm.ctypes.data), "oracle_dispatch")
     return {"counts": counts, "offsets": offsets, "perm": perm}
+
+
+# ---------------------------------------------------------------- neighbours
+def dense_ffn(x, layer, eps, mutation=0) -> np.ndarray:
+    """Dense feed-forward block: x + down(silu(gate xn) * (up xn)), xn =
+    RMSNorm(x) * norm_gain; layer holds norm_gain [d] f32, w_gate_up [2I,d]
+    and w_down [d,I] (f32 or bf16). Returns out [N,d] f64."""
+    xk, xp, xdt = _raw(x)
+    g = _f32(layer["norm_gain"])
+    wgu, wgp, wdt = _raw(layer["w_gate_up"])
+    wd, wdp, wdt2 = _raw(layer["w_down"])
+    assert wdt == wdt2
+    N, d = xk.shape
+    I = wgu.shape[0] // 2
+    out = np.zeros((N, d), np.float64)
+    _check(lib().oracle_dense_ffn(N, d, I, eps, xp, xdt, g.data_ptr(), wgp, wdp, wdt,
+                                  out.ctypes.data, mutation), "oracle_dense_ffn")
+    return out
+
+
+def shortconv(x, layer, eps, state_in=None, mutation=0):
+    """Short-convolution block on x [B,T,d]: x + w_out (u * conv3(g * v)),
+    [g; u; v] = w_in RMSNorm(x) * norm_gain. layer holds norm_gain [d] f32,
+    w_in [3d,d] and w_out [d,d] (f32 or bf16), conv [d,3] f32 indexed by lag.
+    state_in: optional [B,2,d] a vectors of positions -2, -1 per sequence.
+    Returns (out [B,T,d] f64, state_out [B,2,d] f64)."""
+    xk, xp, xdt = _raw(x)
+    B, T, d = xk.shape
+    g = _f32(layer["norm_gain"])
+    win, wip, wdt = _raw(layer["w_in"])
+    wo, wop, wdt2 = _raw(layer["w_out"])
+    assert wdt == wdt2
+    kc = _f32(layer["conv"])
+    assert tuple(kc.shape) == (d, 3)
+    sp = None
+    if state_in is not None:
+        st = np.ascontiguousarray(np.asarray(state_in, dtype=np.float64))
+        assert st.shape == (B, 2, d)
+        sp = st.ctypes.data
+    out = np.zeros((B, T, d), np.float64)
+    so = np.zeros((B, 2, d), np.float64)
+    _check(lib().oracle_shortconv(B, T, d, eps, xp, xdt, g.data_ptr(), wip, wop, wdt,
+                                  kc.data_ptr(), sp, out.ctypes.data, so.ctypes.data, mutation),
+           "oracle_shortconv")
+    return out, so

@@ -83,7 +83,12 @@ enum {
     MUT_MARGIN_ON_S = 17,     /* margin on the unbiased s instead of c = s + b */
     MUT_FORCED_IGNORED = 18,  /* a forced selection is ignored                 */
     MUT_FORCED_WEIGHTS_OWN = 19, /* forced experts, but weights of the oracle's own choice */
-    MUT_COUNT = 20
+    MUT_CONV_LAG_REVERSED = 20, /* conv tap l applied at lag 2 - l               */
+    MUT_CONV_CENTERED = 21,   /* conv window t-1 .. t+1 instead of t-2 .. t      */
+    MUT_CONV_GATE_AFTER = 22, /* g multiplied after the convolution, not before  */
+    MUT_CONV_SEQ_LEAK = 23,   /* history carried across sequences of the batch   */
+    MUT_CONV_UV_SWAPPED = 24, /* streams u and v taken in the other order        */
+    MUT_COUNT = 25
 };
 
 /* Value of an e4m3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa
@@ -497,5 +502,148 @@ int oracle_dispatch(int N, int E, int k, const int32_t *idx, int32_t *counts,
         for (int t = 0; t < N; ++t)
             for (int j = 0; j < k; ++j)
                 if (idx[(size_t)t * k + j] == e) perm[pos++] = t * k + j;
+    return 0;
+}
+
+
+/* ------------------------------------------------------------------------
+ * The neighbouring steps of the block ("LFM2.5-24B-A2B: Biased Routing,
+ * Short Convolutions and Ten KV Caches", section "The exact checkpoint": the
+ * first two layers are dense and convolutional; a block normalises before
+ * its mixer and before its feed-forward network, each with a residual).
+ *
+ * Dense feed-forward: out = x + down( silu(gate xn) * (up xn) ), xn the
+ * RMSNorm of x, gate/up packed [2I][d] (gate rows first), down [d][I]: the
+ * gated SiLU MLP of one expert, applied to every token with weight 1. */
+int oracle_dense_ffn(int N, int d, int I, double eps, const void *x, int xdt, const float *gain,
+                     const void *w_gate_up, const void *w_down, int wdt, double *out,
+                     int mutation)
+{
+    if (N < 0 || d <= 0 || I <= 0 || wdt == OR_E4M3) return -1;
+#pragma omp parallel
+    {
+        double *xn = (double *)malloc(sizeof(double) * (size_t)d);
+        double *xq = (double *)malloc(sizeof(double) * (size_t)d);
+        double *gt = (double *)malloc(sizeof(double) * (size_t)I);
+        double *up = (double *)malloc(sizeof(double) * (size_t)I);
+        double *a = (double *)malloc(sizeof(double) * (size_t)I);
+        double *y = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int t = 0; t < N; ++t) {
+            rmsnorm_row(d, eps, x, xdt, (size_t)t, gain, xn, mutation);
+            expert_mlp(d, I, xn, w_gate_up, w_down, wdt, NULL, NULL, 0, xq, gt, up, a, y,
+                       mutation);
+            double *o = out + (size_t)t * d;
+            for (int j = 0; j < d; ++j)
+                o[j] = ((mutation == MUT_NO_RESIDUAL) ? 0.0 : ld(x, xdt, (size_t)t * d + j)) + y[j];
+        }
+        free(xn); free(xq); free(gt); free(up); free(a); free(y);
+    }
+    return 0;
+}
+
+/* Short-convolution block ("LFM2.5-24B-A2B: Biased Routing, Short
+ * Convolutions and Ten KV Caches", section "A short convolution is a local
+ * mixer, not an embedding lookup"): the normalised row is projected into
+ * three width-d streams g, u, v (B, C and x of the implementation; packed
+ * w_in [3d][d] in that order); a = g * v; a depthwise causal convolution of
+ * width three, c_t = sum_{l=0..2} k[l] * a_{t-l} per channel (k indexed by
+ * lag: kconv[channel][l] multiplies a_{t-l}); y = u * c; out = x + w_out y,
+ * w_out [d][d]. No bias in the projections or the convolution, no
+ * activation on the gates (the page: direct linear projections).
+ * x is [B][T][d]; each of the B sequences has its own history: the a vectors
+ * of its two positions before t = 0, state_in[b][0] (position -2) and
+ * state_in[b][1] (position -1), or zeros when state_in is NULL. state_out
+ * (may be NULL) receives each sequence's a vectors of its last two
+ * positions in the same layout (for T = 1: the old position -1, then a_0),
+ * so that running T1 then T2 tokens with the state carried equals running
+ * T1 + T2 at once. */
+int oracle_shortconv(int B, int T, int d, double eps, const void *x, int xdt, const float *gain,
+                     const void *w_in, const void *w_out, int wdt, const float *kconv,
+                     const double *state_in, double *out, double *state_out, int mutation)
+{
+    if (B < 0 || T < 0 || d <= 0 || wdt == OR_E4M3) return -1;
+    const size_t D = (size_t)d;
+    /* a of every position, with two history positions in front per sequence */
+    double *a = (double *)malloc(sizeof(double) * (size_t)B * (size_t)(T + 2) * D);
+    double *u = (double *)malloc(sizeof(double) * (size_t)B * (size_t)T * D);
+    double *g = (double *)malloc(sizeof(double) * (size_t)B * (size_t)T * D);
+    if (!a || !u || !g) { free(a); free(u); free(g); return -4; }
+    const int uo = (mutation == MUT_CONV_UV_SWAPPED) ? 2 : 1;   /* row block of u */
+    const int vo = (mutation == MUT_CONV_UV_SWAPPED) ? 1 : 2;   /* row block of v */
+    for (int b = 0; b < B; ++b) {
+        double *ab = a + (size_t)b * (T + 2) * D;
+        for (int j = 0; j < 2; ++j)
+            for (size_t c = 0; c < D; ++c) {
+                int src = b;
+                if (mutation == MUT_CONV_SEQ_LEAK) src = b - 1;  /* previous sequence's state */
+                ab[j * D + c] = (state_in && src >= 0) ? state_in[((size_t)src * 2 + j) * D + c] : 0.0;
+            }
+    }
+#pragma omp parallel
+    {
+        double *xn = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(dynamic, 4)
+        for (int r = 0; r < B * T; ++r) {
+            const int b = r / T, t = r % T;
+            rmsnorm_row(d, eps, x, xdt, (size_t)r, gain, xn, mutation);
+            double *ab = a + ((size_t)b * (T + 2) + 2 + t) * D;
+            for (size_t c = 0; c < D; ++c) {
+                double sg = 0.0, su = 0.0, sv = 0.0;
+                for (size_t j = 0; j < D; ++j) {
+                    sg += ld(w_in, wdt, c * D + j) * xn[j];
+                    su += ld(w_in, wdt, ((size_t)uo * D + c) * D + j) * xn[j];
+                    sv += ld(w_in, wdt, ((size_t)vo * D + c) * D + j) * xn[j];
+                }
+                g[(size_t)r * D + c] = sg;
+                u[(size_t)r * D + c] = su;
+                ab[c] = (mutation == MUT_CONV_GATE_AFTER) ? sv : sg * sv;
+            }
+        }
+        free(xn);
+    }
+    if (mutation == MUT_CONV_SEQ_LEAK) {
+        /* the history of sequence b > 0 is the previous sequence's last two a */
+        for (int b = B - 1; b >= 1; --b)
+            for (int j = 0; j < 2; ++j)
+                for (size_t c = 0; c < D; ++c)
+                    a[((size_t)b * (T + 2) + j) * D + c] =
+                        (T >= 2 - j) ? a[((size_t)(b - 1) * (T + 2) + T + j) * D + c] : 0.0;
+    }
+#pragma omp parallel
+    {
+        double *y = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(dynamic, 4)
+        for (int r = 0; r < B * T; ++r) {
+            const int b = r / T, t = r % T;
+            const double *ab = a + (size_t)b * (T + 2) * D;   /* position p at ab[(p + 2) D] */
+            for (size_t c = 0; c < D; ++c) {
+                double cv = 0.0;
+                for (int l = 0; l < 3; ++l) {
+                    int p = t - l;                               /* lag l */
+                    double k = (double)kconv[c * 3 + l];
+                    if (mutation == MUT_CONV_LAG_REVERSED) k = (double)kconv[c * 3 + (2 - l)];
+                    if (mutation == MUT_CONV_CENTERED) p = t + 1 - l;
+                    double av = (p + 2 < T + 2) ? ab[(size_t)(p + 2) * D + c] : 0.0;
+                    cv += k * av;
+                }
+                if (mutation == MUT_CONV_GATE_AFTER) cv *= g[(size_t)r * D + c];
+                y[c] = u[(size_t)r * D + c] * cv;
+            }
+            double *o = out + (size_t)r * D;
+            for (size_t j = 0; j < D; ++j) {
+                double acc = 0.0;
+                for (size_t c = 0; c < D; ++c) acc += ld(w_out, wdt, j * D + c) * y[c];
+                o[j] = ((mutation == MUT_NO_RESIDUAL) ? 0.0 : ld(x, xdt, (size_t)r * D + j)) + acc;
+            }
+        }
+        free(y);
+    }
+    if (state_out)
+        for (int b = 0; b < B; ++b)
+            for (int j = 0; j < 2; ++j)
+                memcpy(state_out + ((size_t)b * 2 + j) * D, a + ((size_t)b * (T + 2) + T + j) * D,
+                       sizeof(double) * D);
+    free(a); free(u); free(g);
     return 0;
 }

@@ -523,10 +523,134 @@ def pin_fp8_zero_block_scale(mut):
     assert np.abs(oa - o0).max() > 0
 
 
+# ------------------------------------------------- neighbouring steps of the block
+# «Biased Routing» §"The exact checkpoint" (the first two layers are dense and
+# convolutional; pre-norm and a residual around mixer and feed-forward) and
+# §"A short convolution is a local mixer, not an embedding lookup".
+
+def conv_layer(d, seed, dtype=torch.float32):
+    g = torch.Generator().manual_seed(seed)
+    return {"norm_gain": (1 + 0.1 * torch.randn(d, generator=g)).float(),
+            "w_in": (torch.randn(3 * d, d, generator=g) / math.sqrt(d)).to(dtype),
+            "w_out": (torch.randn(d, d, generator=g) / math.sqrt(d)).to(dtype),
+            "conv": torch.randn(d, 3, generator=g).float()}
+
+
+def conv_textbook(x, layer, eps=EPS, state=None):
+    """The block with torch.nn.functional in float64: rms_norm, one linear for
+    the three streams, a depthwise conv1d (weights reversed: conv1d's tap j
+    multiplies position t - 2 + j, i.e. lag 2 - j), a linear back."""
+    B, T, d = x.shape
+    xn = F.rms_norm(x.double(), (d,), weight=layer["norm_gain"].double(), eps=eps)
+    g, u, v = F.linear(xn, layer["w_in"].double()).split(d, dim=-1)
+    a = (g * v).transpose(1, 2)                              # [B, d, T]
+    hist = torch.zeros(B, d, 2, dtype=torch.float64) if state is None else \
+        torch.as_tensor(state).double().transpose(1, 2)
+    a = torch.cat([hist, a], dim=2)                          # positions -2 .. T-1
+    c = F.conv1d(a, layer["conv"].double().flip(1)[:, None, :], groups=d)   # [B, d, T]
+    y = u * c.transpose(1, 2)
+    return (x.double() + F.linear(y, layer["w_out"].double())).numpy()
+
+
+def pin_dense_ffn(mut):
+    """Dense feed-forward block = x + SwiGLU(RMSNorm(x)) written with
+    torch.nn.functional in float64; W_down = 0 gives x exactly."""
+    d, I = 24, 40
+    g = torch.Generator().manual_seed(13)
+    layer = {"norm_gain": (1 + 0.1 * torch.randn(d, generator=g)).float(),
+             "w_gate_up": (torch.randn(2 * I, d, generator=g) / math.sqrt(d)).float(),
+             "w_down": (torch.randn(d, I, generator=g) / math.sqrt(I)).float()}
+    x = rand_x(9, d, 13)
+    out = oracle.dense_ffn(x, layer, EPS, mutation=mut)
+    xn = F.rms_norm(x.double(), (d,), weight=layer["norm_gain"].double(), eps=EPS)
+    Wg, Wu = layer["w_gate_up"][:I].double(), layer["w_gate_up"][I:].double()
+    want = x.double() + F.linear(F.silu(F.linear(xn, Wg)) * F.linear(xn, Wu),
+                                 layer["w_down"].double())
+    np.testing.assert_allclose(out, want.numpy(), rtol=1e-12, atol=1e-12)
+    z = dict(layer, w_down=torch.zeros_like(layer["w_down"]))
+    assert np.array_equal(oracle.dense_ffn(x, z, EPS, mutation=mut), x.double().numpy())
+
+
+def pin_shortconv_textbook(mut):
+    """The short-convolution block against its torch.nn.functional form, with
+    and without a carried state, on two sequences."""
+    d, B, T = 12, 2, 7
+    layer = conv_layer(d, 17)
+    x = torch.randn(B, T, d, generator=torch.Generator().manual_seed(18))
+    out, _ = oracle.shortconv(x, layer, EPS, mutation=mut)
+    np.testing.assert_allclose(out, conv_textbook(x, layer), rtol=1e-11, atol=1e-12)
+    st = np.random.default_rng(19).normal(size=(B, 2, d))
+    out, _ = oracle.shortconv(x, layer, EPS, state_in=st, mutation=mut)
+    np.testing.assert_allclose(out, conv_textbook(x, layer, state=st), rtol=1e-11, atol=1e-12)
+
+
+def pin_shortconv_delta_kernels(mut):
+    """Closed forms: a delta kernel at lag 0 makes the block position-wise,
+    x + W_out (u g v); a delta at lag 1 is the identity shift, c_t = a_{t-1}
+    (zero before the sequence); zero u rows give out = x exactly."""
+    d, B, T = 8, 1, 6
+    layer = conv_layer(d, 21)
+    x = torch.randn(B, T, d, generator=torch.Generator().manual_seed(22))
+    xn = F.rms_norm(x.double(), (d,), weight=layer["norm_gain"].double(), eps=EPS)
+    g, u, v = F.linear(xn, layer["w_in"].double()).split(d, dim=-1)
+    Wo = layer["w_out"].double()
+    for lag in (0, 1):
+        k = torch.zeros(d, 3)
+        k[:, lag] = 1.0
+        out, _ = oracle.shortconv(x, dict(layer, conv=k), EPS, mutation=mut)
+        a = g * v
+        if lag == 1:
+            a = torch.cat([torch.zeros(B, 1, d, dtype=torch.float64), a[:, :-1]], dim=1)
+        want = x.double() + F.linear(u * a, Wo)
+        np.testing.assert_allclose(out, want.numpy(), rtol=1e-12, atol=1e-12)
+    w_in = layer["w_in"].clone()
+    w_in[d:2 * d] = 0.0
+    out, _ = oracle.shortconv(x, dict(layer, w_in=w_in), EPS, mutation=mut)
+    assert np.array_equal(out, x.double().numpy())
+
+
+def pin_shortconv_causal(mut):
+    """Receptive field of three positions, causal, per sequence: changing one
+    token changes only its own output and the next two, and no other
+    sequence of the batch."""
+    d, B, T = 8, 2, 9
+    layer = conv_layer(d, 23)
+    x = torch.randn(B, T, d, generator=torch.Generator().manual_seed(24))
+    o0, _ = oracle.shortconv(x, layer, EPS, mutation=mut)
+    for tp in (3, T - 1):
+        x2 = x.clone()
+        x2[0, tp] += 1.0
+        o1, _ = oracle.shortconv(x2, layer, EPS, mutation=mut)
+        changed = np.abs(o1 - o0).max(axis=2) > 0
+        want = np.zeros((B, T), bool)
+        want[0, tp:min(T, tp + 3)] = True
+        assert np.array_equal(changed, want), (tp, changed)
+
+
+def pin_shortconv_state_chaining(mut):
+    """Running T1 then T2 positions with the state carried equals running
+    T1 + T2 at once, outputs and final state bit for bit; decode (T = 1
+    steps) too."""
+    d, B, T = 8, 2, 7
+    layer = conv_layer(d, 25)
+    x = torch.randn(B, T, d, generator=torch.Generator().manual_seed(26))
+    full, s_full = oracle.shortconv(x, layer, EPS, mutation=mut)
+    a, s = oracle.shortconv(x[:, :4].contiguous(), layer, EPS, mutation=mut)
+    b, s2 = oracle.shortconv(x[:, 4:].contiguous(), layer, EPS, state_in=s, mutation=mut)
+    assert np.array_equal(np.concatenate([a, b], 1), full) and np.array_equal(s2, s_full)
+    st, outs = None, []
+    for t in range(T):
+        o, st = oracle.shortconv(x[:, t:t + 1].contiguous(), layer, EPS, state_in=st, mutation=mut)
+        outs.append(o)
+    assert np.array_equal(np.concatenate(outs, 1), full) and np.array_equal(st, s_full)
+
+
 PINS = [pin_five_candidate, pin_rmsnorm, pin_router_sigmoid, pin_weights_sum_below_one,
         pin_k1, pin_tie_break, pin_brute_force_subsets, pin_zero_bias_is_logit_topk,
         pin_bias_shift_invariance, pin_all_selected_bias_invariance,
         pin_zero_down_is_identity, pin_identical_experts, pin_routed_scale_is_linear,
         pin_margin, pin_forced_selection, pin_e4m3_codec, pin_fp8_quant,
         pin_fp8_expert_blocks, pin_fp8_forward_error_bound, pin_fp8_scale_code_trade,
-        pin_fp8_sign_symmetry, pin_fp8_zero_block_scale]
+        pin_fp8_sign_symmetry, pin_fp8_zero_block_scale,
+        pin_dense_ffn, pin_shortconv_textbook, pin_shortconv_delta_kernels,
+        pin_shortconv_causal, pin_shortconv_state_chaining]
