@@ -37,8 +37,10 @@ from sigmoid_bias_top_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (d2048,E64,top4,I1536) + % of HBM / bf16 TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DEFAULT_STEPS = {"decode": 2000, "prefill": 200, "skewed": 100, "stacked": 20, "tiny": 2000,
+DEFAULT_STEPS = {"decode": 2000, "prefill": 200, "skewed": 100, "stacked": 100, "tiny": 2000,
                  "verify": 1000, "decode_fp8": 2000, "prefill_fp8": 100}
+# measured after the headline workload in a default one-GPU run
+EXTRA = "prefill,skewed,stacked,verify,decode_fp8,prefill_fp8"
 ROTATE = 4  # distinct weight copies cycled through (each step reads >= 1 GB > L2)
 
 
@@ -198,11 +200,54 @@ def make_layers(w, device, n_copies):
     return [W.make_layer(w, l, device) for l in range(n)]
 
 
-def run_ours(args, w, world, rank, local):
+def roofline(w, dom, mean_ms, U, peaks, src, clk, timed_s):
+    """(bound, work per launch, achieved, peak, unit, peak key) of the
+    dominant kernel. Weight-streaming batches (fewer than 64 grouped rows per
+    active expert) are bound by HBM; the rest by the tensor cores, against the
+    burst bf16 peak unless the clocks saw the power cap or the timed region
+    lasted seconds (then the sustained one)."""
+    N = w.n_tokens
+    n_assign = N * w.top_k
+    bpe = 2 if w.dtype == "bf16" else 4
+    fp8 = w.dtype == "fp8"
+    if n_assign / max(U, 1) < 64:
+        if fp8:                  # FP8_BLOCK: both contractions in one launch
+            work = A.fp8_experts_bytes(U, n_assign, w.d, w.d_ff)
+        elif dom == "experts":   # both contractions in one launch
+            work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + A.down_bytes(U, w.d, w.d_ff, bpe)
+                    + 2 * n_assign * (w.d + w.d_ff) * bpe)
+        elif dom == "gate_up":
+            work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe)
+        elif dom == "down":
+            work = A.down_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe
+        else:
+            work = A.decode_bytes(U, N, w.d, w.d_ff, w.n_experts, bpe, bpe)
+        achieved = work / (mean_ms[dom] / 1e3) / 1e9
+        return "hbm", work, achieved, peaks["hbm_gbs"], "GB/s", "hbm_gbs"
+    if dom == "experts":
+        work = A.gate_up_flops(n_assign, w.d, w.d_ff) + A.down_flops(n_assign, w.d, w.d_ff)
+    else:
+        work = (A.gate_up_flops(n_assign, w.d, w.d_ff) if dom == "gate_up"
+                else A.down_flops(n_assign, w.d, w.d_ff))
+    achieved = work / (mean_ms[dom] / 1e3) / 1e12
+    sustained = "sw_power_cap" in clk.get("reasons", []) or timed_s >= 1.0
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = peaks.get(key, peaks["bf16_tflops"])
+    if fp8:  # e4m3 dense peak = the measured bf16 peak x the nominal 4.5 / 2.25
+        peak *= 2.0
+        key += " x 2 (e4m3 / bf16 nominal ratio)"
+    return "tensor", work, achieved, peak, "TFLOP/s", key
+
+
+def measure(w, args, steps, world, rank, local, headline):
+    """One workload: W warm-up steps, then `repeats` timed blocks of exactly
+    `steps` steps (each bracketed by barrier + synchronize, CUDA events on the
+    launching stream); the median block gives the throughput. Then a second,
+    separate pass of the same steps with events between the launches gives
+    the per-kernel durations. The headline workload also measures the
+    end-to-end path through host buffers and the oracle's CPU baseline."""
     from sigmoid_bias_top_b200 import MoeLayer
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    init_dist(world, "nccl")
     N = w.n_tokens
     layers = make_layers(w, dev, args.rotate)
     mods = [MoeLayer(l, w.top_k, w.eps, w.routed_scale, max_tokens=N) for l in layers]
@@ -230,33 +275,33 @@ def run_ours(args, w, world, rank, local):
 
     # routing statistics of the timed batches (distinct active experts per layer)
     active = []
-    for r in range(min(n_rot, len(mods)) if w.n_layers == 1 else 1):
+    for r in range(n_rot if w.n_layers == 1 else 1):
         mods[r].forward(xs[r % len(xs)], outs[0], stream)
         off = mods[r].debug_routing(N)["offsets"].cpu().numpy()
         active.append(int((np.diff(off) > 0).sum()))
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.15)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    block_s = []
+    for _ in range(args.repeats):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        block_s.append(e0.elapsed_time(e1) / 1e3)
     clk = clocks.stop()
     barrier(world)
-    local_s = e0.elapsed_time(e1) / 1e3
-    # per-kernel durations: a second pass of the same steps with CUDA events
-    # recorded between the launches on the launching stream (the events
-    # separate the launches, so these durations include launch gaps)
+    local_s = statistics.median(block_s)
     for m in mods:
         m.profile(True)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i)
     torch.cuda.synchronize()
     ktimes = {}
@@ -265,102 +310,116 @@ def run_ours(args, w, world, rank, local):
             ktimes.setdefault(name, []).append(ms)
         m.profile(False)
         assert m.status() == 0
-    value, secs = job_throughput(N * args.steps, local_s, world, dev)
-    ms_per_step = secs / args.steps * 1e3
-
-    # end to end through the C ABI with host buffers (H2D + forward + D2H per step)
-    xh = xs[0].cpu().pin_memory()
-    oh = torch.empty_like(xh).pin_memory()
-    e2e_steps = max(10, min(args.steps, 500))
-    for _ in range(3):
-        mods[0].forward_host(xh, oh)
-    barrier(world)
-    t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        if w.n_layers > 1:
-            # first block from host, the chain on device, last block back to host
-            xd = xh.to(dev, non_blocking=True)
-            h = xd
-            for l, m in enumerate(mods):
-                dst = outs[l & 1]
-                m.forward(h, dst, stream)
-                h = dst
-            oh.copy_(h, non_blocking=True)
-            torch.cuda.synchronize()
-        else:
-            mods[0].forward_host(xh, oh)
-    e2e_local = time.perf_counter() - t0
-    e2e_value, _ = job_throughput(N * e2e_steps, e2e_local, world, dev)
-    nbytes = xh.numel() * xh.element_size()
-
-    # roofline of the dominant kernel
-    peaks, src = load_peaks()
-    mean_ms = {k: float(np.mean(v)) for k, v in ktimes.items()}   # per launch
-    per_layer = mean_ms
-    dom = max(mean_ms, key=mean_ms.get)
+    value, secs = job_throughput(N * steps, local_s, world, dev)
+    per_layer = {k: float(np.mean(v)) for k, v in ktimes.items()}   # per launch
+    dom = max(per_layer, key=per_layer.get)
     U = float(np.mean(active))
-    n_assign = N * w.top_k
-    bpe = 2 if w.dtype == "bf16" else 4
-    fp8 = w.dtype == "fp8"
-    tc_peak_key = "bf16_tflops_sustained"
-    if N * w.top_k / max(U, 1) < 64:  # weight-streaming regime: HBM-bound
-        bound = "hbm"
-        if fp8:                # FP8_BLOCK: both contractions in one launch
-            work = A.fp8_experts_bytes(U, n_assign, w.d, w.d_ff)
-        elif dom == "experts":   # both contractions in one launch
-            work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + A.down_bytes(U, w.d, w.d_ff, bpe)
-                    + 2 * n_assign * (w.d + w.d_ff) * bpe)
-        elif dom == "gate_up":
-            work = (A.gate_up_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe)
-        elif dom == "down":
-            work = A.down_bytes(U, w.d, w.d_ff, bpe) + n_assign * (w.d + w.d_ff) * bpe
-        else:
-            work = A.decode_bytes(U, N, w.d, w.d_ff, w.n_experts, bpe, bpe)
-        achieved = work / (mean_ms[dom] / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        unit = "GB/s"
-    else:
-        bound = "tensor"
-        if dom == "experts":
-            work = A.gate_up_flops(n_assign, w.d, w.d_ff) + A.down_flops(n_assign, w.d, w.d_ff)
-        else:
-            work = (A.gate_up_flops(n_assign, w.d, w.d_ff) if dom == "gate_up"
-                    else A.down_flops(n_assign, w.d, w.d_ff))
-        achieved = work / (mean_ms[dom] / 1e3) / 1e12
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        if fp8:  # e4m3 dense peak = the measured bf16 peak x the nominal 4.5 / 2.25
-            peak *= 2.0
-            tc_peak_key = "bf16_tflops_sustained x 2 (e4m3 / bf16 nominal ratio)"
-        unit = "TFLOP/s"
-    traffic = traffic_from_profiles(dom, args.workload)
-    launches = mods[0].launches_per_forward(N) * args.steps * (len(mods) if w.n_layers > 1 else 1)
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3" if fp8 else w.dtype,
-        "data": "synthetic (seeded; random-init weights of the layer's shapes)",
-        "config": {"workload": w.name, "tokens_per_gpu": N, "layers": w.n_layers,
-                   "d": w.d, "experts": w.n_experts, "top_k": w.top_k, "d_ff": w.d_ff,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": (f"weights rotate over {n_rot} copies; each step streams one copy's "
-                          "active experts, >= 0.5 GB (> 126 MB L2)"
-                          if w.n_layers == 1 else "38 distinct layers, 45.9 GB per step (> L2)"),
-                   "active_experts_per_layer": U},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
-                "d2h_bytes_per_step": nbytes},
-        "gpu_launches": launches,
+    peaks, src = load_peaks()
+    bound, work, achieved, peak, unit, key = roofline(w, dom, per_layer, U, peaks, src, clk,
+                                                      sum(block_s))
+    res = {
+        "workload": w.name, "value": value, "unit": "tokens/s", "steps": steps,
+        "repeats": args.repeats, "ms_per_step": secs / steps * 1e3,
+        "ms_per_step_blocks": [b / steps * 1e3 for b in block_s],
+        "dtype": "e4m3" if w.dtype == "fp8" else w.dtype,
+        "tokens_per_gpu": N, "layers": w.n_layers, "active_experts_per_layer": U,
+        "l2": (f"weights rotate over {n_rot} copies; each step streams one copy's active "
+               "experts, >= 0.5 GB (> 126 MB L2)" if w.n_layers == 1
+               else f"{w.n_layers} distinct layers, {w.n_layers * 1.21:.1f} GB per step (> L2)"),
+        "gpu_launches": mods[0].launches_per_forward(N) * steps * args.repeats
+                        * (len(mods) if w.n_layers > 1 else 1),
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
-                     "unit": unit, "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{src} ({'hbm_gbs' if bound == 'hbm' else tc_peak_key})",
-                     "work_per_launch": work},
+                     "unit": unit, "frac": achieved / peak,
+                     "traffic": traffic_from_profiles(dom, args_name(w)),
+                     "peak_source": f"{src} ({key})", "work_per_launch": work,
+                     "kernel_time": "mean per launch from the separate event-separated pass"},
         "kernel_ms": per_layer,
+        "kernel_ms_note": ("per launch, from a second pass of the same steps with CUDA events "
+                           "recorded between the launches (the events break the programmatic "
+                           "dependent-launch overlap, so these durations include launch gaps)"),
         "clocks": clk,
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, xs[0], layers[0], budget_s=args.cpu_budget)
+    if headline:
+        # end to end through the C ABI with host buffers (H2D + forward + D2H per step)
+        xh = xs[0].cpu().pin_memory()
+        oh = torch.empty_like(xh).pin_memory()
+        e2e_steps = max(10, min(steps * args.repeats, 500))
+        for _ in range(3):
+            mods[0].forward_host(xh, oh)
+        barrier(world)
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            if w.n_layers > 1:
+                # first block from host, the chain on device, last block back to host
+                h = xh.to(dev, non_blocking=True)
+                for l, m in enumerate(mods):
+                    dst = outs[l & 1]
+                    m.forward(h, dst, stream)
+                    h = dst
+                oh.copy_(h, non_blocking=True)
+                torch.cuda.synchronize()
+            else:
+                mods[0].forward_host(xh, oh)
+        e2e_local = time.perf_counter() - t0
+        e2e_value, _ = job_throughput(N * e2e_steps, e2e_local, world, dev)
+        nbytes = xh.numel() * xh.element_size()
+        res["e2e"] = {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+                      "d2h_bytes_per_step": nbytes}
+        if rank == 0 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w, xs[0], layers[0], budget_s=args.cpu_budget)
     for m in mods:
         m.close()
+    del mods, layers, xs, outs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def args_name(w):
+    """Short workload name (the key of W.WORKLOADS) used by the profile files."""
+    for k, v in W.WORKLOADS.items():
+        if v.name == w.name:
+            return k
+    return w.name
+
+
+def run_ours(args, w, world, rank, local):
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    head = measure(w, args, args.steps, world, rank, local, headline=True)
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "repeats": args.repeats,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": head["dtype"],
+        "data": "synthetic (seeded; random-init weights of the layer's shapes)",
+        "config": {"workload": w.name, "tokens_per_gpu": w.n_tokens, "layers": w.n_layers,
+                   "d": w.d, "experts": w.n_experts, "top_k": w.top_k, "d_ff": w.d_ff,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": head["l2"], "active_experts_per_layer": head["active_experts_per_layer"],
+                   "timing": (f"median of {args.repeats} timed blocks of exactly {args.steps} "
+                              "steps, each bracketed by barrier + synchronize")},
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "roofline": head["roofline"],
+        "kernel_ms": head["kernel_ms"],
+        "kernel_ms_note": head["kernel_ms_note"],
+        "ms_per_step_blocks": head["ms_per_step_blocks"],
+        "clocks": head["clocks"],
+    }
+    if "cpu_baseline" in head:
+        line["cpu_baseline"] = head["cpu_baseline"]
+    # the other configurations, each with its own step count, on one GPU only
+    extra = [x for x in args.extra.split(",") if x] if world == 1 else []
+    if extra:
+        line["workloads"] = {}
+        for name in extra:
+            if name == args.workload:
+                continue
+            ew = W.WORKLOADS[name]
+            r = measure(ew, args, DEFAULT_STEPS[name], world, rank, local, headline=False)
+            line["workloads"][name] = r
     return line
 
 
@@ -439,11 +498,20 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="distinct weight copies cycled through (single-layer workloads)")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed blocks of --steps steps; the median block is reported")
+    ap.add_argument("--extra", default=None,
+                    help="comma-separated further workloads measured after the headline "
+                         "one on a single GPU (default: all others for decode, none otherwise)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.steps is None:
         args.steps = DEFAULT_STEPS[args.workload]
+    if args.extra is None:
+        args.extra = EXTRA if args.workload == "decode" else ""
+    if args.repeats < 1:
+        ap.error("--repeats must be >= 1")
     w = W.WORKLOADS[args.workload]
     world, rank, local = dist_env()
     if args.impl == "reference":

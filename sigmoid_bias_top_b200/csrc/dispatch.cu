@@ -21,9 +21,11 @@
 //      rounds of 32 (__match_any_sync), the warps' counts are prefixed, and a
 //      second pass assigns positions;
 //   3. replica 0 writes perm (grouped row -> assignment t*k+j) and inv (the
-//      reverse); replica r writes the normalised rows of every replicas-th
-//      assignment, one warp per row: xp[row] = x[t] * rinv[t] * gain, the same
-//      fp32 products as the router's input, rounded once to the storage type.
+//      reverse); the replicas share out the chunk's tokens, split into column
+//      segments, one warp per (token, segment): the segment of the normalised
+//      row x[t] * rinv[t] * gain (the same fp32 products as the router's
+//      input, rounded once to the storage type) is formed once and stored at
+//      each of the token's k grouped positions.
 // The grouped rows let the gate/up GEMM load contiguous 128-row TMA boxes.
 // For FP8_BLOCK layers ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig verbraucht wie ein 2B-Modell",
 // inferencekey.com, section "Für Engineers", paragraph "Quantisierung":
@@ -197,32 +199,43 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     __syncthreads();
 
-    // 3. normalised rows, one warp per row, 16-byte vectors, 8 loads in flight
-    if constexpr (kQuant) {
-        // bf16 input; d % 128 == 0, so each half-warp's 16 vectors (128
-        // values) are one quantisation group and are all in or all out of the row
-        const int vpr = d / 8;
-        const int gpr = d / kFp8Block;
-        const uint4 *xv = static_cast<const uint4 *>(p.x);
-        constexpr int U = 4;
-        for (int i = rep + warp * p.replicas; i < na; i += kWarps * p.replicas) {
-            const int pos = pos_s[i];
-            if (pos < 0) continue;
-            const int t = (a0 + i) / k;
-            const float r = p.rinv[t];
-            const uint4 *src = xv + static_cast<size_t>(t) * vpr;
-            uint2 *dst = reinterpret_cast<uint2 *>(xq + static_cast<size_t>(pos) * d);
-            for (int v0 = 0; v0 < vpr; v0 += 32 * U) {
+    // 3. normalised rows. A token's row is the same for its k assignments, so
+    // it is normalised (and for FP8 quantised) once and stored at each of
+    // its k grouped positions. Work unit: one token x one column segment (a
+    // run of 32-vector blocks), one warp per unit; the segments split each
+    // row as far as needed to give every warp of the launch a unit.
+    const int ntc = max(0, t1 - t0);
+    const int vpr = kQuant ? d / 8 : d * p.elem_bytes / 16;  // 16-byte vectors per row
+    const int nblk = (vpr + 31) / 32;
+    const int warps_all = kWarps * p.replicas;
+    int nseg = warps_all / max(ntc, 1);
+    nseg = nseg < 1 ? 1 : nseg > nblk ? nblk : nseg;
+    const int units = ntc * nseg;
+    const uint4 *xv = static_cast<const uint4 *>(p.x);
+    for (int u0 = rep + warp * p.replicas; u0 < units; u0 += warps_all) {
+        const int tl = u0 / nseg, sg = u0 % nseg;
+        const int t = t0 + tl;
+        const int *dst = pos_s + tl * k;  // grouped positions of the token's k slots
+        const float r = p.rinv[t];
+        const uint4 *src = xv + static_cast<size_t>(t) * vpr;
+        const int v_begin = (sg * nblk / nseg) * 32;
+        const int v_end = min(vpr, ((sg + 1) * nblk / nseg) * 32);
+        if constexpr (kQuant) {
+            // bf16 input; d % 128 == 0, so each half-warp's 16 vectors (128
+            // values) are one quantisation group, all in or all out of the row
+            const int gpr = d / kFp8Block;
+            constexpr int U = 4;
+            for (int v0 = v_begin; v0 < v_end; v0 += 32 * U) {
                 uint4 raw[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int v = v0 + u * 32 + lane;
-                    raw[u] = v < vpr ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+                    raw[u] = v < v_end ? src[v] : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int v = v0 + u * 32 + lane;
-                    const bool in = v < vpr;
+                    const bool in = v < v_end;
                     const float *g = gs + (in ? v : 0) * 8;
                     const float4 g0 = *reinterpret_cast<const float4 *>(g);
                     const float4 g1 = *reinterpret_cast<const float4 *>(g + 4);
@@ -237,61 +250,58 @@ __global__ void __launch_bounds__(kThreads, 4)
                     float sc;
                     const uint2 codes = quant8(xnv, &sc);  // every lane takes part
                     if (in) {
-                        dst[v] = codes;
-                        if ((lane & 15) == 0) xs[static_cast<size_t>(pos) * gpr + v / 16] = sc;
+                        for (int j = 0; j < k; ++j) {
+                            const int pos = dst[j];
+                            if (pos < 0) continue;
+                            reinterpret_cast<uint2 *>(xq + static_cast<size_t>(pos) * d)[v] = codes;
+                            if ((lane & 15) == 0) xs[static_cast<size_t>(pos) * gpr + v / 16] = sc;
+                        }
                     }
                 }
             }
-        }
-        return;
-    }
-    const int vpr = d * p.elem_bytes / 16;  // vectors per row
-    const int epv = 16 / p.elem_bytes;      // elements per vector
-    const uint4 *xv = static_cast<const uint4 *>(p.x);
-    uint4 *xpv = static_cast<uint4 *>(p.xp);
-    constexpr int U = 8;
-    for (int i = rep + warp * p.replicas; i < na; i += kWarps * p.replicas) {
-        const int pos = pos_s[i];
-        if (pos < 0) continue;
-        const int t = (a0 + i) / k;
-        const float r = p.rinv[t];
-        const uint4 *src = xv + static_cast<size_t>(t) * vpr;
-        uint4 *dst = xpv + static_cast<size_t>(pos) * vpr;
-        for (int v0 = 0; v0 < vpr; v0 += 32 * U) {
-            uint4 raw[U];
+        } else {
+            const int epv = 16 / p.elem_bytes;  // elements per vector
+            uint4 *xpv = static_cast<uint4 *>(p.xp);
+            constexpr int U = 8;
+            for (int v0 = v_begin; v0 < v_end; v0 += 32 * U) {
+                uint4 raw[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int v = v0 + u * 32 + lane;
-                if (v < vpr) raw[u] = src[v];
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int v = v0 + u * 32 + lane;
-                if (v >= vpr) continue;
-                const float *g = gs + v * epv;
-                uint4 o;
-                if (p.elem_bytes == 2) {
-                    const float4 g0 = *reinterpret_cast<const float4 *>(g);
-                    const float4 g1 = *reinterpret_cast<const float4 *>(g + 4);
-                    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-                    uint32_t q[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                            bf16_to_f32(w[h] & 0xFFFFu) * r * gg[2 * h],
-                            bf16_to_f32(w[h] >> 16) * r * gg[2 * h + 1]);
-                        q[h] = *reinterpret_cast<uint32_t *>(&b2);
-                    }
-                    o = make_uint4(q[0], q[1], q[2], q[3]);
-                } else {
-                    const float4 g0 = *reinterpret_cast<const float4 *>(g);
-                    o = make_uint4(__float_as_uint(__uint_as_float(raw[u].x) * r * g0.x),
-                                   __float_as_uint(__uint_as_float(raw[u].y) * r * g0.y),
-                                   __float_as_uint(__uint_as_float(raw[u].z) * r * g0.z),
-                                   __float_as_uint(__uint_as_float(raw[u].w) * r * g0.w));
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < v_end) raw[u] = src[v];
                 }
-                dst[v] = o;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v >= v_end) continue;
+                    const float *g = gs + v * epv;
+                    uint4 o;
+                    if (p.elem_bytes == 2) {
+                        const float4 g0 = *reinterpret_cast<const float4 *>(g);
+                        const float4 g1 = *reinterpret_cast<const float4 *>(g + 4);
+                        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+                        uint32_t q[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                                bf16_to_f32(w[h] & 0xFFFFu) * r * gg[2 * h],
+                                bf16_to_f32(w[h] >> 16) * r * gg[2 * h + 1]);
+                            q[h] = *reinterpret_cast<uint32_t *>(&b2);
+                        }
+                        o = make_uint4(q[0], q[1], q[2], q[3]);
+                    } else {
+                        const float4 g0 = *reinterpret_cast<const float4 *>(g);
+                        o = make_uint4(__float_as_uint(__uint_as_float(raw[u].x) * r * g0.x),
+                                       __float_as_uint(__uint_as_float(raw[u].y) * r * g0.y),
+                                       __float_as_uint(__uint_as_float(raw[u].z) * r * g0.z),
+                                       __float_as_uint(__uint_as_float(raw[u].w) * r * g0.w));
+                    }
+                    for (int j = 0; j < k; ++j) {
+                        const int pos = dst[j];
+                        if (pos >= 0) xpv[static_cast<size_t>(pos) * vpr + v] = o;
+                    }
+                }
             }
         }
     }
