@@ -186,6 +186,73 @@ int moe_route_noalloc(const void *x, int dtype, const float *norm_gain, const fl
                       const float *expert_bias, int n_tokens, int d, int n_experts, int top_k,
                       float eps, float routed_scale, int32_t *idx, float *w, void *stream);
 
+/* ---------------------------------------------------------------------------
+ * Expert parallelism. The page notes that once the experts are spread over
+ * devices, dispatch, token regrouping and uneven expert loads decide the cost,
+ * and names expert parallelism as how the layer is deployed at scale
+ * ("LFM2.5-24B-A2B: Biased Routing, Short Convolutions and Ten KV Caches",
+ * section "The router has two different scores"); it gives no implementation.
+ * Here each rank (one process per GPU) routes and dispatches ITS OWN tokens
+ * over all E experts but holds the weights of one contiguous block of
+ * experts, [expert_first, expert_first + n_local). A forward is
+ *   moe_ep_dispatch -> exchange rows -> moe_ep_experts -> exchange outputs
+ *   -> moe_ep_combine,
+ * with both exchanges done by the caller (NCCL grouped send/recv or any
+ * transport) between the buffers of moe_ep_buffers:
+ *   send_rows [max_tokens*k][d]: after moe_ep_dispatch, the normalised rows
+ *     grouped by expert (ascending), token order within an expert; the rows
+ *     of expert e are rows offsets[e] .. offsets[e+1]-1, offsets being the
+ *     exclusive prefix of the counts moe_ep_dispatch returns;
+ *   recv_rows [max_recv_rows][d]: the caller places here the rows of the
+ *     local experts from every rank, grouped by local expert (ascending),
+ *     any fixed order within an expert (source rank order, say);
+ *   send_y [max_recv_rows][d]: after moe_ep_experts, the expert output of
+ *     each received row, in the same position as the row;
+ *   recv_y [max_tokens*k][d]: the caller places here each of its own rows'
+ *     outputs, in the position of the row in send_rows.
+ * Storage type of rows and outputs = the layer dtype. MOE_F32 and MOE_BF16
+ * layers only (MOE_ERR_INVALID_ARG otherwise). Buffers are context-owned
+ * device memory, valid until moe_ep_destroy. No kernel of this library reads
+ * another GPU's memory. */
+typedef struct moe_ep_ctx moe_ep_ctx;
+
+/* As moe_create, except: w->w_gate_up [n_local][2I][d] and w->w_down
+ * [n_local][d][I] hold the local experts only (router_w [E][d] and
+ * expert_bias [E] stay whole); max_recv_rows bounds the rows one rank may
+ * receive (W * max_tokens * k covers any routing). */
+int moe_ep_create(int d, int n_experts, int d_ff, int top_k, float eps, const moe_weights *w,
+                  int max_tokens, int expert_first, int n_local, int max_recv_rows,
+                  moe_ep_ctx **out);
+
+/* Route and dispatch x[n_tokens][d] (device) into send_rows; writes the
+ * per-expert row counts [E] to counts_host and waits for the stream (the
+ * exchange sizes come from them). */
+int moe_ep_dispatch(moe_ep_ctx *h, const void *x, int n_tokens, int32_t *counts_host,
+                    void *stream);
+
+/* Device addresses of the four exchange buffers (any may be NULL). */
+int moe_ep_buffers(moe_ep_ctx *h, void **send_rows, void **recv_rows, void **send_y,
+                   void **recv_y);
+
+/* Both expert contractions of the local experts over the first
+ * sum(local_counts_host) rows of recv_rows, local_counts_host[n_local] rows
+ * per local expert in order; outputs into send_y. More rows than
+ * max_recv_rows give MOE_ERR_TOO_MANY_TOKENS. Asynchronous on stream. */
+int moe_ep_experts(moe_ep_ctx *h, const int32_t *local_counts_host, void *stream);
+
+/* out[N][d] = x + sum_j w_j y_j for the last dispatched batch (N tokens),
+ * reading recv_y. x is the batch given to moe_ep_dispatch; out == x is
+ * allowed. Asynchronous on stream. */
+int moe_ep_combine(moe_ep_ctx *h, const void *x, void *out, void *stream);
+
+/* As moe_debug_routing, for the last moe_ep_dispatch (offsets over all E). */
+int moe_ep_debug_routing(moe_ep_ctx *h, int32_t *idx, float *w, int32_t *perm,
+                         int32_t *offsets, void *stream);
+
+/* As moe_status and moe_destroy. */
+int moe_ep_status(moe_ep_ctx *h);
+int moe_ep_destroy(moe_ep_ctx *h);
+
 /* Static description of a moe_err code. */
 const char *moe_strerror(int code);
 

@@ -71,6 +71,21 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc.restype = I
         L.moe_strerror.argtypes = [I]
         L.moe_strerror.restype = ctypes.c_char_p
+        # expert parallelism (ep.py)
+        L.moe_ep_create.argtypes = [I, I, I, I, F, ctypes.POINTER(MoeWeights), I, I, I, I,
+                                    ctypes.POINTER(P)]
+        L.moe_ep_dispatch.argtypes = [P, P, I, P, P]
+        L.moe_ep_buffers.argtypes = [P, ctypes.POINTER(P), ctypes.POINTER(P),
+                                     ctypes.POINTER(P), ctypes.POINTER(P)]
+        L.moe_ep_experts.argtypes = [P, P, P]
+        L.moe_ep_combine.argtypes = [P, P, P, P]
+        L.moe_ep_debug_routing.argtypes = [P, P, P, P, P, P]
+        L.moe_ep_status.argtypes = [P]
+        L.moe_ep_destroy.argtypes = [P]
+        for f in (L.moe_ep_create, L.moe_ep_dispatch, L.moe_ep_buffers, L.moe_ep_experts,
+                  L.moe_ep_combine, L.moe_ep_debug_routing, L.moe_ep_status,
+                  L.moe_ep_destroy):
+            f.restype = I
         for f in (L.moe_create, L.moe_forward, L.moe_forward_host, L.moe_destroy,
                   L.moe_status, L.moe_debug_routing, L.moe_debug_fp8_rows, L.moe_profile,
                   L.moe_kernel_times,

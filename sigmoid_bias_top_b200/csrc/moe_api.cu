@@ -78,20 +78,8 @@ struct moe_ctx {
 
 static const char *kKernelNames[] = {"route", "dispatch", "gate_up", "down", "combine"};
 static const char *kFusedKernelNames[] = {"route", "dispatch", "experts", "combine"};
-constexpr int kChunkAssign = 512;  // assignments per dispatch chunk (target)
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// Token chunks of the dispatch: about kChunkAssign assignments each, a whole
-// number of route groups (32 tokens), histogram within 64 KB of shared memory.
-static void chunk_plan(int N, int k, int max_chunks, int *nchunk, int *chunk_tokens) {
-    int n = (N * k + kChunkAssign - 1) / kChunkAssign;
-    n = n < 1 ? 1 : n > max_chunks ? max_chunks : n;
-    int ct = (N + n - 1) / n;
-    ct = (ct + 31) / 32 * 32;
-    *chunk_tokens = ct;
-    *nchunk = (N + ct - 1) / ct;
-}
 
 int moe::ensure_smem_ptr(const void *kern, size_t smem) {
     static std::mutex mu;
@@ -185,7 +173,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->route_tc = (h->use_tc || h->fp8) && route_tc_ok(d, n_experts);
 
     h->e_pad = (n_experts + 63) / 64 * 64;
-    h->max_chunks = 16384 / n_experts < 256 ? 16384 / n_experts : 256;
+    h->max_chunks = max_dispatch_chunks(n_experts);
 
     // workspace layout (every block 256-byte aligned)
     const size_t N = max_tokens, R = h->rows_cap, E = n_experts;
@@ -400,7 +388,7 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
         MOE_TRY(launch_dispatch(dp, s));
     MOE_MARK();
 
-    GroupedParams gp;
+    GroupedParams gp = {};
     gp.offsets = h->offsets; gp.mt_start = h->mt_start; gp.status = h->status;
     gp.E = h->E; gp.d = h->d; gp.I = h->I; gp.k = h->k; gp.rows_cap = h->rows_cap;
     const int max_mtiles = (N * h->k + tile_m - 1) / tile_m + h->E;

@@ -86,7 +86,20 @@ struct GroupedParams {
     int *status;
     int E, d, I, k;
     int rows_cap;             // allocated grouped rows (act, y)
+    // epilogue inputs of the dense and short-convolution blocks (CTA-pair kernel)
+    const void *resid;        // kEpiResid: [rows][d] added to the product
+    const void *aux;          // kEpiConv: a [rows][d] (bf16), convolved along each sequence
+    const float *conv;        // kEpiConv: taps [d][3] by lag
+    const float *state_in;    // kEpiConv: [rows/seq_len][2][d] a of positions -2, -1, or null
+    int seq_len;              // kEpiConv: positions per sequence (rows are sequence-major)
 };
+
+// Epilogue modes of the CTA-pair GEMM (launch_gemm_tc2_mode).
+constexpr int kEpiSiluMul = 0;  // paired rows: silu(gate) * up          (4-D weight map)
+constexpr int kEpiPlain = 1;    // plain product                          (2-D weight map)
+constexpr int kEpiMul = 2;      // paired rows: gate * up, no activation  (4-D weight map)
+constexpr int kEpiConv = 3;     // u * depthwise causal conv of a         (2-D weight map)
+constexpr int kEpiResid = 4;    // residual + product                     (2-D weight map)
 
 struct DecodeParams {
     // the fused small-batch expert kernel (gate/up and down in one launch)
@@ -142,6 +155,14 @@ int launch_selftest_timeout(int *status, int timeout_us, cudaStream_t s);
 constexpr int kTcPairTileM = 256;
 int launch_gemm_tc2_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
 int launch_gemm_tc2_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s);
+// Any epilogue mode on given maps: w = weights (4-D paired-row map for
+// kEpiSiluMul / kEpiMul, 2-D box-128 map otherwise), t = token rows (box 128).
+int launch_gemm_tc2_mode(int mode, const CUtensorMap &w, const CUtensorMap &t,
+                         const GroupedParams &p, int n_sm, cudaStream_t s);
+// 4-D paired-row view of a row-major [rows_total][d] bf16 matrix: 16-row
+// group g of the first block and the rows up_offset further (box 64x16x2x4).
+int tc_encode_pair_4d(CUtensorMap *m, const void *base, uint64_t rows_total, int d,
+                      uint64_t up_offset);
 constexpr int kDecodeRowsPerExpert = 32;  // the fused kernel is used up to this mean load
 int decode_build_maps(void **holder, const void *xp, const void *act, const void *wgu,
                       const void *wd, int rows_cap, int E, int d, int I);
@@ -168,6 +189,19 @@ inline int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, 
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess
                ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Token chunks of the dispatch: about kChunkAssign assignments each, a whole
+// number of route groups (32 tokens), histogram within 64 KB of shared memory.
+constexpr int kChunkAssign = 512;  // assignments per dispatch chunk (target)
+inline int max_dispatch_chunks(int E) { return 16384 / E < 256 ? 16384 / E : 256; }
+inline void chunk_plan(int N, int k, int max_chunks, int *nchunk, int *chunk_tokens) {
+    int n = (N * k + kChunkAssign - 1) / kChunkAssign;
+    n = n < 1 ? 1 : n > max_chunks ? max_chunks : n;
+    int ct = (N + n - 1) / n;
+    ct = (ct + 31) / 32 * 32;
+    *chunk_tokens = ct;
+    *nchunk = (N + ct - 1) / ct;
 }
 
 // Raises a kernel's dynamic shared-memory limit (once per kernel and size).

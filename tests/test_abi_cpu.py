@@ -14,14 +14,20 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_symbols():
-    src = open(os.path.join(ROOT, "include", "moe.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names.update(re.findall(r"\b(moe_[a-z_]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert "moe_create" in names and "moe_forward" in names and "moe_destroy" in names
+    for n in ("moe_create", "moe_forward", "moe_destroy", "moe_ep_create", "moe_ep_dispatch",
+              "moe_dense_create", "moe_conv_forward", "moe_block_destroy"):
+        assert n in names, n
     L = sb.lib()
     missing = [n for n in names if not hasattr(L, n)]
     assert not missing, missing
@@ -124,3 +130,37 @@ def test_calls_on_null_handle_are_rejected():
     assert L.moe_status(None) == -1
     assert L.moe_destroy(None) == 0
     assert L.moe_profile(None, 1) == -1
+
+
+def test_ep_create_validates_before_touching_the_device():
+    L = sb.lib()
+    h = ctypes.c_void_p(99)
+    w = _weights()
+
+    def create(d=2048, E=64, I=1536, k=4, first=0, n_local=8, cap=1024, ww=w):
+        return L.moe_ep_create(d, E, I, k, 1e-6, ctypes.byref(ww), 16, first, n_local, cap,
+                               ctypes.byref(h))
+    assert create(first=60, n_local=8) == -2 and not h.value    # block past E
+    assert create(n_local=0) == -2
+    assert create(cap=0) == -2
+    assert create(ww=_weights(dtype=sb.MOE_FP8_BLOCK)) == -1    # bf16 / f32 only
+    assert create(d=2000) == -2
+
+
+def test_block_create_validates_before_touching_the_device():
+    from sigmoid_bias_top_b200 import blocks as B
+    L = B.lib()
+    h = ctypes.c_void_p(99)
+    dw = B.DenseWeights(sb.MOE_BF16, 256, 256, 256)
+    assert L.moe_dense_create(2000, 6144, 1e-6, ctypes.byref(dw), 16, ctypes.byref(h)) == -2
+    assert L.moe_dense_create(2048, 6100, 1e-6, ctypes.byref(dw), 16, ctypes.byref(h)) == -2
+    assert L.moe_dense_create(2048, 6144, 1e-6, ctypes.byref(B.DenseWeights(sb.MOE_F32, 256,
+                              256, 256)), 16, ctypes.byref(h)) == -1
+    assert L.moe_dense_create(2048, 6144, 1e-6, ctypes.byref(B.DenseWeights(sb.MOE_BF16, 258,
+                              256, 256)), 16, ctypes.byref(h)) == -3
+    cw = B.ConvWeights(sb.MOE_BF16, 256, 256, 256, 256)
+    assert L.moe_conv_create(100, 1e-6, ctypes.byref(cw), 16, ctypes.byref(h)) == -2
+    assert L.moe_conv_create(2048, 1e-6, ctypes.byref(B.ConvWeights(sb.MOE_BF16, 256, 256, 0,
+                             256)), 16, ctypes.byref(h)) == -1
+    assert not h.value
+    assert L.moe_block_destroy(None) == 0 and L.moe_block_status(None) == -1
