@@ -38,9 +38,12 @@ from sigmoid_bias_top_b200 import workloads as W  # noqa: E402
 METRIC = "MoE-layer tokens/s (d2048,E64,top4,I1536) + % of HBM / bf16 TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DEFAULT_STEPS = {"decode": 2000, "prefill": 200, "skewed": 100, "stacked": 100, "tiny": 2000,
-                 "verify": 1000, "decode_fp8": 2000, "prefill_fp8": 100}
+                 "verify": 1000, "decode_fp8": 2000, "prefill_fp8": 100,
+                 "dense_prefill": 100, "dense_decode": 1000, "conv_prefill": 200,
+                 "conv_decode": 1000}
 # measured after the headline workload in a default one-GPU run
-EXTRA = "prefill,skewed,stacked,verify,decode_fp8,prefill_fp8"
+EXTRA = ("prefill,skewed,stacked,verify,decode_fp8,prefill_fp8,"
+         "dense_prefill,dense_decode,conv_prefill,conv_decode")
 ROTATE = 4  # distinct weight copies cycled through (each step reads >= 1 GB > L2)
 
 
@@ -375,9 +378,105 @@ def measure(w, args, steps, world, rank, local, headline):
     return res
 
 
+def measure_block(w, args, steps, world, rank, local):
+    """A dense or short-convolution block workload: as measure(), with the
+    weights and inputs rotated over copies so that every step's weights and
+    rows exceed L2 together."""
+    from sigmoid_bias_top_b200.blocks import ConvBlock, DenseBlock
+    dev = torch.device("cuda", local)
+    N = w.n_tokens
+    per_copy = (3 * w.d * w.d_ff if w.kind == "dense" else 4 * w.d * w.d) * 2 + 2 * N * w.d * 2
+    n_rot = max(2, -(-(3 * 126 * 2 ** 20) // per_copy))  # >= 3x L2 over the rotation
+    n_rot = min(n_rot, 8)
+    layers = [W.make_block_layer(w, dev, layer=i) for i in range(n_rot)]
+    Cls = DenseBlock if w.kind == "dense" else ConvBlock
+    mods = [Cls(l, w.eps, max_tokens=N) for l in layers]
+    xs = [W.make_block_x(w, dev, seed=w.seed + 17 * rank + i) for i in range(n_rot)]
+    outs = [torch.empty_like(xs[0]) for _ in range(2)]
+    states = ([W.make_conv_state(w, dev, seed=w.seed + i) for i in range(n_rot)]
+              if w.kind == "conv" and w.with_state else None)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        r = i % n_rot
+        if w.kind == "dense":
+            mods[r].forward(xs[r], outs[i & 1], stream=stream)
+        else:
+            st = states[r] if states else None
+            mods[r].forward(xs[r], outs[i & 1], state_in=st, state_out=st, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    for m in mods:
+        assert m.status() == 0
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.15)
+    block_s = []
+    for _ in range(args.repeats):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        block_s.append(e0.elapsed_time(e1) / 1e3)
+    clk = clocks.stop()
+    barrier(world)
+    for m in mods:
+        m.profile(True)
+    for i in range(steps):
+        step(i)
+    torch.cuda.synchronize()
+    ktimes = {}
+    for m in mods:
+        for name, ms in m.kernel_times().items():
+            ktimes.setdefault(name, []).append(ms)
+        m.profile(False)
+        assert m.status() == 0
+    value, secs = job_throughput(N * steps, statistics.median(block_s), world, dev)
+    per = {k: float(np.mean(v)) for k, v in ktimes.items()}
+    dom = max(per, key=per.get)
+    flops, nbytes = A.block_kernel_work(w.kind, dom, N, w.d, w.d_ff)
+    peaks, src = load_peaks()
+    if w.seq_len > 1:   # prefill: tensor-bound
+        sustained = "sw_power_cap" in clk.get("reasons", []) or sum(block_s) >= 1.0
+        key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+        bound, work, unit, peak = "tensor", flops, "TFLOP/s", peaks.get(key, peaks["bf16_tflops"])
+        achieved = flops / (per[dom] / 1e3) / 1e12
+    else:               # decode: weight streaming, HBM-bound
+        key = "hbm_gbs"
+        bound, work, unit, peak = "hbm", nbytes, "GB/s", peaks["hbm_gbs"]
+        achieved = nbytes / (per[dom] / 1e3) / 1e9
+    res = {
+        "workload": w.name, "value": value, "unit": "tokens/s", "steps": steps,
+        "repeats": args.repeats, "ms_per_step": secs / steps * 1e3,
+        "ms_per_step_blocks": [b / steps * 1e3 for b in block_s], "dtype": "bf16",
+        "tokens_per_gpu": N, "sequences": w.n_seqs, "seq_len": w.seq_len,
+        "l2": f"weights and inputs rotate over {n_rot} copies (>= 3x the 126 MB L2)",
+        "block_tflops": A.block_flops_per_token(w.kind, w.d, w.d_ff) * N / secs * steps / 1e12,
+        "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+                     "unit": unit, "frac": achieved / peak,
+                     "traffic": traffic_from_profiles(dom, args_name(w)),
+                     "peak_source": f"{src} ({key})", "work_per_launch": work,
+                     "kernel_time": "mean per launch from the separate event-separated pass"},
+        "kernel_ms": per, "clocks": clk,
+    }
+    for m in mods:
+        m.close()
+    del mods, layers, xs, outs, states
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
 def args_name(w):
     """Short workload name (the key of W.WORKLOADS) used by the profile files."""
-    for k, v in W.WORKLOADS.items():
+    for k, v in list(W.WORKLOADS.items()) + list(W.BLOCK_WORKLOADS.items()):
         if v.name == w.name:
             return k
     return w.name
@@ -417,8 +516,12 @@ def run_ours(args, w, world, rank, local):
         for name in extra:
             if name == args.workload:
                 continue
-            ew = W.WORKLOADS[name]
-            r = measure(ew, args, DEFAULT_STEPS[name], world, rank, local, headline=False)
+            if name in W.BLOCK_WORKLOADS:
+                r = measure_block(W.BLOCK_WORKLOADS[name], args, DEFAULT_STEPS[name], world,
+                                  rank, local)
+            else:
+                r = measure(W.WORKLOADS[name], args, DEFAULT_STEPS[name], world, rank, local,
+                            headline=False)
             line["workloads"][name] = r
     return line
 

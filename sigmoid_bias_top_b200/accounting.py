@@ -72,3 +72,36 @@ def fp8_experts_bytes(active_experts: int, n_assign: int, d: int, d_ff: int) -> 
     act = 2 * n_assign * (d_ff + 4 * (-(-d_ff // 128)))
     return (active_experts * expert_weights(d, d_ff) + fp8_scale_bytes(active_experts, d, d_ff)
             + rows_in + act + n_assign * d * 2)
+
+
+# Neighbouring steps of the block ("LFM2.5-24B-A2B: Biased Routing, Short
+# Convolutions and Ten KV Caches", sections "The exact checkpoint" and "A
+# short convolution is a local mixer, not an embedding lookup"): per launch
+# of each kernel, the tensor FLOPs (multiply-add = 2) and the bytes it must
+# move at least (weights once, its input rows read, its output rows written;
+# bf16 = 2 bytes).
+
+def block_kernel_work(kind: str, kernel: str, n: int, d: int, d_ff: int = 0):
+    """(flops, bytes) of one launch of a dense / conv block kernel over n tokens."""
+    b = 2
+    if kind == "dense":
+        I = d_ff
+        table = {
+            "norm": (0, 2 * n * d * b),
+            "gate_up": (2 * n * 2 * I * d, 2 * I * d * b + n * d * b + n * I * b),
+            "down_residual": (2 * n * d * I, d * I * b + n * I * b + 2 * n * d * b),
+        }
+    else:
+        table = {
+            "norm": (0, 2 * n * d * b),
+            "in_gv": (2 * n * 2 * d * d, 2 * d * d * b + n * d * b + n * d * b),
+            "in_u_conv": (2 * n * d * d, d * d * b + n * d * b + n * d * b + n * d * b),
+            "out_residual": (2 * n * d * d, d * d * b + n * d * b + 2 * n * d * b),
+            "state": (0, 0),
+        }
+    return table[kernel]
+
+
+def block_flops_per_token(kind: str, d: int, d_ff: int = 0) -> int:
+    """Tensor FLOPs per token of a whole dense or conv block."""
+    return 2 * 3 * d * d_ff if kind == "dense" else 2 * 4 * d * d

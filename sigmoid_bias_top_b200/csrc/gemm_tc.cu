@@ -371,19 +371,24 @@ int encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// 4-D bf16 view of the packed gate/up matrix [E*2I][d] for the CTA-pair
-// kernel: element (k, y, z, g) = row 16 g + y + z I, column k, i.e. 16-row
-// group g of the gate block (z = 0) or the up row I further (z = 1). Groups
-// run up to E*2I - I rows, so every addressed row lies inside the matrix; a
-// box of {64, 16, 2, 4} lands in shared memory as 16 gate rows, the matching
-// 16 up rows, the next 16 gate rows, ... (128 rows, 128-byte swizzle).
-int encode_gate_up_4d(CUtensorMap *m, const void *base, int E, int d, int I) {
+// 4-D bf16 view of a packed paired-row matrix [rows_total][d] for the
+// CTA-pair kernel: element (k, y, z, g) = row 16 g + y + z up_offset, column
+// k, i.e. 16-row group g of the first block (z = 0) or the row up_offset
+// further (z = 1). For the experts' gate/up matrices [E*2I][d], up_offset =
+// I (gate row f, up row f + I); for the short-convolution input projection
+// [g; u; v] = [3d][d], up_offset = 2d pairs g with v. Groups run up to
+// rows_total - up_offset rows, so every addressed row lies inside the
+// matrix; a box of {64, 16, 2, 4} lands in shared memory as 16 first-block
+// rows, the matching 16 partner rows, the next 16, ... (128 rows, 128-byte
+// swizzle).
+int encode_pair_4d(CUtensorMap *m, const void *base, uint64_t rows_total, int d,
+                   uint64_t up_offset) {
     EncodeTiledFn enc = get_encoder();
     if (!enc) return MOE_ERR_CUDA;
-    const uint64_t groups = (static_cast<uint64_t>(E) * 2 * I - I) / 16;
+    const uint64_t groups = (rows_total - up_offset) / 16;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), 16, 2, groups};
     const cuuint64_t row = static_cast<cuuint64_t>(d) * 2;
-    const cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(I), row * 16};
+    const cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(up_offset), row * 16};
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(BK), 16, 2, 4};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
@@ -409,6 +414,11 @@ int tc_encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
     return encode_2d(m, base, rows, cols, box_rows);
 }
 
+int tc_encode_pair_4d(CUtensorMap *m, const void *base, uint64_t rows_total, int d,
+                      uint64_t up_offset) {
+    return encode_pair_4d(m, base, rows_total, d, up_offset);
+}
+
 int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, const void *wd,
                   int rows_cap, int E, int d, int I) {
     int rc;
@@ -419,7 +429,9 @@ int tc_build_maps(TcMaps *m, const void *xp, const void *act, const void *wgu, c
     if ((rc = encode_2d(&m->w_down, wd, static_cast<uint64_t>(E) * d, I, BN)) != MOE_OK)
         return rc;
     if (I % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if ((rc = encode_gate_up_4d(&m->w_gate_up_4d, wgu, E, d, I)) != MOE_OK) return rc;
+    if ((rc = encode_pair_4d(&m->w_gate_up_4d, wgu, static_cast<uint64_t>(E) * 2 * I, d, I)) !=
+        MOE_OK)
+        return rc;
     if ((rc = encode_2d(&m->w_down_half, wd, static_cast<uint64_t>(E) * d, I, BN / 2)) != MOE_OK)
         return rc;
     return MOE_OK;

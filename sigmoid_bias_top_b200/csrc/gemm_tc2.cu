@@ -35,6 +35,11 @@
 // keeps up with the MMAs of the next tile.
 // All waits are bounded (1 s) and report MOE_ERR_DEVICE_TIMEOUT; the pair
 // meets at a cluster barrier before TMEM is freed.
+// The same pipeline serves the neighbouring dense and short-convolution
+// blocks (one "expert", every token) through its epilogue mode: SiLU(gate) *
+// up (kEpiSiluMul), a plain product g * v of paired rows (kEpiMul), a plain
+// store (kEpiPlain), the store plus a residual (kEpiResid), or the u stream
+// times the depthwise causal width-3 convolution of a stored a (kEpiConv).
 #include <cooperative_groups.h>
 
 #include "moe_internal.cuh"
@@ -167,10 +172,12 @@ __device__ __forceinline__ Item decode(int item, int NW, const int32_t *mts, con
 // rounded to bf16); saturates to g for large g and to -0 for large -g.
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <bool GATE_UP>
+template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_tc2_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmT, GroupedParams p) {
+    // paired-row modes stage gate/up-style interleaved weight rows (4-D map)
+    constexpr bool GATE_UP = MODE == kEpiSiluMul || MODE == kEpiMul;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -345,7 +352,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             const float got = __shfl_xor_sync(0xffffffffu, is_gate ? mine_hi : mine_lo, 16);
                             const float g = is_gate ? mine_lo : got;
                             const float u = is_gate ? got : mine_hi;
-                            if (j < lim) *dst = __float2bfloat16_rn(silu(g) * u);
+                            const float r = MODE == kEpiSiluMul ? silu(g) * u : g * u;
+                            if (j < lim) *dst = __float2bfloat16_rn(r);
                             dst += NOUT;
                         }
                     }
@@ -360,11 +368,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tmem_ld_wait();
                     if (n < NOUT) {
                         const int lim = nvalid - c0;
-                        __nv_bfloat16 *dst = c + static_cast<size_t>(it.t0 + c0) * NOUT + n;
+                        const size_t r0 = static_cast<size_t>(it.t0 + c0);
+                        __nv_bfloat16 *dst = c + r0 * NOUT + n;
+                        if constexpr (MODE == kEpiPlain) {
 #pragma unroll
-                        for (int j = 0; j < 64; ++j) {
-                            if (j < lim) *dst = __float2bfloat16_rn(__uint_as_float(v[j >> 5][j & 31]));
-                            dst += NOUT;
+                            for (int j = 0; j < 64; ++j) {
+                                if (j < lim) *dst = __float2bfloat16_rn(__uint_as_float(v[j >> 5][j & 31]));
+                                dst += NOUT;
+                            }
+                        } else if constexpr (MODE == kEpiResid) {
+                            // out = x + acc (x read and out written by this thread: in place is fine)
+                            const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(p.resid) +
+                                                      r0 * NOUT + n;
+#pragma unroll
+                            for (int j = 0; j < 64; ++j) {
+                                if (j < lim)
+                                    *dst = __float2bfloat16_rn(__bfloat162float(*xr) +
+                                                               __uint_as_float(v[j >> 5][j & 31]));
+                                dst += NOUT;
+                                xr += NOUT;
+                            }
+                        } else {  // kEpiConv: y = u * (k0 a_t + k1 a_{t-1} + k2 a_{t-2}) per sequence
+                            const __nv_bfloat16 *a = static_cast<const __nv_bfloat16 *>(p.aux);
+                            const float k0 = p.conv[n * 3], k1 = p.conv[n * 3 + 1], k2 = p.conv[n * 3 + 2];
+#pragma unroll
+                            for (int j = 0; j < 64; ++j) {
+                                if (j < lim) {
+                                    const size_t r = r0 + j;
+                                    const int b = static_cast<int>(r / p.seq_len);
+                                    const int t = static_cast<int>(r - static_cast<size_t>(b) * p.seq_len);
+                                    const float a0 = __bfloat162float(a[r * NOUT + n]);
+                                    float a1, a2;
+                                    if (t >= 1) a1 = __bfloat162float(a[(r - 1) * NOUT + n]);
+                                    else a1 = p.state_in ? p.state_in[(static_cast<size_t>(b) * 2 + 1) * NOUT + n] : 0.f;
+                                    if (t >= 2) a2 = __bfloat162float(a[(r - 2) * NOUT + n]);
+                                    else a2 = p.state_in ? p.state_in[(static_cast<size_t>(b) * 2 + t) * NOUT + n] : 0.f;
+                                    const float cv = fmaf(k2, a2, fmaf(k1, a1, k0 * a0));
+                                    *dst = __float2bfloat16_rn(__uint_as_float(v[j >> 5][j & 31]) * cv);
+                                }
+                                dst += NOUT;
+                            }
                         }
                     }
                 }
@@ -406,26 +449,37 @@ int resident_pairs(const void *kern, size_t smem, int n_sm) {
     return n < n_sm / 2 ? n : n_sm / 2;
 }
 
-template <bool GATE_UP>
+template <int MODE>
 int launch(const CUtensorMap &w, const CUtensorMap &t, const GroupedParams &p, int n_sm,
            cudaStream_t s) {
-    auto kern = grouped_tc2_kernel<GATE_UP>;
+    auto kern = grouped_tc2_kernel<MODE>;
     const size_t smem = smem_bytes(p.E);
     if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
-    static int pairs[2] = {0, 0};  // per kernel, for the device model of the process
-    if (pairs[GATE_UP] == 0)
-        pairs[GATE_UP] = resident_pairs(reinterpret_cast<const void *>(kern), smem, n_sm);
-    return launch_k(kern, dim3(2 * pairs[GATE_UP]), dim3(kThreads), smem, s, w, t, p);
+    static int pairs = 0;  // per kernel, for the device model of the process
+    if (pairs == 0) pairs = resident_pairs(reinterpret_cast<const void *>(kern), smem, n_sm);
+    return launch_k(kern, dim3(2 * pairs), dim3(kThreads), smem, s, w, t, p);
 }
 
 }  // namespace
 
 int launch_gemm_tc2_gate_up(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s) {
-    return launch<true>(m.w_gate_up_4d, m.a_gate_up, p, n_sm, s);
+    return launch<kEpiSiluMul>(m.w_gate_up_4d, m.a_gate_up, p, n_sm, s);
 }
 
 int launch_gemm_tc2_down(const TcMaps &m, const GroupedParams &p, int n_sm, cudaStream_t s) {
-    return launch<false>(m.w_down_half, m.a_down, p, n_sm, s);
+    return launch<kEpiPlain>(m.w_down_half, m.a_down, p, n_sm, s);
+}
+
+int launch_gemm_tc2_mode(int mode, const CUtensorMap &w, const CUtensorMap &t,
+                         const GroupedParams &p, int n_sm, cudaStream_t s) {
+    switch (mode) {
+        case kEpiSiluMul: return launch<kEpiSiluMul>(w, t, p, n_sm, s);
+        case kEpiPlain: return launch<kEpiPlain>(w, t, p, n_sm, s);
+        case kEpiMul: return launch<kEpiMul>(w, t, p, n_sm, s);
+        case kEpiConv: return launch<kEpiConv>(w, t, p, n_sm, s);
+        case kEpiResid: return launch<kEpiResid>(w, t, p, n_sm, s);
+        default: return MOE_ERR_INVALID_ARG;
+    }
 }
 
 }  // namespace moe

@@ -205,3 +205,86 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
     """x plus the weights of every layer of the workload."""
     layers = [make_layer(w, l, device, seed) for l in range(w.n_layers)]
     return make_x(w, device, seed), layers
+
+
+# ---------------------------------------------------------------------------
+# The neighbouring steps of the block: dense feed-forward (layers 0-1) and the
+# short-convolution mixer ("LFM2.5-24B-A2B: Biased Routing, Short
+# Convolutions and Ten KV Caches", sections "The exact checkpoint" and "A
+# short convolution is a local mixer, not an embedding lookup"). The page
+# gives the width (2048) but not the dense intermediate width; 6144 = 3 x
+# 2048 is the dense SwiGLU width the family's drafter uses at hidden 2048
+# ("LFM2.5-24B-A2B-DSpark ist live auf Hugging Face", orcarouter.ai), taken
+# here as the workload's. Tensors:
+#   dense: norm_gain [d] f32, w_gate_up [2I, d], w_down [d, I] bf16
+#   conv:  norm_gain [d] f32, w_in [3d, d] (g, u, v rows), w_out [d, d] bf16,
+#          conv [d, 3] f32 taps by lag; x [B, T, d] bf16; state [B, 2, d] f32
+
+@dataclass(frozen=True)
+class BlockWorkload:
+    name: str
+    kind: str                  # "dense" or "conv"
+    n_seqs: int                # B
+    seq_len: int               # T
+    d: int
+    d_ff: int = 0              # dense intermediate width
+    seed: int = 0
+    eps: float = 1e-6
+    x_std: float = 1.0
+    gain_jitter: float = 0.02
+    w_std: float = 0.02        # projection weights N(0, w_std^2)
+    conv_std: float = 0.5      # taps N(0, conv_std^2)
+    state_std: float = 0.8     # carried a vectors N(0, state_std^2) (decode)
+    with_state: bool = False   # decode steps continue sequences with a carried state
+
+    @property
+    def n_tokens(self) -> int:
+        return self.n_seqs * self.seq_len
+
+    def scaled(self, **kw) -> "BlockWorkload":
+        return replace(self, **kw)
+
+
+DENSE_PREFILL = BlockWorkload("dense_prefill_B4xT2048_d2048_I6144", "dense", 4, 2048, 2048, 6144,
+                              seed=21)
+DENSE_DECODE = BlockWorkload("dense_decode_B32_d2048_I6144", "dense", 32, 1, 2048, 6144, seed=22)
+CONV_PREFILL = BlockWorkload("conv_prefill_B4xT2048_d2048", "conv", 4, 2048, 2048, seed=23)
+CONV_DECODE = BlockWorkload("conv_decode_B32_d2048", "conv", 32, 1, 2048, seed=24,
+                            with_state=True)
+
+BLOCK_WORKLOADS: Dict[str, BlockWorkload] = {
+    "dense_prefill": DENSE_PREFILL, "dense_decode": DENSE_DECODE,
+    "conv_prefill": CONV_PREFILL, "conv_decode": CONV_DECODE,
+}
+
+
+def make_block_layer(w: BlockWorkload, device="cpu", layer: int = 0) -> Dict[str, torch.Tensor]:
+    g = _gen(device, 1_000_003 * (w.seed + 1) + 7919 * (layer + 1))
+    d = w.d
+    gain = torch.ones(d, device=device, dtype=torch.float32)
+    if w.gain_jitter:
+        gain = gain + _normal((d,), w.gain_jitter, g, device, torch.float32)
+    out = {"norm_gain": gain.contiguous()}
+    if w.kind == "dense":
+        out["w_gate_up"] = _normal((2 * w.d_ff, d), w.w_std, g, device, torch.bfloat16).contiguous()
+        out["w_down"] = _normal((d, w.d_ff), w.w_std, g, device, torch.bfloat16).contiguous()
+    else:
+        out["w_in"] = _normal((3 * d, d), w.w_std, g, device, torch.bfloat16).contiguous()
+        out["conv"] = _normal((d, 3), w.conv_std, g, device, torch.float32).contiguous()
+        out["w_out"] = _normal((d, d), w.w_std, g, device, torch.bfloat16).contiguous()
+    return out
+
+
+def make_block_x(w: BlockWorkload, device="cpu", seed: Optional[int] = None) -> torch.Tensor:
+    """x: [N, d] for the dense block, [B, T, d] for the conv block (bf16)."""
+    base = w.seed if seed is None else seed
+    g = _gen(device, 7 * (base + 1) + 5)
+    shape = (w.n_tokens, w.d) if w.kind == "dense" else (w.n_seqs, w.seq_len, w.d)
+    return _normal(shape, w.x_std, g, device, torch.bfloat16).contiguous()
+
+
+def make_conv_state(w: BlockWorkload, device="cpu", seed: Optional[int] = None) -> torch.Tensor:
+    """A carried state [B, 2, d] f32 (the a vectors of two earlier positions)."""
+    base = w.seed if seed is None else seed
+    g = _gen(device, 11 * (base + 1) + 1)
+    return _normal((w.n_seqs, 2, w.d), w.state_std, g, device, torch.float32).contiguous()
