@@ -1,0 +1,716 @@
+// gemm_fp8_tc2.cu -- the FP8_BLOCK expert GEMMs of large batches on CTA
+// pairs (tcgen05.mma.cta_group::2.kind::f8f6f4), weights as the 256-row MMA
+// operand and tokens as N ("swap AB"), one launch per contraction.
+//
+// The gated SiLU expert of "LFM2.5-24B-A2B: Biased Routing, Short Convolutions
+// and Ten KV Caches" (flozi.net, English page, section "The router has two
+// different scores") with the FP8_BLOCK storage of the FP8 checkpoint
+// ("LFM2.5-24B-A2B: ein 24B-Reasoning-Modell, das pro Wortstück so wenig
+// verbraucht wie ein 2B-Modell", inferencekey.com, section "Für Engineers",
+// paragraph "Quantisierung": weights FP8 in static 128x128 blocks,
+// activations FP8 dynamic per group of 128):
+//   gate/up: aq, as = Q( silu(xq . Wg) * (xq . Wu) )  per group of 128 features
+//   down:    y      = bf16( aq . Wd )
+// where every product over one 128-wide K block carries the weight block's
+// scale sw and the token group's scale sa.
+//
+// Tiles as in the bf16 pair kernel (gemm_tc2.cu): M = 256 weight rows per
+// pair, 128 per CTA. gate/up: CTA h stages the gate and up rows of features
+// f0+64h..+63 interleaved in 16-row groups (one 4-D TMA box), so its rows
+// lie in two weight row blocks (the gate block and the up block of f0) and
+// TMEM lanes l, l+16 of each quarter hold gate and up of one feature. down:
+// CTA h stages Wd rows n0+128h..+127, one weight row block. N = the tokens of
+// one token tile of an expert (equal tiles of at most 128, rounded to 16),
+// N/2 token rows per CTA.
+//
+// The scales differ per K block, so the tensor cores cannot add one K block
+// onto the next: each K block's four MMAs (K = 32) start a fresh sum in one
+// of four 128-column TMEM buffers, and the epilogue warps (8 per CTA, two per
+// TMEM lane quarter, 64 token columns each) load it and add partial * f[col]
+// into fp32 registers, f[col] = sw * sa[token][kb] taken from a shared-memory
+// table of the tile's factors (gate and up factors of four columns side by
+// side, so the two half-warps read different banks). An eleventh warp builds
+// that table one chunk of 16 K blocks ahead (two chunk buffers), issuing all
+// of a chunk's scale loads before using any, so the scale reads' latency stays
+// off the epilogue's path; 11 warps keep the 168-register budget of 10 (the
+// fullest of the four register-file quarters holds three warps). At the
+// end of a gate/up tile the two threads of a feature swap half of their
+// columns (shuffle) and each forms SiLU(gate) * up for 32 tokens; the group
+// maximum over the pair's 128 features per token is a reduce-scatter
+// butterfly over the 16 features of a half-warp, then the four lane quarters
+// through shared memory, then the two CTAs through distributed shared memory
+// (each writes its maxima into both CTAs and arrives on both CTAs' barrier);
+// s = amax / 448 and codes e4m3(a / s) (IEEE division, nearest-even,
+// saturating) go to aq and as. A down tile stores bf16 y.
+// All waits are bounded (1 s) and report MOE_ERR_DEVICE_TIMEOUT; the pair
+// meets at a cluster barrier before TMEM is freed. No load uses multicast.
+#include <cooperative_groups.h>
+#include <cuda_fp8.h>
+
+#include <new>
+
+#include "moe_fp8.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace moe {
+namespace {
+
+constexpr int WM = 128;                  // weight rows per CTA (MMA M = 256 per pair)
+constexpr int TN = kFp8PairTileM;        // most tokens per tile (MMA N)
+constexpr int BK = kFp8Block;            // K per stage: one scale block, 128 bytes per row
+constexpr int UK = 32;                   // K per tcgen05.mma kind::f8f6f4
+constexpr int STAGES = 6;
+constexpr int A_BYTES = WM * BK;         // 16 KB of weights
+constexpr int B_ROWS = TN / 2;           // token rows per CTA
+constexpr int B_BYTES = B_ROWS * BK;     // 8 KB of tokens
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NBUF = 4;                  // TMEM buffers of one K block each
+constexpr int TMEM_COLS = NBUF * TN;     // 512
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kTblWarp = 2 + kEpiWarps;  // builds the tiles' factor tables
+constexpr int kThreads = 64 + kEpiThreads + 32;
+constexpr int CW = TN / 2;               // token columns per epilogue warp
+constexpr int TBL = 16;                  // K blocks per chunk of a warp's factor table
+constexpr int kEpiBar = 1;               // named barrier of the epilogue threads
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // shared::cluster address in the pair's even CTA
+
+struct Ctl {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[NBUF];
+    uint64_t tempty[NBUF];
+    uint64_t pair_red[2];       // gate/up: both CTAs' column maxima of a tile have arrived
+    uint64_t tbl_full[2];       // a factor-table chunk is written
+    uint64_t tbl_empty[2];      // every epilogue warp is done with it
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    float red_local[4][TN];     // per lane quarter: column maxima over its 16 features
+    float red_pair[2][2][TN];   // [tile parity][CTA][column]
+    float col_scale[2][TN];     // [tile parity][column]: amax / 448
+    // two chunks of factors sw * sa: per K block of the chunk, per 4 token
+    // columns, the 4 gate (or down) factors, then the 4 up factors
+    float4 tbl[2][TBL][TN / 4][2];
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, int *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_wait(bar, parity, globaltimer_ns() + kWaitNs)) return true;
+    set_status(status, kStatusTimeout);
+    atomicExch(&ctl->abort, 1);
+    return false;
+}
+
+__device__ __forceinline__ bool aborted(Ctl *ctl) {
+    return *reinterpret_cast<volatile int *>(&ctl->abort) != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m, int x, int y,
+                                                 uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar) & kPeerBitMask)
+        : "memory");
+}
+
+// gate/up weight box {128 K bytes, 16 rows, gate|up, 4 row groups}; w = first group
+__device__ __forceinline__ void tma_load_4d_pair(void *dst, const CUtensorMap *m, int x, int w,
+                                                 uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(0), "r"(0), "r"(w),
+        "r"(smem_u32(bar) & kPeerBitMask)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+// Arrival on the barrier at the same offset in CTA `rank`. The plain form
+// orders nothing beyond this thread's TMEM reads (fenced by the caller with
+// tcgen05.fence::before_thread_sync), which is all the TMEM buffer release
+// needs; the _release form also makes this thread's earlier shared-memory
+// writes to the peer (the column maxima) visible to its acquiring waiter.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(peer_addr(bar, rank))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote_release(uint64_t *bar, uint32_t rank) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                     peer_addr(bar, rank))
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Wait on a local barrier with cluster-scope acquire (remote arrivals release).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t dl) {
+    uint32_t ok = 0, it = 0;
+    while (true) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if ((++it & 63u) == 0 && globaltimer_ns() > dl) return false;
+    }
+}
+
+__device__ __forceinline__ void epi_bar_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kEpiBar), "n"(kEpiThreads) : "memory");
+}
+
+// The epilogue threads meet and learn whether any of them passed `v`.
+__device__ __forceinline__ bool epi_bar_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "n"(kEpiBar), "n"(kEpiThreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ int find_expert(const int32_t *mts, int E, int q) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (mts[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+struct Item {
+    int e, wt, t0, rows, N;
+};
+
+// Expert-major items, the token tile fastest, so consecutive pairs share a
+// weight tile in L2; an expert's c rows in ceil(c/TN) equal tiles rounded to 16.
+__device__ __forceinline__ Item decode(int item, int NW, const int32_t *mts, const int32_t *offs,
+                                       int E) {
+    Item it;
+    it.e = find_expert(mts, E, item / NW);
+    const int ntt = mts[it.e + 1] - mts[it.e];
+    const int local = item - mts[it.e] * NW;
+    it.wt = local / ntt;
+    const int tt = local - it.wt * ntt;
+    const int c = offs[it.e + 1] - offs[it.e];
+    const int ts = ((c + ntt - 1) / ntt + 15) & ~15;
+    it.t0 = offs[it.e] + tt * ts;
+    it.rows = min(ts, c - tt * ts);
+    it.N = (it.rows + 15) & ~15;
+    return it;
+}
+
+struct PairMaps {
+    CUtensorMap w_gate_up_4d;  // e4m3 [E*2I][d] as {d, 16, 2, groups}, box 128 x 16 x 2 x 4
+    CUtensorMap w_down;        // e4m3 [E*d][I], box 128 x 128
+    CUtensorMap xq;            // e4m3 [rows][d], box 128 x 64
+    CUtensorMap aq;            // e4m3 [rows][I], box 128 x 64
+};
+
+template <bool GATE_UP>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    fp8_pair_kernel(const __grid_constant__ PairMaps maps, Fp8PairParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + STAGES * STAGE_BYTES);
+    int32_t *mts = reinterpret_cast<int32_t *>(ctl + 1);  // [E+1]
+    int32_t *offs = mts + (p.E + 1);                        // [E+1]
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int half = static_cast<int>(cluster.block_rank());
+    const bool leader = half == 0;
+    const int pair = blockIdx.x / 2, npairs = gridDim.x / 2;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], 2 * kEpiWarps);  // one per epilogue warp of both CTAs
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->pair_red[b], 2 * TN);  // TN local + TN remote
+            mbar_init(&ctl->tbl_full[b], 1);
+            mbar_init(&ctl->tbl_empty[b], kEpiWarps);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&ctl->tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(GATE_UP ? &maps.w_gate_up_4d : &maps.w_down);
+        tma_prefetch_desc(GATE_UP ? &maps.xq : &maps.aq);
+    }
+    pdl_trigger();
+    pdl_wait();
+    for (int i = threadIdx.x; i <= E; i += kThreads) {
+        mts[i] = p.mt_start[i];
+        offs[i] = p.offsets[i];
+    }
+    tc_fence_before();
+    cluster.sync();  // barriers initialised and TMEM allocated in both CTAs
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+
+    // weight tiles per expert: 128 features (gate/up) or 256 output rows (down;
+    // with d % 256 == 128 the second CTA of an expert's last tile has no rows)
+    const int NW = GATE_UP ? p.I / 128 : (p.d + 2 * WM - 1) / (2 * WM);
+    const int K = GATE_UP ? p.d : p.I;
+    const int nk = K / BK;
+    const int total = mts[E] * NW;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs) ----------------
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_parity[STAGES];
+            bool issued[STAGES];
+            for (int i = 0; i < STAGES; ++i) issued[i] = false;
+            const CUtensorMap *tm = GATE_UP ? &maps.xq : &maps.aq;
+            for (int item = pair; item < total && !aborted(ctl); item += npairs) {
+                const Item it = decode(item, NW, mts, offs, E);
+                const int trow = it.t0 + half * (it.N / 2);
+                const int wc = GATE_UP ? (it.e * 2 * p.I + it.wt * 128 + half * 64) / 16
+                                       : it.e * p.d + it.wt * 2 * WM + half * WM;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) { ok = false; break; }
+                    uint8_t *sa = smem + s * STAGE_BYTES;
+                    uint8_t *sb = sa + A_BYTES;
+                    if (leader) mbar_arrive_expect_tx(&ctl->full[s], 2 * STAGE_BYTES);
+                    if (GATE_UP)
+                        tma_load_4d_pair(sa, &maps.w_gate_up_4d, kb * BK, wc, &ctl->full[s]);
+                    else
+                        tma_load_2d_pair(sa, &maps.w_down, kb * BK, wc, &ctl->full[s]);
+                    tma_load_2d_pair(sb, tm, kb * BK, trow, &ctl->full[s]);
+                    issued[s] = true;
+                    issued_parity[s] = ph;
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            if (aborted(ctl) && leader) {  // the pair's copies complete on the leader's barriers
+                const uint64_t dl = globaltimer_ns() + kWaitNs;
+                for (int i = 0; i < STAGES; ++i)
+                    if (issued[i]) mbar_wait(&ctl->full[i], issued_parity[i], dl);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------- MMA issuer (leader only) ----------------
+            int s = 0;
+            uint32_t ph = 0, nblk = 0;
+            bool any = false;
+            for (int item = pair; item < total && !aborted(ctl); item += npairs) {
+                const Item it = decode(item, NW, mts, offs, E);
+                const uint32_t idesc = idesc_e4m3_f32(2 * WM, it.N);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    const int buf = static_cast<int>(nblk % NBUF);
+                    const uint32_t use = nblk / NBUF;
+                    if (!wait_bar(&ctl->tempty[buf], (use & 1u) ^ 1u, ctl, p.status)) { ok = false; break; }
+                    if (!wait_bar(&ctl->full[s], ph, ctl, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * TN);
+                    const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / UK; ++kk)  // a fresh sum per K block
+                        umma_e4m3_pair(d_tmem, sw128_kmajor_desc(a0 + kk * UK),
+                                       sw128_kmajor_desc(b0 + kk * UK), idesc, kk != 0 ? 1u : 0u);
+                    any = true;
+                    umma_commit_pair(&ctl->empty[s]);
+                    umma_commit_pair(&ctl->tfull[buf]);
+                    ++nblk;
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            if (any) {
+                asm volatile(
+                    "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                        smem_u32(&ctl->drain))
+                    : "memory");
+                mbar_wait(&ctl->drain, 0, globaltimer_ns() + kWaitNs);
+            }
+        }
+    } else if (warp == kTblWarp) {
+        // ---------------- factor tables (warp 10, both CTAs) ----------------
+        // per chunk of TBL K blocks of every tile: f = sw[kb] * sa[token][kb]
+        // for the tile's TN token columns; lane l takes columns 4l..4l+3,
+        // and lane j (j < 16) loads the gate (or down) weight block scale of
+        // K block kb0+j, lane 16+j the up one. All loads of a chunk are
+        // issued before any is used.
+        const float *sa_all = GATE_UP ? p.xs : p.as_in;
+        const int ng = K / BK;
+        uint32_t nchunk = 0;
+        for (int item = pair; item < total && !aborted(ctl); item += npairs) {
+            const Item it = decode(item, NW, mts, offs, E);
+            const bool rows_ok = GATE_UP || it.wt * 2 + half < p.d / 128;
+            const float *swg, *swu;
+            if (GATE_UP) {
+                const size_t rbg = static_cast<size_t>(it.e) * (2 * p.I / 128) + it.wt;
+                swg = p.sgu + rbg * ng;
+                swu = p.sgu + (rbg + p.I / 128) * ng;
+            } else {
+                swg = p.sdn + (static_cast<size_t>(it.e) * (p.d / 128) + (rows_ok ? it.wt * 2 + half : 0)) * ng;
+                swu = swg;
+            }
+            bool ok = true;
+            for (int kb0 = 0; kb0 < nk; kb0 += TBL, ++nchunk) {
+                const int slot = static_cast<int>(nchunk & 1u);
+                const bool got = wait_bar(&ctl->tbl_empty[slot], ((nchunk >> 1) & 1u) ^ 1u, ctl, p.status);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                const int n = min(TBL, nk - kb0);
+                const int jj = lane & 15;
+                const float wsc = jj < n ? __ldg((lane < 16 ? swg : swu) + kb0 + jj) : 0.f;
+                float sa[4][TBL];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int col = 4 * lane + c;
+                    const bool valid = rows_ok && col < it.rows;
+                    const float *sa_row = sa_all + static_cast<size_t>(it.t0 + (valid ? col : 0)) * ng + kb0;
+#pragma unroll
+                    for (int j = 0; j < TBL; ++j) sa[c][j] = (valid && j < n) ? __ldg(sa_row + j) : 0.f;
+                }
+                float4 (*t)[TN / 4][2] = ctl->tbl[slot];
+#pragma unroll
+                for (int j = 0; j < TBL; ++j) {
+                    const float wg = __shfl_sync(0xffffffffu, wsc, j);
+                    const float wu = GATE_UP ? __shfl_sync(0xffffffffu, wsc, 16 + j) : wg;
+                    t[j][lane][0] = make_float4(sa[0][j] * wg, sa[1][j] * wg, sa[2][j] * wg, sa[3][j] * wg);
+                    t[j][lane][1] = make_float4(sa[0][j] * wu, sa[1][j] * wu, sa[2][j] * wu, sa[3][j] * wu);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->tbl_full[slot]);
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ---------------- epilogue (warps 2..9, both CTAs) ----------------
+        const int ew = warp - 2;
+        const int q = warp & 3;          // TMEM lane quarter
+        const int ch = ew >> 2;          // token columns ch*CW .. +CW-1
+        const bool is_up = GATE_UP && lane >= 16;
+        const int role = is_up ? 1 : 0;
+        const float4 (*tbl)[TN / 4][2] = ctl->tbl[0];
+        // The gate/up epilogue threads meet at named barriers inside every
+        // tile, so they leave the tile loop together: the abort flag is
+        // agreed on at the start of a tile, and a wait that times out inside
+        // a tile skips the rest of its work but not its meeting points.
+        uint32_t nblk = 0, ntile = 0, nchunk = 0;
+        for (int item = pair; item < total; item += npairs, ++ntile) {
+            if constexpr (GATE_UP) {
+                if (epi_bar_or(aborted(ctl))) break;
+            } else {
+                if (aborted(ctl)) break;
+            }
+            const Item it = decode(item, NW, mts, offs, E);
+            // this CTA's weight rows exist (always for gate/up; for down, row
+            // block 2 wt + half must lie inside the expert's d rows)
+            const bool rows_ok = GATE_UP || it.wt * 2 + half < p.d / 128;
+            const bool has_cols = ch * CW < it.N;
+            float acc[CW];
+#pragma unroll
+            for (int j = 0; j < CW; ++j) acc[j] = 0.f;
+            const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                    static_cast<uint32_t>(ch * CW);
+            bool ok = true;
+            for (int kb = 0; kb < nk && ok; ++kb) {
+                if (kb % TBL == 0) {  // the next chunk of factors
+                    const int slot = static_cast<int>(nchunk & 1u);
+                    const bool got = wait_bar(&ctl->tbl_full[slot], (nchunk >> 1) & 1u, ctl, p.status);
+                    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                    tbl = ctl->tbl[slot];
+                }
+                const int buf = static_cast<int>(nblk % NBUF);
+                // the whole warp goes on or stops together (the TMEM loads are warp-wide)
+                const bool got = wait_bar(&ctl->tfull[buf], (nblk / NBUF) & 1u, ctl, p.status);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t v[2][32];
+                if (has_cols) {
+                    tmem_ld_32x32b_x32(t_lane + buf * TN, v[0]);
+                    tmem_ld_32x32b_x32(t_lane + buf * TN + 32, v[1]);
+                    tmem_ld_wait();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(&ctl->tempty[buf], 0);  // the leader's barrier
+                ++nblk;
+                if (has_cols) {
+                    const float4 (*row)[2] = tbl[kb % TBL] + ch * (CW / 4);
+#pragma unroll
+                    for (int j4 = 0; j4 < CW / 4; ++j4) {
+                        const float4 f = row[j4][role];
+                        acc[4 * j4 + 0] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 0) & 31]), f.x, acc[4 * j4 + 0]);
+                        acc[4 * j4 + 1] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 1) & 31]), f.y, acc[4 * j4 + 1]);
+                        acc[4 * j4 + 2] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 2) & 31]), f.z, acc[4 * j4 + 2]);
+                        acc[4 * j4 + 3] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 3) & 31]), f.w, acc[4 * j4 + 3]);
+                    }
+                }
+                if (kb % TBL == TBL - 1 || kb == nk - 1) {  // done with this chunk of factors
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->tbl_empty[static_cast<int>(nchunk & 1u)]);
+                    ++nchunk;
+                }
+            }
+            if constexpr (!GATE_UP) {
+                if (!ok) break;
+                if (has_cols && rows_ok) {
+                    const int n = it.wt * 2 * WM + half * WM + q * 32 + lane;
+                    const int lim = it.rows - ch * CW;
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) +
+                                         static_cast<size_t>(it.t0 + ch * CW) * p.d + n;
+#pragma unroll
+                    for (int j = 0; j < CW; ++j) {
+                        if (j < lim) *dst = __float2bfloat16_rn(acc[j]);
+                        dst += p.d;
+                    }
+                }
+            } else {
+            // gate/up: the gate thread (lane < 16) finishes columns 0..31 of
+            // the warp's 64, the up thread (lane + 16) columns 32..63
+            float a[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float lo = acc[j], hi = acc[32 + j];
+                const float got = __shfl_xor_sync(0xffffffffu, is_up ? lo : hi, 16);
+                const float g = is_up ? got : lo;
+                const float u = is_up ? hi : got;
+                a[j] = __fdividef(g, 1.0f + __expf(-g)) * u;
+            }
+            // column maxima over the 16 features of the half-warp: a
+            // reduce-scatter butterfly leaves lane l with columns 2(l&15), +1
+            // of its 32 (non-negative floats order like their bit patterns)
+            float m[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) m[j] = fabsf(a[j]);
+#pragma unroll
+            for (int dist = 8, n = 32; dist >= 1; dist >>= 1, n >>= 1) {
+                const bool upper = (lane & dist) != 0;
+#pragma unroll
+                for (int i = 0; i < n / 2; ++i) {
+                    const float give = upper ? m[i] : m[i + n / 2];
+                    const float keep = upper ? m[i + n / 2] : m[i];
+                    m[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, dist));
+                }
+            }
+            const int cbase = ch * CW + (is_up ? 32 : 0);  // tile column of a[0]
+            const int cl = cbase + 2 * (lane & 15);
+            ctl->red_local[q][cl] = m[0];
+            ctl->red_local[q][cl + 1] = m[1];
+            epi_bar_sync();
+            const int par = static_cast<int>(ntile & 1u);
+            const int et = threadIdx.x - 64;  // epilogue thread 0..255
+            if (et < TN) {
+                const float cm = fmaxf(fmaxf(ctl->red_local[0][et], ctl->red_local[1][et]),
+                                       fmaxf(ctl->red_local[2][et], ctl->red_local[3][et]));
+                float *slot = &ctl->red_pair[par][half][et];
+                *slot = cm;
+                st_cluster_f32(peer_addr(slot, half ^ 1), cm);
+                mbar_arrive(&ctl->pair_red[par]);
+                mbar_arrive_remote_release(&ctl->pair_red[par], half ^ 1);
+            }
+            if (!mbar_wait_cluster(&ctl->pair_red[par], (ntile >> 1) & 1u,
+                                   globaltimer_ns() + kWaitNs)) {
+                set_status(p.status, kStatusTimeout);
+                atomicExch(&ctl->abort, 1);
+                ok = false;
+            }
+            const int ngo = p.I / kFp8Block;  // output groups per row
+            if (et < TN) {
+                const float amax = fmaxf(ctl->red_pair[par][0][et], ctl->red_pair[par][1][et]);
+                const float sc = __fdiv_rn(amax, 448.f);
+                ctl->col_scale[par][et] = sc;
+                if (half == 0 && et < it.rows)
+                    p.as_out[static_cast<size_t>(it.t0 + et) * ngo + it.wt] = sc;
+            }
+            epi_bar_sync();
+            if (has_cols && ok) {
+                const int f = it.wt * 128 + half * 64 + q * 16 + (lane & 15);
+                const int lim = it.rows - cbase;
+                uint8_t *dst = p.aq + static_cast<size_t>(it.t0 + cbase) * p.I + f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    if (j < lim) {
+                        const float sc = ctl->col_scale[par][cbase + j];
+                        *dst = sc > 0.f ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(
+                                              __fdiv_rn(a[j], sc), __NV_SATFINITE, __NV_E4M3))
+                                        : static_cast<uint8_t>(0);
+                    }
+                    dst += p.I;
+                }
+            }
+            }  // gate/up tile end
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster.sync();  // the leader's MMAs into this CTA's TMEM and the peer's DSMEM writes are done
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+size_t smem_bytes(int E) {
+    return 1024 + STAGES * STAGE_BYTES + sizeof(Ctl) + 2 * (E + 1) * sizeof(int32_t);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(fn);
+}
+
+// byte matrix [rows][cols], box 128 bytes x box_rows, 128-byte swizzle, zero fill
+int encode_u8_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encoder();
+    if (!enc) return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+               ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// 4-D byte view of the packed gate/up codes [E*2I][d]: element (k, y, z, g) =
+// row 16 g + y + z I, column k (gate row f, up row f + I); a {128, 16, 2, 4}
+// box lands as 16 gate rows, the matching 16 up rows, ... (128 rows).
+int encode_u8_gate_up_4d(CUtensorMap *m, const void *base, int E, int d, int I) {
+    EncodeTiledFn enc = encoder();
+    if (!enc) return MOE_ERR_CUDA;
+    const uint64_t groups = (static_cast<uint64_t>(E) * 2 * I - I) / 16;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), 16, 2, groups};
+    const cuuint64_t row = static_cast<cuuint64_t>(d);
+    const cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(I), row * 16};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(BK), 16, 2, 4};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+               ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int resident_pairs(const void *kern, size_t smem, int n_sm) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_sm / 2 * 2);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = n_sm / 2;
+    }
+    return n < n_sm / 2 ? n : n_sm / 2;
+}
+
+template <bool GATE_UP>
+int launch(const PairMaps &m, const Fp8PairParams &p, int n_sm, cudaStream_t s) {
+    auto kern = fp8_pair_kernel<GATE_UP>;
+    const size_t smem = smem_bytes(p.E);
+    if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
+    static int pairs = 0;  // per kernel, for the device model of the process
+    if (pairs == 0) pairs = resident_pairs(reinterpret_cast<const void *>(kern), smem, n_sm);
+    return launch_k(kern, dim3(2 * pairs), dim3(kThreads), smem, s, m, p);
+}
+
+}  // namespace
+
+struct Fp8PairMapsHolder {
+    PairMaps m;
+};
+
+int fp8_pair_build_maps(void **holder, const void *xq, const void *aq, const void *wgu,
+                        const void *wd, int rows_cap, int E, int d, int I) {
+    Fp8PairMapsHolder *h = new (std::nothrow) Fp8PairMapsHolder;
+    if (!h) return MOE_ERR_OOM;
+    int rc;
+    if ((rc = encode_u8_gate_up_4d(&h->m.w_gate_up_4d, wgu, E, d, I)) != MOE_OK ||
+        (rc = encode_u8_2d(&h->m.w_down, wd, static_cast<uint64_t>(E) * d, I, WM)) != MOE_OK ||
+        (rc = encode_u8_2d(&h->m.xq, xq, rows_cap, d, B_ROWS)) != MOE_OK ||
+        (rc = encode_u8_2d(&h->m.aq, aq, rows_cap, I, B_ROWS)) != MOE_OK) {
+        delete h;
+        return rc;
+    }
+    *holder = h;
+    return MOE_OK;
+}
+
+void fp8_pair_free_maps(void *holder) { delete static_cast<Fp8PairMapsHolder *>(holder); }
+
+int launch_fp8_pair_gate_up(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s) {
+    return launch<true>(static_cast<const Fp8PairMapsHolder *>(holder)->m, p, n_sm, s);
+}
+
+int launch_fp8_pair_down(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s) {
+    return launch<false>(static_cast<const Fp8PairMapsHolder *>(holder)->m, p, n_sm, s);
+}
+
+}  // namespace moe

@@ -44,6 +44,8 @@ struct moe_ctx {
     // FP8_BLOCK layers: e4m3 rows and group scales (carved from xp and act)
     bool fp8;
     void *fp8_maps;
+    void *fp8_pair_maps; // the CTA-pair FP8 GEMMs of large batches
+    int fp8_pair_mode;   // -1 above the small-batch load, 0 never, 1 whenever not small
     uint8_t *xq, *aq;
     float *xs, *as;
 
@@ -88,9 +90,14 @@ int moe::ensure_smem_ptr(const void *kern, size_t smem) {
     std::lock_guard<std::mutex> lock(mu);
     size_t &cur = set[kern];
     if (smem <= cur) return MOE_OK;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    const cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem));
+    if (err != cudaSuccess) {
+        if (getenv("MOE_DEBUG"))
+            fprintf(stderr, "moe: shared memory of %zu bytes refused: %s\n", smem,
+                    cudaGetErrorString(err));
         return MOE_ERR_CUDA;
+    }
     cur = smem;
     return MOE_OK;
 }
@@ -169,6 +176,10 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         // MOE_ROUTE_TC=0 / 1 likewise for the tensor-core and the SIMT routers
         e = getenv("MOE_ROUTE_TC");
         h->route_tc_mode = (e && e[0] == '0') ? 0 : (e && e[0] == '1') ? 1 : -1;
+        // MOE_FP8_PAIR=0 keeps FP8_BLOCK batches of every size on the persistent
+        // kernel instead of the CTA-pair GEMMs (both compute the same result)
+        e = getenv("MOE_FP8_PAIR");
+        h->fp8_pair_mode = (e && e[0] == '0') ? 0 : -1;
     }
     h->route_tc = (h->use_tc || h->fp8) && route_tc_ok(d, n_experts);
 
@@ -265,11 +276,15 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     if (h->fp8) {
         rc = fp8_build_maps(&h->fp8_maps, h->xq, h->aq, w->w_gate_up, w->w_down, h->rows_cap,
                             n_experts, d, d_ff);
+        if (rc == MOE_OK)
+            rc = fp8_pair_build_maps(&h->fp8_pair_maps, h->xq, h->aq, w->w_gate_up, w->w_down,
+                                     h->rows_cap, n_experts, d, d_ff);
         if (rc == MOE_OK && h->route_tc)
             rc = tc_encode_2d(&h->w3_map, h->router_w3, 3 * static_cast<uint64_t>(n_experts), d,
                               3 * n_experts);
         if (rc != MOE_OK) {
             if (h->fp8_maps) fp8_free_maps(h->fp8_maps);
+            if (h->fp8_pair_maps) fp8_pair_free_maps(h->fp8_pair_maps);
             cudaFree(h->ws);
             delete h;
             return rc;
@@ -283,10 +298,20 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
 // launch) serves bf16 layers while the mean load stays at or below
 // kDecodeRowsPerExpert grouped rows per expert; larger batches use the two
 // row-tiled grouped GEMMs.
+static bool small_batch(const moe_ctx *h, int N) {
+    return static_cast<long long>(N) * h->k <= static_cast<long long>(kDecodeRowsPerExpert) * h->E;
+}
+
+// FP8_BLOCK layers above the small-batch load run the two CTA-pair FP8 GEMMs
+// (token tiles up to 128, K blocks promoted per tile); below it, and with
+// MOE_FP8_PAIR=0, the persistent FP8 kernel takes both contractions.
+static bool use_fp8_pair(const moe_ctx *h, int N) {
+    return h->fp8 && h->fp8_pair_mode != 0 && !small_batch(h, N);
+}
+
 static bool use_fused_experts(const moe_ctx *h, int N) {
-    if (h->fp8) return true;
-    return h->use_tc && static_cast<long long>(N) * h->k <=
-                            static_cast<long long>(kDecodeRowsPerExpert) * h->E;
+    if (h->fp8) return !use_fp8_pair(h, N);
+    return h->use_tc && small_batch(h, N);
 }
 
 // The tensor-core router (bf16 batches) from kRouteTcMinTokens tokens on; the
@@ -353,8 +378,10 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     int nchunk = 1, chunk_tokens = N;
     chunk_plan(N, h->k, h->max_chunks, &nchunk, &chunk_tokens);
     const bool fused = use_fused_experts(h, N);
+    const bool fp8_pair = use_fp8_pair(h, N);
     const bool pair = !fused && use_pair_gemms(h);
-    const int tile_m = !h->use_tc ? kSimtTileM : pair ? kTcPairTileM : kTcTileM;
+    const int tile_m = fp8_pair ? kFp8PairTileM
+                       : !h->use_tc ? kSimtTileM : pair ? kTcPairTileM : kTcTileM;
 
     MOE_MARK();
     RouteParams rp;
@@ -393,7 +420,17 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     gp.E = h->E; gp.d = h->d; gp.I = h->I; gp.k = h->k; gp.rows_cap = h->rows_cap;
     const int max_mtiles = (N * h->k + tile_m - 1) / tile_m + h->E;
 
-    if (h->fp8) {
+    if (fp8_pair) {
+        Fp8PairParams fp;
+        fp.offsets = h->offsets; fp.mt_start = h->mt_start;
+        fp.sgu = h->w.w_gate_up_scale; fp.sdn = h->w.w_down_scale;
+        fp.xs = h->xs; fp.as_in = h->as; fp.aq = h->aq; fp.as_out = h->as; fp.y = h->y;
+        fp.status = h->status; fp.E = h->E; fp.d = h->d; fp.I = h->I;
+        MOE_TRY(launch_fp8_pair_gate_up(h->fp8_pair_maps, fp, h->n_sm, s));
+        MOE_MARK();
+        MOE_TRY(launch_fp8_pair_down(h->fp8_pair_maps, fp, h->n_sm, s));
+        MOE_MARK();
+    } else if (h->fp8) {
         Fp8ExpertParams fp;
         fp.offsets = h->offsets; fp.sgu = h->w.w_gate_up_scale; fp.sdn = h->w.w_down_scale;
         fp.xs = h->xs; fp.aq = h->aq; fp.as = h->as; fp.y = h->y; fp.sched = h->sched;
@@ -488,6 +525,7 @@ extern "C" int moe_destroy(moe_ctx *h) {
     free_ring(h);
     if (h->decode_maps) decode_free_maps(h->decode_maps);
     if (h->fp8_maps) fp8_free_maps(h->fp8_maps);
+    if (h->fp8_pair_maps) fp8_pair_free_maps(h->fp8_pair_maps);
     if (cudaFree(h->ws) != cudaSuccess) rc = MOE_ERR_CUDA;
     delete h;
     return rc;

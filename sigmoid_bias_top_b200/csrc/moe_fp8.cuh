@@ -32,6 +32,29 @@ struct Fp8ExpertParams {
     int E, d, I;
 };
 
+// The large-batch path: two launches of the CTA-pair FP8 GEMM (gemm_fp8_tc2.cu)
+// over token tiles of at most kFp8PairTileM rows (the dispatch's row-tile
+// prefix mt_start must be built with that tile size).
+constexpr int kFp8PairTileM = 128;
+struct Fp8PairParams {
+    const int32_t *offsets;   // [E+1] row range of each expert in the grouped order
+    const int32_t *mt_start;  // [E+1] prefix of per-expert token tiles of kFp8PairTileM rows
+    const float *sgu;         // [E][2I/128][d/128] block scales of w_gate_up
+    const float *sdn;         // [E][d/128][I/128] block scales of w_down
+    const float *xs;          // gate/up input: [rows][d/128] group scales of the grouped rows
+    const float *as_in;       // down input: [rows][I/128] group scales of aq
+    uint8_t *aq;              // gate/up output: [rows][I] e4m3 codes of SiLU(gate)*up
+    float *as_out;            // gate/up output: [rows][I/128] their group scales
+    void *y;                  // down output: [rows][d] bf16
+    int *status;
+    int E, d, I;
+};
+int fp8_pair_build_maps(void **holder, const void *xq, const void *aq, const void *wgu,
+                        const void *wd, int rows_cap, int E, int d, int I);
+void fp8_pair_free_maps(void *holder);
+int launch_fp8_pair_gate_up(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s);
+int launch_fp8_pair_down(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s);
+
 // Grouped, quantised rows from the dispatch: codes [rows][d], scales [rows][d/128].
 int launch_dispatch_fp8(const DispatchParams &p, uint8_t *xq, float *xs, cudaStream_t s);
 

@@ -474,3 +474,59 @@ def test_fp8_deterministic_and_in_place():
     torch.cuda.synchronize()
     assert m.status() == 0
     assert torch.equal(a, b) and torch.equal(a, xi)
+
+
+def _fp8_layer_pair(w, layer, pair_mode):
+    """A context over the layer with the CTA-pair FP8 GEMMs on (default) or
+    off (MOE_FP8_PAIR=0: the persistent FP8 kernel for every batch)."""
+    import os
+    old = os.environ.pop("MOE_FP8_PAIR", None)
+    try:
+        if pair_mode == 0:
+            os.environ["MOE_FP8_PAIR"] = "0"
+        return MoeLayer(layer, w.top_k, w.eps, w.routed_scale, max_tokens=w.n_tokens)
+    finally:
+        os.environ.pop("MOE_FP8_PAIR", None)
+        if old is not None:
+            os.environ["MOE_FP8_PAIR"] = old
+
+
+@pytest.mark.parametrize("shape", [dict(n_experts=16, top_k=4, d=384, d_ff=640, n_tokens=700),
+                                   dict(n_experts=64, top_k=4, d=2048, d_ff=1536, n_tokens=2048)])
+def test_fp8_pair_and_persistent_kernels_agree(shape):
+    """Large FP8_BLOCK batches through the CTA-pair GEMMs and through the
+    persistent kernel: the same e4m3 products, per-K-block promotion with the
+    same factors, the same SiLU and quantisation, so the outputs agree to the
+    bf16 rounding of y and out (measured: most rows bit-identical)."""
+    w = fp8_small(**shape)
+    layer = W.make_layer(w, 0, DEV)
+    x = W.make_x(w, DEV)
+    a = _fp8_layer_pair(w, layer, -1)
+    b = _fp8_layer_pair(w, layer, 0)
+    assert a.launches_per_forward(w.n_tokens) == 5 and b.launches_per_forward(w.n_tokens) == 4
+    oa, ob = a(x), b(x)
+    torch.cuda.synchronize()
+    assert a.status() == 0 and b.status() == 0
+    ra, rb = a.debug_routing(w.n_tokens), b.debug_routing(w.n_tokens)
+    assert torch.equal(ra["idx"], rb["idx"]) and torch.equal(ra["perm"], rb["perm"])
+    da, db = (oa.double() - x.double()), (ob.double() - x.double())
+    rel = (da - db).norm(dim=1) / da.norm(dim=1).clamp_min(1e-30)
+    assert rel.max().item() <= 2e-2, rel.max().item()
+    a.close()
+    b.close()
+
+
+def test_fp8_large_batch_deterministic_and_in_place():
+    w = W.DECODE_FP8.scaled(n_tokens=1500)
+    layer = W.make_layer(w, 0, DEV)
+    x = W.make_x(w, DEV)
+    m = MoeLayer(layer, w.top_k, w.eps, max_tokens=w.n_tokens)
+    assert m.launches_per_forward(w.n_tokens) == 5
+    a = m(x)
+    b = m(x)
+    xi = x.clone()
+    m(xi, out=xi)
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    assert torch.equal(a, b) and torch.equal(a, xi)
+    m.close()
