@@ -323,6 +323,9 @@ extern "C" int moe_dense_forward(moe_block_ctx *h, const void *x, void *out, int
     gp = group_params(h, false, h->d, h->I);
     gp.c = out;
     gp.resid = x;
+    // the act rows (N x I) outweigh W_down (d x I) as soon as N > d: then
+    // each token tile is read once while the weight tiles stay in L2
+    gp.wt_fastest = n_tokens > h->d;
     BLOCK_TRY(launch_gemm_tc2_mode(kEpiResid, h->m_w2, h->m_mid, gp, h->n_sm, s));
     BLOCK_MARK();
     return MOE_OK;

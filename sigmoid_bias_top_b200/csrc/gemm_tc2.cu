@@ -147,19 +147,29 @@ __device__ __forceinline__ int find_expert(const int32_t *mts, int E, int q) {
 }
 
 // Work item: expert e, weight tile wt, token tile of `rows` tokens from
-// grouped row t0, computed with N = rows rounded up to 16.
+// grouped row t0, computed with N = rows rounded up to 16. Items run expert
+// by expert; within an expert the token tile varies fastest (the expert's
+// weight tile is read from L2 by consecutive pairs), or with wt_fastest the
+// weight tile does (for one large group whose token rows outgrow L2: each
+// token tile is then read once while the weights stay in L2).
 struct Item {
     int e, wt, t0, rows, N;
 };
 
 __device__ __forceinline__ Item decode(int item, int NW, const int32_t *mts, const int32_t *offs,
-                                       int E) {
+                                       int E, bool wt_fastest) {
     Item it;
     it.e = find_expert(mts, E, item / NW);
     const int ntt = mts[it.e + 1] - mts[it.e];
     const int local = item - mts[it.e] * NW;
-    it.wt = local / ntt;
-    const int tt = local - it.wt * ntt;
+    int tt;
+    if (wt_fastest) {  // all weight tiles of a token tile, then the next token tile
+        tt = local / NW;
+        it.wt = local - tt * NW;
+    } else {           // all token tiles of a weight tile, then the next weight tile
+        it.wt = local / ntt;
+        tt = local - it.wt * ntt;
+    }
     const int c = offs[it.e + 1] - offs[it.e];
     const int ts = ((c + ntt - 1) / ntt + 15) & ~15;
     it.t0 = offs[it.e] + tt * ts;
@@ -247,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool issued[STAGES];
             for (int i = 0; i < STAGES; ++i) issued[i] = false;
             for (int item = pair; item < total && !aborted(ctl); item += npairs) {
-                const Item it = decode(item, NW, mts, offs, E);
+                const Item it = decode(item, NW, mts, offs, E, p.wt_fastest != 0);
                 const int trow = it.t0 + half * (it.N / 2);
                 const int wc = wcoord(it);
                 bool ok = true;
@@ -281,7 +291,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int tile = 0;
             bool any = false;
             for (int item = pair; item < total && !aborted(ctl); item += npairs, ++tile) {
-                const Item it = decode(item, NW, mts, offs, E);
+                const Item it = decode(item, NW, mts, offs, E, p.wt_fastest != 0);
                 const uint32_t idesc = idesc_bf16_f32(2 * WM, it.N);
                 const int buf = tile & 1;
                 const uint32_t use = static_cast<uint32_t>(tile >> 1);
@@ -325,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t use = static_cast<uint32_t>(tile >> 1);
             if (!wait_bar(&ctl->tfull[buf], use & 1u, ctl, p.status)) break;
             tc_fence_after();
-            const Item it = decode(item, NW, mts, offs, E);
+            const Item it = decode(item, NW, mts, offs, E, p.wt_fastest != 0);
             const uint32_t t_lane = tmem_base + static_cast<uint32_t>(buf * TN) +
                                     (static_cast<uint32_t>(q * 32) << 16);
             const int nvalid = min(it.rows, p.rows_cap - it.t0);  // tokens stored
@@ -377,36 +387,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 dst += NOUT;
                             }
                         } else if constexpr (MODE == kEpiResid) {
-                            // out = x + acc (x read and out written by this thread: in place is fine)
+                            // out = x + acc. out may be x, so a store may not move
+                            // ahead of the load of its own element: the loads of 16
+                            // rows are issued together, then their 16 stores (each
+                            // thread reads and writes only its own elements).
                             const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(p.resid) +
                                                       r0 * NOUT + n;
 #pragma unroll
-                            for (int j = 0; j < 64; ++j) {
-                                if (j < lim)
-                                    *dst = __float2bfloat16_rn(__bfloat162float(*xr) +
-                                                               __uint_as_float(v[j >> 5][j & 31]));
-                                dst += NOUT;
-                                xr += NOUT;
+                            for (int j0 = 0; j0 < 64; j0 += 16) {
+                                float xv[16];
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    xv[j] = j0 + j < lim ? __bfloat162float(xr[static_cast<size_t>(j0 + j) * NOUT]) : 0.f;
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    if (j0 + j < lim)
+                                        dst[static_cast<size_t>(j0 + j) * NOUT] = __float2bfloat16_rn(
+                                            xv[j] + __uint_as_float(v[(j0 + j) >> 5][(j0 + j) & 31]));
                             }
                         } else {  // kEpiConv: y = u * (k0 a_t + k1 a_{t-1} + k2 a_{t-2}) per sequence
-                            const __nv_bfloat16 *a = static_cast<const __nv_bfloat16 *>(p.aux);
+                            // this thread's rows r0 .. r0+63 of channel n: a rolling
+                            // window over a, the two values before the chunk from a
+                            // (same sequence) or the sequence's carried state, the
+                            // chunk's own a loaded 16 rows at a time
+                            const __nv_bfloat16 *a = static_cast<const __nv_bfloat16 *>(p.aux) + n;
                             const float k0 = p.conv[n * 3], k1 = p.conv[n * 3 + 1], k2 = p.conv[n * 3 + 2];
+                            const int T = p.seq_len;
+                            int b = static_cast<int>(r0 / T);
+                            int t = static_cast<int>(r0 - static_cast<size_t>(b) * T);
+                            auto hist = [&](int seq, int slot) {  // a of position slot - 2 of seq
+                                return p.state_in ? p.state_in[(static_cast<size_t>(seq) * 2 + slot) * NOUT + n] : 0.f;
+                            };
+                            float am1 = t >= 1 ? __bfloat162float(a[(r0 - 1) * NOUT]) : hist(b, 1);
+                            float am2 = t >= 2 ? __bfloat162float(a[(r0 - 2) * NOUT])
+                                               : t == 1 ? hist(b, 1) : hist(b, 0);
 #pragma unroll
-                            for (int j = 0; j < 64; ++j) {
-                                if (j < lim) {
-                                    const size_t r = r0 + j;
-                                    const int b = static_cast<int>(r / p.seq_len);
-                                    const int t = static_cast<int>(r - static_cast<size_t>(b) * p.seq_len);
-                                    const float a0 = __bfloat162float(a[r * NOUT + n]);
-                                    float a1, a2;
-                                    if (t >= 1) a1 = __bfloat162float(a[(r - 1) * NOUT + n]);
-                                    else a1 = p.state_in ? p.state_in[(static_cast<size_t>(b) * 2 + 1) * NOUT + n] : 0.f;
-                                    if (t >= 2) a2 = __bfloat162float(a[(r - 2) * NOUT + n]);
-                                    else a2 = p.state_in ? p.state_in[(static_cast<size_t>(b) * 2 + t) * NOUT + n] : 0.f;
-                                    const float cv = fmaf(k2, a2, fmaf(k1, a1, k0 * a0));
-                                    *dst = __float2bfloat16_rn(__uint_as_float(v[j >> 5][j & 31]) * cv);
+                            for (int j0 = 0; j0 < 64; j0 += 16) {
+                                float av[16];
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    av[j] = j0 + j < lim ? __bfloat162float(a[(r0 + j0 + j) * NOUT]) : 0.f;
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) {
+                                    if (j0 + j < lim) {
+                                        if (t == 0) {  // a new sequence starts at this row
+                                            am1 = hist(b, 1);
+                                            am2 = hist(b, 0);
+                                        }
+                                        const float cv = fmaf(k2, am2, fmaf(k1, am1, k0 * av[j]));
+                                        dst[static_cast<size_t>(j0 + j) * NOUT] = __float2bfloat16_rn(
+                                            __uint_as_float(v[(j0 + j) >> 5][(j0 + j) & 31]) * cv);
+                                        am2 = am1;
+                                        am1 = av[j];
+                                        if (++t == T) { t = 0; ++b; }
+                                    }
                                 }
-                                dst += NOUT;
                             }
                         }
                     }

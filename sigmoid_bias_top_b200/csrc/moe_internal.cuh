@@ -8,6 +8,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 
 #include <utility>
 
@@ -92,6 +94,7 @@ struct GroupedParams {
     const float *conv;        // kEpiConv: taps [d][3] by lag
     const float *state_in;    // kEpiConv: [rows/seq_len][2][d] a of positions -2, -1, or null
     int seq_len;              // kEpiConv: positions per sequence (rows are sequence-major)
+    int wt_fastest;           // CTA-pair kernel: weight tiles vary fastest within an expert
 };
 
 // Epilogue modes of the CTA-pair GEMM (launch_gemm_tc2_mode).
@@ -187,8 +190,18 @@ inline int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess
-               ? MOE_OK : MOE_ERR_CUDA;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (err == cudaSuccess) return MOE_OK;
+    if (getenv("MOE_DEBUG")) {  // diagnostics on request: why the launch was refused
+        cudaFuncAttributes fa = {};
+        cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(kern));
+        fprintf(stderr,
+                "moe: launch failed: %s (grid %u, block %u, smem %zu; kernel: %d regs, "
+                "max %d threads, max dyn smem %d)\n",
+                cudaGetErrorString(err), grid.x, block.x, smem, fa.numRegs, fa.maxThreadsPerBlock,
+                fa.maxDynamicSharedSizeBytes);
+    }
+    return MOE_ERR_CUDA;
 }
 
 // Token chunks of the dispatch: about kChunkAssign assignments each, a whole
