@@ -485,6 +485,16 @@ def args_name(w):
 def run_ours(args, w, world, rank, local):
     torch.cuda.set_device(local)
     init_dist(world, "nccl")
+    if isinstance(w, W.BlockWorkload):
+        # a dense or conv block on its own (profiling runs): its measurement
+        # is the line; no host-buffer path or oracle leg
+        r = measure_block(w, args, args.steps, world, rank, local)
+        r.update({"metric": f"{w.kind} block tokens/s", "n_gpus": world, "warmup": args.warmup,
+                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                  "data": "synthetic (seeded; random-init weights of the block's shapes)",
+                  "config": {"workload": w.name, "parallelism": "single" if world == 1 else
+                             f"replicas{world}"}})
+        return r
     head = measure(w, args, args.steps, world, rank, local, headline=True)
     line = {
         "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
@@ -516,12 +526,17 @@ def run_ours(args, w, world, rank, local):
         for name in extra:
             if name == args.workload:
                 continue
-            if name in W.BLOCK_WORKLOADS:
-                r = measure_block(W.BLOCK_WORKLOADS[name], args, DEFAULT_STEPS[name], world,
-                                  rank, local)
-            else:
-                r = measure(W.WORKLOADS[name], args, DEFAULT_STEPS[name], world, rank, local,
-                            headline=False)
+            try:
+                if name in W.BLOCK_WORKLOADS:
+                    r = measure_block(W.BLOCK_WORKLOADS[name], args, DEFAULT_STEPS[name], world,
+                                      rank, local)
+                else:
+                    r = measure(W.WORKLOADS[name], args, DEFAULT_STEPS[name], world, rank, local,
+                                headline=False)
+            except Exception as exc:  # one workload's failure must not lose the headline line
+                r = {"error": f"{type(exc).__name__}: {exc}"}
+                torch.cuda.synchronize()
+                torch.cuda.empty_cache()
             line["workloads"][name] = r
     return line
 
@@ -595,7 +610,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="decode",
+                    choices=sorted(W.WORKLOADS) + sorted(W.BLOCK_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
@@ -615,8 +631,10 @@ def main(argv=None):
         args.extra = EXTRA if args.workload == "decode" else ""
     if args.repeats < 1:
         ap.error("--repeats must be >= 1")
-    w = W.WORKLOADS[args.workload]
+    w = W.WORKLOADS.get(args.workload) or W.BLOCK_WORKLOADS[args.workload]
     world, rank, local = dist_env()
+    if args.impl == "reference" and isinstance(w, W.BlockWorkload):
+        ap.error("the reference arm times the MoE block's oracle; pick an MoE workload")
     if args.impl == "reference":
         line = run_reference(args, w, world, rank)
     else:

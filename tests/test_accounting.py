@@ -44,3 +44,35 @@ def test_fp8_bytes():
     assert w == 56 * (A.expert_weights(2048, 1536) + 2304)
     assert A.fp8_experts_bytes(56, 128, 2048, 1536) - w == \
         128 * (2048 + 64) + 2 * 128 * (1536 + 48) + 128 * 2048 * 2
+
+
+def test_block_work_sums_to_the_block_flops():
+    """The per-kernel FLOPs of the dense and conv blocks add up to the
+    block's per-token count (dense: three d x I matrices; conv: W_in's three
+    d x d streams and W_out), times the tokens."""
+    n, d, I = 8192, 2048, 6144
+    dense = sum(A.block_kernel_work("dense", k, n, d, I)[0]
+                for k in ("norm", "gate_up", "down_residual"))
+    conv = sum(A.block_kernel_work("conv", k, n, d)[0]
+               for k in ("norm", "in_gv", "in_u_conv", "out_residual", "state"))
+    assert dense == n * A.block_flops_per_token("dense", d, I) == 2 * n * 3 * d * I
+    assert conv == n * A.block_flops_per_token("conv", d) == 2 * n * 4 * d * d
+
+
+def test_bench_takes_the_burst_peak_unless_power_capped_or_long():
+    import bench
+    from sigmoid_bias_top_b200 import workloads as W
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    w = W.PREFILL
+    ms = {"gate_up": 0.35}
+    calm = {"reasons": []}
+    capped = {"reasons": ["sw_power_cap"]}
+    b = bench.roofline(w, "gate_up", ms, 64, peaks, "measured", calm, 0.2)
+    assert b[0] == "tensor" and b[3] == 1600.0
+    assert bench.roofline(w, "gate_up", ms, 64, peaks, "measured", capped, 0.2)[3] == 1400.0
+    assert bench.roofline(w, "gate_up", ms, 64, peaks, "measured", calm, 1.5)[3] == 1400.0
+    fp8 = bench.roofline(W.PREFILL_FP8, "experts", {"experts": 1.0}, 64, peaks, "measured",
+                         calm, 0.2)
+    assert fp8[3] == 3200.0                       # e4m3: twice the bf16 peak
+    dec = bench.roofline(W.DECODE, "experts", {"experts": 0.17}, 54, peaks, "measured", calm, 0.1)
+    assert dec[0] == "hbm" and dec[3] == 6000.0
