@@ -89,9 +89,16 @@ int moe_block_destroy(moe_block_ctx *h);
 
 /* Per-kernel timing, as moe_profile / moe_kernel_times / moe_kernel_name:
  * CUDA events between the launches of every forward while enabled (the
- * events separate the launches); mean milliseconds per launch; names
- * norm, gate_up, down_residual (dense) or norm, in_gv, in_u_conv,
- * out_residual, state (conv). */
+ * events separate the launches); mean milliseconds per launch; names of the
+ * last forward's launches: norm, gate_up, down_residual (dense) or norm,
+ * in_gv, in_u_conv, out_residual, state (conv). Small batches, whose GEMMs
+ * would leave most of the GPU idle, split K: a GEMM then writes fp32 partial
+ * sums ("gate_up_split", "down_split", "in_gv_split", "in_u_split",
+ * "out_split") and a second launch adds them and finishes the step
+ * ("gate_up_reduce", "down_residual_reduce", "in_gv_reduce",
+ * "in_u_conv_reduce", "out_residual_reduce"). The environment variable
+ * MOE_BLOCK_SPLIT=0, read at create, keeps every GEMM unsplit (the same
+ * result; for testing both paths). */
 int moe_block_profile(moe_block_ctx *h, int enable);
 int moe_block_kernel_times(moe_block_ctx *h, float *ms, int n);
 const char *moe_block_kernel_name(moe_block_ctx *h, int i);

@@ -90,6 +90,12 @@ def block_kernel_work(kind: str, kernel: str, n: int, d: int, d_ff: int = 0):
             "norm": (0, 2 * n * d * b),
             "gate_up": (2 * n * 2 * I * d, 2 * I * d * b + n * d * b + n * I * b),
             "down_residual": (2 * n * d * I, d * I * b + n * I * b + 2 * n * d * b),
+            # split-K (small batches): the GEMMs' fp32 partial sums are
+            # intermediates; the reduce launches write the step's output
+            "gate_up_split": (2 * n * 2 * I * d, 2 * I * d * b + n * d * b),
+            "gate_up_reduce": (0, n * I * b),
+            "down_split": (2 * n * d * I, d * I * b + n * I * b),
+            "down_residual_reduce": (0, 2 * n * d * b),
         }
     else:
         table = {
@@ -98,6 +104,12 @@ def block_kernel_work(kind: str, kernel: str, n: int, d: int, d_ff: int = 0):
             "in_u_conv": (2 * n * d * d, d * d * b + n * d * b + n * d * b + n * d * b),
             "out_residual": (2 * n * d * d, d * d * b + n * d * b + 2 * n * d * b),
             "state": (0, 0),
+            "in_gv_split": (2 * n * 2 * d * d, 2 * d * d * b + n * d * b),
+            "in_gv_reduce": (0, n * d * b),
+            "in_u_split": (2 * n * d * d, d * d * b + n * d * b),
+            "in_u_conv_reduce": (0, 2 * n * d * b),
+            "out_split": (2 * n * d * d, d * d * b + n * d * b),
+            "out_residual_reduce": (0, 2 * n * d * b),
         }
     return table[kernel]
 

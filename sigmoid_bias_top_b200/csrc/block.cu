@@ -33,7 +33,8 @@ using namespace moe;
 namespace {
 
 constexpr int kNormThreads = 256;
-constexpr int kMaxLaunches = 5;
+constexpr int kMaxLaunches = 8;
+constexpr size_t kPartialBytes = size_t(16) << 20;  // fp32 partial sums of split-K GEMMs
 
 // xn[r] = bf16(x[r] * rinv * gain), rinv = 1 / sqrt(mean(x[r]^2) + eps), one
 // warp per row (bf16 rows, d % 8 == 0). Block 0 also writes the one-group
@@ -112,6 +113,56 @@ __global__ void conv_state_kernel(const __nv_bfloat16 *a, const float *state_in,
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Split-K GEMMs of small batches leave fp32 partial sums part[S][N][width];
+// this kernel adds the S slices in slice order (deterministic) and finishes
+// the step, for outputs [N][W]:
+//   kRedSiluMul: width 2W (gate, then up): act = bf16(silu(sum g) * sum u)
+//   kRedMul:     width 2W (g, then v):     a   = bf16(sum g * sum v)
+//   kRedConv:    width W (u): y = bf16(sum u * (k0 a_t + k1 a_{t-1} + k2 a_{t-2}))
+//                along each sequence of T rows, the carried state before it
+//   kRedResid:   width W: out = bf16(x + sum)
+// SiLU and the convolution are formed as in the pair GEMM's epilogues.
+enum { kRedSiluMul = 0, kRedMul = 1, kRedConv = 2, kRedResid = 3 };
+
+template <int KIND>
+__global__ void __launch_bounds__(256)
+    block_reduce_kernel(const float *part, int S, int N, int W, const __nv_bfloat16 *x,
+                        __nv_bfloat16 *dst, const float *conv, const __nv_bfloat16 *a,
+                        const float *state_in, int T) {
+    pdl_trigger();
+    pdl_wait();
+    const bool paired = KIND == kRedSiluMul || KIND == kRedMul;
+    const size_t width = paired ? 2 * static_cast<size_t>(W) : static_cast<size_t>(W);
+    const size_t n = static_cast<size_t>(N) * W;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const size_t r = i / W, c = i % W;
+        float g = 0.f, u = 0.f;
+        for (int sl = 0; sl < S; ++sl) {
+            const float *row = part + (static_cast<size_t>(sl) * N + r) * width;
+            g += row[c];
+            if (paired) u += row[W + c];
+        }
+        float v;
+        if (KIND == kRedSiluMul) {
+            v = __fdividef(g, 1.0f + __expf(-g)) * u;
+        } else if (KIND == kRedMul) {
+            v = g * u;
+        } else if (KIND == kRedConv) {
+            const int b = static_cast<int>(r / T), t = static_cast<int>(r % T);
+            const float a0 = __bfloat162float(a[r * W + c]);
+            const float a1 = t >= 1 ? __bfloat162float(a[(r - 1) * W + c])
+                                    : state_in ? state_in[(static_cast<size_t>(b) * 2 + 1) * W + c] : 0.f;
+            const float a2 = t >= 2 ? __bfloat162float(a[(r - 2) * W + c])
+                             : state_in ? state_in[(static_cast<size_t>(b) * 2 + t) * W + c] : 0.f;
+            v = g * fmaf(conv[c * 3 + 2], a2, fmaf(conv[c * 3 + 1], a1, conv[c * 3] * a0));
+        } else {
+            v = __bfloat162float(x[i]) + g;
+        }
+        dst[i] = __float2bfloat16_rn(v);
+    }
+}
+
 }  // namespace
 
 struct moe_block_ctx {
@@ -127,6 +178,11 @@ struct moe_block_ctx {
     int *status;
     CUtensorMap m_w1, m_w2, m_w3;  // dense: gate/up 4-D, down; conv: g/v 4-D, u rows, w_out
     CUtensorMap m_xn, m_mid;       // token rows: xn, and act (dense) or y (conv)
+    float *partial;               // split-K partial sums (kPartialBytes)
+    bool split_ok;                // MOE_BLOCK_SPLIT=0 at create keeps every GEMM unsplit
+    // the launch sequence of the last forward (it depends on the batch size)
+    const char *names[kMaxLaunches + 4];
+    int n_names;
     // profiling: events between the launches of every forward since enabled
     bool profile;
     int n_launch;
@@ -134,8 +190,6 @@ struct moe_block_ctx {
     size_t ev_used;
 };
 
-static const char *kDenseNames[] = {"norm", "gate_up", "down_residual"};
-static const char *kConvNames[] = {"norm", "in_gv", "in_u_conv", "out_residual", "state"};
 
 static void block_free(moe_block_ctx *h) {
     if (!h) return;
@@ -145,6 +199,8 @@ static void block_free(moe_block_ctx *h) {
 }
 
 static int block_alloc(moe_block_ctx *h, const size_t *sizes, int n, void **ptrs) {
+    const char *e = getenv("MOE_BLOCK_SPLIT");  // "0": no split-K (both paths compute the same)
+    h->split_ok = !(e && e[0] == '0');
     size_t total = 0, off[8];
     for (int i = 0; i < n; ++i) {
         off[i] = total;
@@ -189,9 +245,10 @@ extern "C" int moe_dense_create(int d, int d_ff, float eps, const moe_dense_weig
     h->n_sm = n_sm; h->eps = eps; h->gain = w->norm_gain; h->w1 = w->w_gate_up;
     h->w2 = w->w_down; h->n_launch = 3;
     const size_t C = max_tokens;
-    const size_t sizes[] = {C * d * 2, C * d_ff * 2, 4 * 4, 256};
-    void *p[4];
-    if ((rc = block_alloc(h, sizes, 4, p)) != MOE_OK) { block_free(h); return rc; }
+    const size_t sizes[] = {C * d * 2, C * d_ff * 2, 4 * 4, 256, kPartialBytes};
+    void *p[5];
+    if ((rc = block_alloc(h, sizes, 5, p)) != MOE_OK) { block_free(h); return rc; }
+    h->partial = static_cast<float *>(p[4]);
     h->xn = static_cast<__nv_bfloat16 *>(p[0]);
     h->mid = static_cast<__nv_bfloat16 *>(p[1]);
     h->loc = static_cast<int32_t *>(p[2]);
@@ -227,9 +284,10 @@ extern "C" int moe_conv_create(int d, float eps, const moe_conv_weights *w, int 
     h->n_sm = n_sm; h->eps = eps; h->gain = w->norm_gain; h->w1 = w->w_in; h->w2 = w->w_out;
     h->conv = w->conv; h->n_launch = 4;
     const size_t C = max_tokens;
-    const size_t sizes[] = {C * d * 2, C * d * 2, C * d * 2, 4 * 4, 256};
-    void *p[5];
-    if ((rc = block_alloc(h, sizes, 5, p)) != MOE_OK) { block_free(h); return rc; }
+    const size_t sizes[] = {C * d * 2, C * d * 2, C * d * 2, 4 * 4, 256, kPartialBytes};
+    void *p[6];
+    if ((rc = block_alloc(h, sizes, 6, p)) != MOE_OK) { block_free(h); return rc; }
+    h->partial = static_cast<float *>(p[5]);
     h->xn = static_cast<__nv_bfloat16 *>(p[0]);
     h->mid = static_cast<__nv_bfloat16 *>(p[1]);
     h->y = static_cast<__nv_bfloat16 *>(p[2]);
@@ -293,9 +351,40 @@ static GroupedParams group_params(moe_block_ctx *h, bool paired, int n_out, int 
     return gp;
 }
 
-#define BLOCK_MARK()                                                                \
+// K slices for one all-token pair GEMM: split while its items (token tiles x
+// weight tiles) leave CTA pairs idle, aiming at two items per pair, within
+// the partial buffer, every slice non-empty. 1 = no split.
+static int pick_split(const moe_block_ctx *h, int N, int items, int K, size_t width) {
+    const int pairs = h->n_sm / 2;
+    if (!h->split_ok || items >= pairs) return 1;
+    const int nk = (K + kTcPairBK - 1) / kTcPairBK;
+    int want = (2 * pairs + items - 1) / items;
+    const size_t cap = kPartialBytes / (static_cast<size_t>(N) * width * 4);
+    if (static_cast<size_t>(want) > cap) want = static_cast<int>(cap);
+    if (want > nk) want = nk;
+    if (want <= 1) return 1;
+    const int nkc = (nk + want - 1) / want;
+    return (nk + nkc - 1) / nkc;
+}
+
+template <int KIND>
+static int reduce_launch(moe_block_ctx *h, int S, int N, int W, const void *x, void *dst,
+                         const void *a, const float *state_in, int T, cudaStream_t s) {
+    const size_t n = static_cast<size_t>(N) * W;
+    int blocks = static_cast<int>((n + 255) / 256);
+    if (blocks > 8 * h->n_sm) blocks = 8 * h->n_sm;
+    return launch_k(block_reduce_kernel<KIND>, dim3(blocks), dim3(256), 0, s,
+                    static_cast<const float *>(h->partial), S, N, W,
+                    static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(dst),
+                    static_cast<const float *>(h->conv), static_cast<const __nv_bfloat16 *>(a),
+                    state_in, T);
+}
+
+#define BLOCK_MARK(name)                                                            \
     do {                                                                            \
-        if (ev && cudaEventRecord(ev[ne++], s) != cudaSuccess) return MOE_ERR_CUDA; \
+        if (ne > 0) h->names[ne - 1] = (name);                                      \
+        if (ev && cudaEventRecord(ev[ne], s) != cudaSuccess) return MOE_ERR_CUDA;   \
+        ++ne;                                                                       \
     } while (0)
 #define BLOCK_TRY(expr)                         \
     do {                                        \
@@ -312,22 +401,45 @@ extern "C" int moe_dense_forward(moe_block_ctx *h, const void *x, void *out, int
     if (!aligned16(x) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaEvent_t *ev = next_events(h);
+    const int N = n_tokens, d = h->d, I = h->I;
+    const int tiles = (N + kTcPairTileM - 1) / kTcPairTileM;
     int ne = 0;
-    BLOCK_MARK();
-    BLOCK_TRY(norm_launch(h, x, n_tokens, s));
-    BLOCK_MARK();
-    GroupedParams gp = group_params(h, true, h->I, h->d);
-    gp.c = h->mid;
-    BLOCK_TRY(launch_gemm_tc2_mode(kEpiSiluMul, h->m_w1, h->m_xn, gp, h->n_sm, s));
-    BLOCK_MARK();
-    gp = group_params(h, false, h->d, h->I);
-    gp.c = out;
-    gp.resid = x;
-    // the act rows (N x I) outweigh W_down (d x I) as soon as N > d: then
-    // each token tile is read once while the weight tiles stay in L2
-    gp.wt_fastest = n_tokens > h->d;
-    BLOCK_TRY(launch_gemm_tc2_mode(kEpiResid, h->m_w2, h->m_mid, gp, h->n_sm, s));
-    BLOCK_MARK();
+    BLOCK_MARK(nullptr);
+    BLOCK_TRY(norm_launch(h, x, N, s));
+    BLOCK_MARK("norm");
+    // gate/up: SiLU(gate) * up into act
+    const int s1 = pick_split(h, N, tiles * ((I + 127) / 128), d, 2 * static_cast<size_t>(I));
+    GroupedParams gp = group_params(h, true, I, d);
+    if (s1 > 1) {
+        gp.ksplit = s1; gp.partial = h->partial; gp.partial_rows = N;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiPartialPaired, h->m_w1, h->m_xn, gp, h->n_sm, s));
+        BLOCK_MARK("gate_up_split");
+        BLOCK_TRY(reduce_launch<kRedSiluMul>(h, s1, N, I, nullptr, h->mid, nullptr, nullptr, 1, s));
+        BLOCK_MARK("gate_up_reduce");
+    } else {
+        gp.c = h->mid;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiSiluMul, h->m_w1, h->m_xn, gp, h->n_sm, s));
+        BLOCK_MARK("gate_up");
+    }
+    // down + residual
+    const int s2 = pick_split(h, N, tiles * ((d + 255) / 256), I, d);
+    gp = group_params(h, false, d, I);
+    if (s2 > 1) {
+        gp.ksplit = s2; gp.partial = h->partial; gp.partial_rows = N;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiPartial, h->m_w2, h->m_mid, gp, h->n_sm, s));
+        BLOCK_MARK("down_split");
+        BLOCK_TRY(reduce_launch<kRedResid>(h, s2, N, d, x, out, nullptr, nullptr, 1, s));
+        BLOCK_MARK("down_residual_reduce");
+    } else {
+        gp.c = out;
+        gp.resid = x;
+        // the act rows (N x I) outweigh W_down (d x I) as soon as N > d: then
+        // each token tile is read once while the weight tiles stay in L2
+        gp.wt_fastest = N > d;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiResid, h->m_w2, h->m_mid, gp, h->n_sm, s));
+        BLOCK_MARK("down_residual");
+    }
+    h->n_names = ne - 1;
     return MOE_OK;
 }
 
@@ -355,38 +467,67 @@ extern "C" int moe_conv_forward(moe_block_ctx *h, const void *x, void *out, int 
     if (!x || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
     const int N = static_cast<int>(n), d = h->d;
+    const int tiles = (N + kTcPairTileM - 1) / kTcPairTileM;
     cudaEvent_t *ev = next_events(h);
     int ne = 0;
-    BLOCK_MARK();
+    BLOCK_MARK(nullptr);
     BLOCK_TRY(norm_launch(h, x, N, s));
-    BLOCK_MARK();
+    BLOCK_MARK("norm");
     // a = g * v
+    const int s1 = pick_split(h, N, tiles * ((d + 127) / 128), d, 2 * static_cast<size_t>(d));
     GroupedParams gp = group_params(h, true, d, d);
-    gp.c = h->mid;
-    BLOCK_TRY(launch_gemm_tc2_mode(kEpiMul, h->m_w1, h->m_xn, gp, h->n_sm, s));
-    BLOCK_MARK();
+    if (s1 > 1) {
+        gp.ksplit = s1; gp.partial = h->partial; gp.partial_rows = N;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiPartialPaired, h->m_w1, h->m_xn, gp, h->n_sm, s));
+        BLOCK_MARK("in_gv_split");
+        BLOCK_TRY(reduce_launch<kRedMul>(h, s1, N, d, nullptr, h->mid, nullptr, nullptr, 1, s));
+        BLOCK_MARK("in_gv_reduce");
+    } else {
+        gp.c = h->mid;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiMul, h->m_w1, h->m_xn, gp, h->n_sm, s));
+        BLOCK_MARK("in_gv");
+    }
     // y = u * (k0 a_t + k1 a_{t-1} + k2 a_{t-2}) along each sequence
+    const int s2 = pick_split(h, N, tiles * ((d + 255) / 256), d, d);
     gp = group_params(h, false, d, d);
-    gp.c = h->y;
-    gp.aux = h->mid;
-    gp.conv = h->conv;
-    gp.state_in = state_in;
-    gp.seq_len = seq_len;
-    BLOCK_TRY(launch_gemm_tc2_mode(kEpiConv, h->m_w2, h->m_xn, gp, h->n_sm, s));
-    BLOCK_MARK();
+    if (s2 > 1) {
+        gp.ksplit = s2; gp.partial = h->partial; gp.partial_rows = N;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiPartial, h->m_w2, h->m_xn, gp, h->n_sm, s));
+        BLOCK_MARK("in_u_split");
+        BLOCK_TRY(reduce_launch<kRedConv>(h, s2, N, d, nullptr, h->y, h->mid, state_in, seq_len, s));
+        BLOCK_MARK("in_u_conv_reduce");
+    } else {
+        gp.c = h->y;
+        gp.aux = h->mid;
+        gp.conv = h->conv;
+        gp.state_in = state_in;
+        gp.seq_len = seq_len;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiConv, h->m_w2, h->m_xn, gp, h->n_sm, s));
+        BLOCK_MARK("in_u_conv");
+    }
     // out = x + W_out y
+    const int s3 = pick_split(h, N, tiles * ((d + 255) / 256), d, d);
     gp = group_params(h, false, d, d);
-    gp.c = out;
-    gp.resid = x;
-    BLOCK_TRY(launch_gemm_tc2_mode(kEpiResid, h->m_w3, h->m_mid, gp, h->n_sm, s));
-    BLOCK_MARK();
+    if (s3 > 1) {
+        gp.ksplit = s3; gp.partial = h->partial; gp.partial_rows = N;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiPartial, h->m_w3, h->m_mid, gp, h->n_sm, s));
+        BLOCK_MARK("out_split");
+        BLOCK_TRY(reduce_launch<kRedResid>(h, s3, N, d, x, out, nullptr, nullptr, 1, s));
+        BLOCK_MARK("out_residual_reduce");
+    } else {
+        gp.c = out;
+        gp.resid = x;
+        BLOCK_TRY(launch_gemm_tc2_mode(kEpiResid, h->m_w3, h->m_mid, gp, h->n_sm, s));
+        BLOCK_MARK("out_residual");
+    }
     if (state_out) {
         const size_t m = static_cast<size_t>(n_seqs) * d;
         const int blocks = static_cast<int>((m + 255) / 256 < 1024 ? (m + 255) / 256 : 1024);
         conv_state_kernel<<<blocks, 256, 0, s>>>(h->mid, state_in, state_out, n_seqs, seq_len, d);
         if (cudaPeekAtLastError() != cudaSuccess) return MOE_ERR_CUDA;
-        BLOCK_MARK();
+        BLOCK_MARK("state");
     }
+    h->n_names = ne - 1;
     return MOE_OK;
 }
 
@@ -445,7 +586,6 @@ extern "C" int moe_block_kernel_times(moe_block_ctx *h, float *ms, int n) {
 }
 
 extern "C" const char *moe_block_kernel_name(moe_block_ctx *h, int i) {
-    if (!h || i < 0) return nullptr;
-    if (h->kind == 0) return i < 3 ? kDenseNames[i] : nullptr;
-    return i < 5 ? kConvNames[i] : nullptr;
+    if (!h || i < 0 || i >= h->n_names) return nullptr;
+    return h->names[i];
 }

@@ -187,7 +187,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_tc2_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmT, GroupedParams p) {
     // paired-row modes stage gate/up-style interleaved weight rows (4-D map)
-    constexpr bool GATE_UP = MODE == kEpiSiluMul || MODE == kEpiMul;
+    constexpr bool GATE_UP = MODE == kEpiSiluMul || MODE == kEpiMul || MODE == kEpiPartialPaired;
+    constexpr bool PARTIAL = MODE == kEpiPartial || MODE == kEpiPartialPaired;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -241,7 +242,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int NW = GATE_UP ? (p.I + 127) / 128 : (p.d + 2 * WM - 1) / (2 * WM);
     const int K = GATE_UP ? p.d : p.I;
     const int nk = (K + BK - 1) / BK;
-    const int total = mts[E] * NW;
+    // split-K: item = tile * S + slice; slice ks covers K blocks [ks*nkc, +nkc)
+    const int S = PARTIAL && p.ksplit > 1 ? p.ksplit : 1;
+    const int nkc = (nk + S - 1) / S;
+    const int total = mts[E] * NW * S;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -257,11 +261,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool issued[STAGES];
             for (int i = 0; i < STAGES; ++i) issued[i] = false;
             for (int item = pair; item < total && !aborted(ctl); item += npairs) {
-                const Item it = decode(item, NW, mts, offs, E, p.wt_fastest != 0);
+                const Item it = decode(item / S, NW, mts, offs, E, p.wt_fastest != 0);
+                const int kb0 = (item % S) * nkc, kb1 = min(nk, kb0 + nkc);
                 const int trow = it.t0 + half * (it.N / 2);
                 const int wc = wcoord(it);
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) { ok = false; break; }
                     uint8_t *sa = smem + s * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
@@ -291,7 +296,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int tile = 0;
             bool any = false;
             for (int item = pair; item < total && !aborted(ctl); item += npairs, ++tile) {
-                const Item it = decode(item, NW, mts, offs, E, p.wt_fastest != 0);
+                const Item it = decode(item / S, NW, mts, offs, E, p.wt_fastest != 0);
+                const int kb0 = (item % S) * nkc, kb1 = min(nk, kb0 + nkc);
                 const uint32_t idesc = idesc_bf16_f32(2 * WM, it.N);
                 const int buf = tile & 1;
                 const uint32_t use = static_cast<uint32_t>(tile >> 1);
@@ -299,7 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * TN);
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bar(&ctl->full[s], ph, ctl, p.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
@@ -308,7 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < BK / UK; ++kk)
                         umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + kk * UK * 2),
                                        sw128_kmajor_desc(b0 + kk * UK * 2), idesc,
-                                       (kb | kk) != 0 ? 1u : 0u);
+                                       (kb != kb0 || kk != 0) ? 1u : 0u);
                     any = true;
                     umma_commit_pair(&ctl->empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -335,11 +341,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t use = static_cast<uint32_t>(tile >> 1);
             if (!wait_bar(&ctl->tfull[buf], use & 1u, ctl, p.status)) break;
             tc_fence_after();
-            const Item it = decode(item, NW, mts, offs, E, p.wt_fastest != 0);
+            const Item it = decode(item / S, NW, mts, offs, E, p.wt_fastest != 0);
+                const int kb0 = (item % S) * nkc, kb1 = min(nk, kb0 + nkc);
             const uint32_t t_lane = tmem_base + static_cast<uint32_t>(buf * TN) +
                                     (static_cast<uint32_t>(q * 32) << 16);
             const int nvalid = min(it.rows, p.rows_cap - it.t0);  // tokens stored
-            if (GATE_UP) {
+            if constexpr (MODE == kEpiPartialPaired) {
+                // raw sums of the K slice: gate rows to columns f, up rows to NOUT + f
+                const int f = it.wt * 128 + half * 64 + q * 16 + (lane & 15);
+                float *prow = p.partial + (static_cast<size_t>(item % S) * p.partial_rows + it.t0) *
+                                              (2 * static_cast<size_t>(NOUT)) +
+                              (lane < 16 ? 0 : NOUT) + f;
+#pragma unroll 1
+                for (int c0 = c_first; c0 < it.N; c0 += 64 * (kEpiWarps / 4)) {
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(t_lane + c0, v[0]);
+                    tmem_ld_32x32b_x32(t_lane + c0 + 32, v[1]);
+                    tmem_ld_wait();
+                    const int lim = f < NOUT ? nvalid - c0 : 0;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (j < lim)
+                            prow[static_cast<size_t>(c0 + j) * (2 * NOUT)] = __uint_as_float(v[j >> 5][j & 31]);
+                }
+            } else if constexpr (MODE == kEpiPartial) {
+                const int n = it.wt * 2 * WM + half * WM + q * 32 + lane;
+                float *prow = p.partial +
+                              (static_cast<size_t>(item % S) * p.partial_rows + it.t0) * NOUT + n;
+#pragma unroll 1
+                for (int c0 = c_first; c0 < it.N; c0 += 64 * (kEpiWarps / 4)) {
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(t_lane + c0, v[0]);
+                    tmem_ld_32x32b_x32(t_lane + c0 + 32, v[1]);
+                    tmem_ld_wait();
+                    const int lim = n < NOUT ? nvalid - c0 : 0;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (j < lim) prow[static_cast<size_t>(c0 + j) * NOUT] = __uint_as_float(v[j >> 5][j & 31]);
+                }
+            } else if (GATE_UP) {
                 // lanes 0..15: gate of features f, lanes 16..31: up of the same f
                 const bool is_gate = lane < 16;
                 const int f = it.wt * 128 + half * 64 + q * 16 + (lane & 15);
@@ -513,6 +553,8 @@ int launch_gemm_tc2_mode(int mode, const CUtensorMap &w, const CUtensorMap &t,
         case kEpiMul: return launch<kEpiMul>(w, t, p, n_sm, s);
         case kEpiConv: return launch<kEpiConv>(w, t, p, n_sm, s);
         case kEpiResid: return launch<kEpiResid>(w, t, p, n_sm, s);
+        case kEpiPartialPaired: return launch<kEpiPartialPaired>(w, t, p, n_sm, s);
+        case kEpiPartial: return launch<kEpiPartial>(w, t, p, n_sm, s);
         default: return MOE_ERR_INVALID_ARG;
     }
 }

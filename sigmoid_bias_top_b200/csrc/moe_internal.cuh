@@ -95,6 +95,14 @@ struct GroupedParams {
     const float *state_in;    // kEpiConv: [rows/seq_len][2][d] a of positions -2, -1, or null
     int seq_len;              // kEpiConv: positions per sequence (rows are sequence-major)
     int wt_fastest;           // CTA-pair kernel: weight tiles vary fastest within an expert
+    // split-K (CTA-pair kernel, kEpiPartial / kEpiPartialPaired): every tile
+    // in ksplit K slices of ceil(nk / ksplit) 64-wide blocks, none empty (the
+    // caller picks ksplit so); slice ks writes fp32 sums to
+    // partial[ks][row][width], row < partial_rows, width = NOUT (plain) or
+    // 2 NOUT (paired: the first block's rows, then the partner rows)
+    int ksplit;
+    float *partial;
+    int partial_rows;
 };
 
 // Epilogue modes of the CTA-pair GEMM (launch_gemm_tc2_mode).
@@ -103,6 +111,9 @@ constexpr int kEpiPlain = 1;    // plain product                          (2-D w
 constexpr int kEpiMul = 2;      // paired rows: gate * up, no activation  (4-D weight map)
 constexpr int kEpiConv = 3;     // u * depthwise causal conv of a         (2-D weight map)
 constexpr int kEpiResid = 4;    // residual + product                     (2-D weight map)
+constexpr int kEpiPartialPaired = 5;  // paired rows, fp32 partial sums of a K slice (4-D)
+constexpr int kEpiPartial = 6;        // fp32 partial sums of a K slice         (2-D weight map)
+constexpr int kTcPairBK = 64;         // K per stage of the CTA-pair kernel
 
 struct DecodeParams {
     // the fused small-batch expert kernel (gate/up and down in one launch)

@@ -36,9 +36,21 @@ def cpu(layer):
     return {k: v.detach().cpu() for k, v in layer.items()}
 
 
+@pytest.fixture(params=["split", "unsplit"])
+def split_mode(request, monkeypatch):
+    """Small batches split K across the GPU (partial sums, then a reduce
+    launch); MOE_BLOCK_SPLIT=0 at create keeps every GEMM whole. Both paths
+    must give the same result."""
+    if request.param == "unsplit":
+        monkeypatch.setenv("MOE_BLOCK_SPLIT", "0")
+    else:
+        monkeypatch.delenv("MOE_BLOCK_SPLIT", raising=False)
+    return request.param
+
+
 # ------------------------------------------------------------------ dense
 @pytest.mark.parametrize("n,d,I", [(300, 256, 320), (1, 128, 64), (513, 192, 448)])
-def test_dense_ragged(n, d, I):
+def test_dense_ragged(n, d, I, split_mode):
     w = W.DENSE_PREFILL.scaled(n_seqs=n, seq_len=1, d=d, d_ff=I, w_std=0.06)
     layer = W.make_block_layer(w, "cuda")
     x = W.make_block_x(w, "cuda")
@@ -67,7 +79,7 @@ def test_dense_full_size_sampled(name):
     blk.close()
 
 
-def test_dense_in_place_and_deterministic():
+def test_dense_in_place_and_deterministic(split_mode):
     w = W.DENSE_PREFILL.scaled(n_seqs=260, seq_len=1, d=256, d_ff=256)
     layer = W.make_block_layer(w, "cuda")
     x = W.make_block_x(w, "cuda")
@@ -88,7 +100,7 @@ def conv_ref(x, layer, eps, state=None):
 
 
 @pytest.mark.parametrize("B,T,d", [(3, 300, 256), (1, 1, 128), (2, 7, 192), (5, 130, 64)])
-def test_conv_ragged(B, T, d):
+def test_conv_ragged(B, T, d, split_mode):
     """Sequences that cross the GEMM's 256-row token tiles, ragged tails, T < 3."""
     w = W.CONV_PREFILL.scaled(n_seqs=B, seq_len=T, d=d, w_std=0.06)
     layer = W.make_block_layer(w, "cuda")
@@ -104,7 +116,7 @@ def test_conv_ragged(B, T, d):
     np.testing.assert_allclose(st_out.double().cpu().numpy(), ref_state, rtol=2e-2, atol=2e-2)
 
 
-def test_conv_carried_state_and_decode_steps():
+def test_conv_carried_state_and_decode_steps(split_mode):
     """Prefill T1 positions, then T2 more with the state carried, then three
     decode steps (T = 1), against the oracle on the whole sequences."""
     B, d = 3, 256
@@ -165,7 +177,7 @@ def test_conv_prefill_full_size_windows():
     blk.close()
 
 
-def test_conv_in_place_and_deterministic():
+def test_conv_in_place_and_deterministic(split_mode):
     w = W.CONV_PREFILL.scaled(n_seqs=2, seq_len=300, d=256)
     layer = W.make_block_layer(w, "cuda")
     x = W.make_block_x(w, "cuda")
