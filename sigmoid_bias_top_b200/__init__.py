@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.moe_kernel_name.restype = ctypes.c_char_p
         L.moe_launches_per_forward.argtypes = [P, I]
         L.moe_selftest_timeout.argtypes = [P, I, P]
+        L.moe_selftest_fp8_divide.argtypes = [P, P, P, P, I, P]
+        L.moe_selftest_fp8_divide.restype = I
         L.moe_route_noalloc.argtypes = [P, I, P, P, P, I, I, I, I, F, F, P, P, P]
         L.moe_route_noalloc.restype = I
         L.moe_strerror.argtypes = [I]
@@ -144,6 +146,20 @@ def route_noalloc(x, layer: Dict, top_k: int, eps: float = 1e-6, routed_scale: f
                                    top_k, eps, routed_scale, idx.data_ptr(), w.data_ptr(),
                                    _stream_ptr(stream)), "moe_route_noalloc")
     return idx, w
+
+
+def selftest_fp8_divide(a, b, stream=None):
+    """(q, q_ref) for fp32 device tensors a, b of one shape: q = a / b as the
+    FP8 quantisers form it, q_ref = the IEEE quotient (moe_selftest_fp8_divide)."""
+    import torch
+    if a.dtype != torch.float32 or b.dtype != torch.float32 or a.shape != b.shape:
+        raise ValueError("a and b: fp32 tensors of one shape")
+    a, b = a.contiguous(), b.contiguous()
+    q, q_ref = torch.empty_like(a), torch.empty_like(a)
+    _check(lib().moe_selftest_fp8_divide(a.data_ptr(), b.data_ptr(), q.data_ptr(),
+                                         q_ref.data_ptr(), a.numel(), _stream_ptr(stream)),
+           "moe_selftest_fp8_divide")
+    return q, q_ref
 
 
 class MoeLayer:

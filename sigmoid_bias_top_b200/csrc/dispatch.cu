@@ -83,9 +83,10 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float *scale) {
     const float s = __fdiv_rn(m, 448.f);
     uint32_t w[2] = {0u, 0u};
     if (s > 0.f) {
+        const float rs = __frcp_rn(s);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {  // byte i of the 8 = value i
-            const uint32_t c = __nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t c = __nv_cvt_float_to_fp8(div_rn(v[i], s, rs), __NV_SATFINITE, __NV_E4M3);
             w[i >> 2] |= c << (8 * (i & 3));
         }
     }

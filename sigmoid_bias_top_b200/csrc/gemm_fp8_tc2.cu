@@ -26,22 +26,27 @@
 // The scales differ per K block, so the tensor cores cannot add one K block
 // onto the next: each K block's four MMAs (K = 32) start a fresh sum in one
 // of four 128-column TMEM buffers, and the epilogue warps (8 per CTA, two per
-// TMEM lane quarter, 64 token columns each) load it and add partial * f[col]
-// into fp32 registers, f[col] = sw * sa[token][kb] taken from a shared-memory
-// table of the tile's factors (gate and up factors of four columns side by
-// side, so the two half-warps read different banks). An eleventh warp builds
-// that table one chunk of 16 K blocks ahead (two chunk buffers), issuing all
-// of a chunk's scale loads before using any, so the scale reads' latency stays
-// off the epilogue's path; 11 warps keep the 168-register budget of 10 (the
-// fullest of the four register-file quarters holds three warps). At the
-// end of a gate/up tile the two threads of a feature swap half of their
-// columns (shuffle) and each forms SiLU(gate) * up for 32 tokens; the group
-// maximum over the pair's 128 features per token is a reduce-scatter
-// butterfly over the 16 features of a half-warp, then the four lane quarters
-// through shared memory, then the two CTAs through distributed shared memory
-// (each writes its maxima into both CTAs and arrives on both CTAs' barrier);
-// s = amax / 448 and codes e4m3(a / s) (IEEE division, nearest-even,
-// saturating) go to aq and as. A down tile stores bf16 y.
+// TMEM lane quarter, 64 token columns each) load it and add
+// partial * (sa[token][kb] * sw[kb]) into fp32 registers. The gate/up
+// epilogue loads 16x256b fragments, in which a thread holds 4 rows x 16 token
+// columns rather than 1 row x 64 columns, so it reads 16 activation scales
+// per K block (plus the two weight block scales) instead of 64 factors; the
+// down epilogue keeps one row per thread (32x32b) and reads the 64 factors
+// sa * sw, which lets it store 32 consecutive outputs of a token per warp
+// directly. An eleventh warp writes the scales of a chunk of 16 K blocks
+// ahead (two chunk buffers), in the order the fragments read them, issuing all
+// of a chunk's scale loads before using any; 11 warps keep the 168-register
+// budget of 10 (the fullest of the four register-file quarters holds three
+// warps). In a gate/up tile the lower fragment holds gate and the upper one
+// up rows of the same features, so at the tile end each thread forms
+// SiLU(gate) * up for its 32 values in place; the group maximum over the
+// pair's 128 features per token is a reduce-scatter butterfly over the 8
+// lanes that share columns, then the four lane quarters through shared
+// memory, then the two CTAs through distributed shared memory (each writes
+// its maxima into both CTAs and arrives on both CTAs' barrier). s = amax / 448
+// and the codes e4m3(a / s) (the IEEE quotient, by a reciprocal and one
+// correction step: div_rn; nearest-even, saturating) are staged in shared
+// memory and written to aq as 16-byte row pieces, s to as.
 // All waits are bounded (1 s) and report MOE_ERR_DEVICE_TIMEOUT; the pair
 // meets at a cluster barrier before TMEM is freed. No load uses multicast.
 #include <cooperative_groups.h>
@@ -74,6 +79,7 @@ constexpr int kThreads = 64 + kEpiThreads + 32;
 constexpr int CW = TN / 2;               // token columns per epilogue warp
 constexpr int TBL = 16;                  // K blocks per chunk of a warp's factor table
 constexpr int kEpiBar = 1;               // named barrier of the epilogue threads
+constexpr int kPitchU8 = 64 + 16;        // staged gate/up codes: bytes per token row
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // shared::cluster address in the pair's even CTA
 
@@ -90,11 +96,69 @@ struct Ctl {
     int abort;
     float red_local[4][TN];     // per lane quarter: column maxima over its 16 features
     float red_pair[2][2][TN];   // [tile parity][CTA][column]
-    float col_scale[2][TN];     // [tile parity][column]: amax / 448
-    // two chunks of factors sw * sa: per K block of the chunk, per 4 token
-    // columns, the 4 gate (or down) factors, then the 4 up factors
-    float4 tbl[2][TBL][TN / 4][2];
+    alignas(16) float2 col_sr[2][TN];  // [tile parity][column]: (amax / 448, RN(1 / that))
+    // two chunks of scales: per K block of the chunk, gate/up: the
+    // activation scale sa of every token column in fragment order (frag_pos)
+    // and the weight block scales sw of the gate and the up rows; down: the
+    // factors sa * sw of the token columns in column order
+    alignas(16) float sa[2][TBL][TN];
+    float2 sw[2][TBL];
+    // a gate/up tile's codes on their way to global memory: [TN][kPitchU8] bytes
+    alignas(16) uint8_t stage[TN * kPitchU8];
 };
+
+// Position of token column c in a factor-table row: the epilogue thread with
+// fragment column pair mq of column half ch reads its 16 columns
+// ch*CW + 8 i + 2 mq + e (i < 8, e < 2) as 16 consecutive floats.
+__device__ __forceinline__ int frag_pos(int c) {
+    const int ch = c / CW, cc = c % CW;
+    return ch * CW + ((cc & 7) >> 1) * 16 + 2 * (cc >> 3) + (cc & 1);
+}
+
+// tcgen05.ld .16x256b.x8: 16 TMEM lanes x 64 columns; thread t gets lane
+// t/4 (registers 4i, 4i+1) and lane t/4 + 8 (4i+2, 4i+3) of columns
+// 8 i + 2 (t % 4) + {0, 1}.
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void load_scales(float (&sv)[16], const float *src) {
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 v = s4[k];
+        sv[4 * k + 0] = v.x;
+        sv[4 * k + 1] = v.y;
+        sv[4 * k + 2] = v.z;
+        sv[4 * k + 3] = v.w;
+    }
+}
+
+// acc[4i + 2h + e] += v[4i + 2h + e] * sa[2i + e] * w, the factor rounded
+// to fp32 before the multiply-add
+__device__ __forceinline__ void promote(float (&acc)[32], const uint32_t (&v)[32],
+                                        const float (&sv)[16], float w) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float f = sv[2 * i + e] * w;
+            acc[4 * i + e] = fmaf(__uint_as_float(v[4 * i + e]), f, acc[4 * i + e]);
+            acc[4 * i + 2 + e] = fmaf(__uint_as_float(v[4 * i + 2 + e]), f, acc[4 * i + 2 + e]);
+        }
+    }
+}
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, int *status) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -385,12 +449,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == kTblWarp) {
-        // ---------------- factor tables (warp 10, both CTAs) ----------------
-        // per chunk of TBL K blocks of every tile: f = sw[kb] * sa[token][kb]
-        // for the tile's TN token columns; lane l takes columns 4l..4l+3,
-        // and lane j (j < 16) loads the gate (or down) weight block scale of
-        // K block kb0+j, lane 16+j the up one. All loads of a chunk are
-        // issued before any is used.
+        // ---------------- scale tables (warp 10, both CTAs) ----------------
+        // per chunk of TBL K blocks of every tile: sa[token][kb] of the tile's
+        // TN token columns (lane l takes columns 4l..4l+3) and the weight
+        // block scales (lane j < 16: the gate (or down) block of K block
+        // kb0+j, lane 16+j the up one). All loads of a chunk are issued
+        // before any is used.
         const float *sa_all = GATE_UP ? p.xs : p.as_in;
         const int ng = K / BK;
         uint32_t nchunk = 0;
@@ -423,13 +487,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < TBL; ++j) sa[c][j] = (valid && j < n) ? __ldg(sa_row + j) : 0.f;
                 }
-                float4 (*t)[TN / 4][2] = ctl->tbl[slot];
+                if constexpr (GATE_UP) {
+                    float *w2 = reinterpret_cast<float *>(&ctl->sw[slot][jj]);
+                    w2[lane < 16 ? 0 : 1] = wsc;
 #pragma unroll
-                for (int j = 0; j < TBL; ++j) {
-                    const float wg = __shfl_sync(0xffffffffu, wsc, j);
-                    const float wu = GATE_UP ? __shfl_sync(0xffffffffu, wsc, 16 + j) : wg;
-                    t[j][lane][0] = make_float4(sa[0][j] * wg, sa[1][j] * wg, sa[2][j] * wg, sa[3][j] * wg);
-                    t[j][lane][1] = make_float4(sa[0][j] * wu, sa[1][j] * wu, sa[2][j] * wu, sa[3][j] * wu);
+                    for (int c = 0; c < 4; ++c) {
+                        const int pos = frag_pos(4 * lane + c);
+#pragma unroll
+                        for (int j = 0; j < TBL; ++j) ctl->sa[slot][j][pos] = sa[c][j];
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < TBL; ++j) {
+                        const float w = __shfl_sync(0xffffffffu, wsc, j);
+                        *reinterpret_cast<float4 *>(&ctl->sa[slot][j][4 * lane]) =
+                            make_float4(sa[0][j] * w, sa[1][j] * w, sa[2][j] * w, sa[3][j] * w);
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->tbl_full[slot]);
@@ -438,76 +511,104 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue (warps 2..9, both CTAs) ----------------
+        // Warp (q, ch) owns TMEM lane quarter q and token columns ch*CW..+CW-1.
+        // It reads them as two 16x256b fragments: lanes 32q..+15 (gate rows of
+        // the quarter's 16 features, or down rows 32q..+15) and 32q+16..+31
+        // (the up rows of the same features, or down rows 32q+16..+31), so a
+        // thread holds, for fragment rows fr and fr + 8, 16 token columns
+        // ch*CW + 8 i + 2 mq + e of both: 16 activation scales per K block
+        // instead of one per column and register.
         const int ew = warp - 2;
         const int q = warp & 3;          // TMEM lane quarter
         const int ch = ew >> 2;          // token columns ch*CW .. +CW-1
-        const bool is_up = GATE_UP && lane >= 16;
-        const int role = is_up ? 1 : 0;
-        const float4 (*tbl)[TN / 4][2] = ctl->tbl[0];
-        // The gate/up epilogue threads meet at named barriers inside every
-        // tile, so they leave the tile loop together: the abort flag is
-        // agreed on at the start of a tile, and a wait that times out inside
-        // a tile skips the rest of its work but not its meeting points.
+        const int mq = lane & 3;         // column pair of each 8 columns
+        const int fr = lane >> 2;        // fragment rows fr and fr + 8
+        const int et = threadIdx.x - 64; // epilogue thread 0..255
+        // The epilogue threads meet at named barriers inside every tile, so
+        // they leave the tile loop together: the abort flag is agreed on at
+        // the start of a tile, and a wait that times out inside a tile skips
+        // the rest of its work but not its meeting points.
         uint32_t nblk = 0, ntile = 0, nchunk = 0;
         for (int item = pair; item < total; item += npairs, ++ntile) {
-            if constexpr (GATE_UP) {
-                if (epi_bar_or(aborted(ctl))) break;
-            } else {
-                if (aborted(ctl)) break;
-            }
+            if (epi_bar_or(aborted(ctl))) break;
             const Item it = decode(item, NW, mts, offs, E);
             // this CTA's weight rows exist (always for gate/up; for down, row
             // block 2 wt + half must lie inside the expert's d rows)
             const bool rows_ok = GATE_UP || it.wt * 2 + half < p.d / 128;
             const bool has_cols = ch * CW < it.N;
-            float acc[CW];
+            if constexpr (!GATE_UP) {
+                // down: a thread owns TMEM lane (output row) 32 q + lane and
+                // token columns ch*CW..+CW-1 (32x32b loads); its factors are the
+                // table's sa * sw of those columns, in column order
+                float acc[CW];
 #pragma unroll
-            for (int j = 0; j < CW; ++j) acc[j] = 0.f;
-            const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                    static_cast<uint32_t>(ch * CW);
-            bool ok = true;
-            for (int kb = 0; kb < nk && ok; ++kb) {
-                if (kb % TBL == 0) {  // the next chunk of factors
-                    const int slot = static_cast<int>(nchunk & 1u);
-                    const bool got = wait_bar(&ctl->tbl_full[slot], (nchunk >> 1) & 1u, ctl, p.status);
-                    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                    tbl = ctl->tbl[slot];
-                }
-                const int buf = static_cast<int>(nblk % NBUF);
-                // the whole warp goes on or stops together (the TMEM loads are warp-wide)
-                const bool got = wait_bar(&ctl->tfull[buf], (nblk / NBUF) & 1u, ctl, p.status);
-                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                tc_fence_after();
-                uint32_t v[2][32];
-                if (has_cols) {
-                    tmem_ld_32x32b_x32(t_lane + buf * TN, v[0]);
-                    tmem_ld_32x32b_x32(t_lane + buf * TN + 32, v[1]);
-                    tmem_ld_wait();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(&ctl->tempty[buf], 0);  // the leader's barrier
-                ++nblk;
-                if (has_cols) {
-                    const float4 (*row)[2] = tbl[kb % TBL] + ch * (CW / 4);
-#pragma unroll
-                    for (int j4 = 0; j4 < CW / 4; ++j4) {
-                        const float4 f = row[j4][role];
-                        acc[4 * j4 + 0] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 0) & 31]), f.x, acc[4 * j4 + 0]);
-                        acc[4 * j4 + 1] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 1) & 31]), f.y, acc[4 * j4 + 1]);
-                        acc[4 * j4 + 2] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 2) & 31]), f.z, acc[4 * j4 + 2]);
-                        acc[4 * j4 + 3] = fmaf(__uint_as_float(v[j4 >> 3][(4 * j4 + 3) & 31]), f.w, acc[4 * j4 + 3]);
+                for (int j = 0; j < CW; ++j) acc[j] = 0.f;
+                const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                        static_cast<uint32_t>(ch * CW);
+                bool ok = true;
+                int tslot = 0;
+                uint32_t v0[32], v1[32];
+                {
+                    const int buf = static_cast<int>(nblk % NBUF);
+                    const bool got = wait_bar(&ctl->tfull[buf], (nblk / NBUF) & 1u, ctl, p.status);
+                    if (!__all_sync(0xffffffffu, got)) ok = false;
+                    tc_fence_after();
+                    if (ok && has_cols) {
+                        tmem_ld_32x32b_x32(t_lane + buf * TN, v0);
+                        tmem_ld_wait(v0);
                     }
                 }
-                if (kb % TBL == TBL - 1 || kb == nk - 1) {  // done with this chunk of factors
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    if (kb % TBL == 0) {
+                        tslot = static_cast<int>(nchunk & 1u);
+                        const bool got = wait_bar(&ctl->tbl_full[tslot], (nchunk >> 1) & 1u, ctl, p.status);
+                        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                    }
+                    const int buf = static_cast<int>(nblk % NBUF);
+                    const float4 *f4 = reinterpret_cast<const float4 *>(&ctl->sa[tslot][kb % TBL][ch * CW]);
+                    if (has_cols) {
+                        tmem_ld_32x32b_x32(t_lane + buf * TN + 32, v1);
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 f = f4[j4];
+                            acc[4 * j4 + 0] = fmaf(__uint_as_float(v0[4 * j4 + 0]), f.x, acc[4 * j4 + 0]);
+                            acc[4 * j4 + 1] = fmaf(__uint_as_float(v0[4 * j4 + 1]), f.y, acc[4 * j4 + 1]);
+                            acc[4 * j4 + 2] = fmaf(__uint_as_float(v0[4 * j4 + 2]), f.z, acc[4 * j4 + 2]);
+                            acc[4 * j4 + 3] = fmaf(__uint_as_float(v0[4 * j4 + 3]), f.w, acc[4 * j4 + 3]);
+                        }
+                        tmem_ld_wait(v1);
+                    }
+                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->tbl_empty[static_cast<int>(nchunk & 1u)]);
-                    ++nchunk;
+                    if (lane == 0) mbar_arrive_remote(&ctl->tempty[buf], 0);  // the leader's barrier
+                    ++nblk;
+                    bool next = false;
+                    if (kb + 1 < nk) {
+                        const int nbuf = static_cast<int>(nblk % NBUF);
+                        const bool got = wait_bar(&ctl->tfull[nbuf], (nblk / NBUF) & 1u, ctl, p.status);
+                        if (!__all_sync(0xffffffffu, got)) ok = false;
+                        tc_fence_after();
+                        next = ok && has_cols;
+                        if (next) tmem_ld_32x32b_x32(t_lane + nbuf * TN, v0);
+                    }
+                    if (has_cols) {
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 f = f4[8 + j4];
+                            acc[32 + 4 * j4 + 0] = fmaf(__uint_as_float(v1[4 * j4 + 0]), f.x, acc[32 + 4 * j4 + 0]);
+                            acc[32 + 4 * j4 + 1] = fmaf(__uint_as_float(v1[4 * j4 + 1]), f.y, acc[32 + 4 * j4 + 1]);
+                            acc[32 + 4 * j4 + 2] = fmaf(__uint_as_float(v1[4 * j4 + 2]), f.z, acc[32 + 4 * j4 + 2]);
+                            acc[32 + 4 * j4 + 3] = fmaf(__uint_as_float(v1[4 * j4 + 3]), f.w, acc[32 + 4 * j4 + 3]);
+                        }
+                    }
+                    if (kb % TBL == TBL - 1 || kb == nk - 1) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ctl->tbl_empty[tslot]);
+                        ++nchunk;
+                    }
+                    if (next) tmem_ld_wait(v0);
                 }
-            }
-            if constexpr (!GATE_UP) {
-                if (!ok) break;
-                if (has_cols && rows_ok) {
+                if (has_cols && rows_ok && ok) {
                     const int n = it.wt * 2 * WM + half * WM + q * 32 + lane;
                     const int lim = it.rows - ch * CW;
                     __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) +
@@ -519,80 +620,165 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
-            // gate/up: the gate thread (lane < 16) finishes columns 0..31 of
-            // the warp's 64, the up thread (lane + 16) columns 32..63
-            float a[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float lo = acc[j], hi = acc[32 + j];
-                const float got = __shfl_xor_sync(0xffffffffu, is_up ? lo : hi, 16);
-                const float g = is_up ? got : lo;
-                const float u = is_up ? hi : got;
-                a[j] = __fdividef(g, 1.0f + __expf(-g)) * u;
-            }
-            // column maxima over the 16 features of the half-warp: a
-            // reduce-scatter butterfly leaves lane l with columns 2(l&15), +1
-            // of its 32 (non-negative floats order like their bit patterns)
-            float m[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) m[j] = fabsf(a[j]);
-#pragma unroll
-            for (int dist = 8, n = 32; dist >= 1; dist >>= 1, n >>= 1) {
-                const bool upper = (lane & dist) != 0;
-#pragma unroll
-                for (int i = 0; i < n / 2; ++i) {
-                    const float give = upper ? m[i] : m[i + n / 2];
-                    const float keep = upper ? m[i + n / 2] : m[i];
-                    m[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, dist));
-                }
-            }
-            const int cbase = ch * CW + (is_up ? 32 : 0);  // tile column of a[0]
-            const int cl = cbase + 2 * (lane & 15);
-            ctl->red_local[q][cl] = m[0];
-            ctl->red_local[q][cl + 1] = m[1];
-            epi_bar_sync();
-            const int par = static_cast<int>(ntile & 1u);
-            const int et = threadIdx.x - 64;  // epilogue thread 0..255
-            if (et < TN) {
-                const float cm = fmaxf(fmaxf(ctl->red_local[0][et], ctl->red_local[1][et]),
-                                       fmaxf(ctl->red_local[2][et], ctl->red_local[3][et]));
-                float *slot = &ctl->red_pair[par][half][et];
-                *slot = cm;
-                st_cluster_f32(peer_addr(slot, half ^ 1), cm);
-                mbar_arrive(&ctl->pair_red[par]);
-                mbar_arrive_remote_release(&ctl->pair_red[par], half ^ 1);
-            }
-            if (!mbar_wait_cluster(&ctl->pair_red[par], (ntile >> 1) & 1u,
-                                   globaltimer_ns() + kWaitNs)) {
-                set_status(p.status, kStatusTimeout);
-                atomicExch(&ctl->abort, 1);
-                ok = false;
-            }
-            const int ngo = p.I / kFp8Block;  // output groups per row
-            if (et < TN) {
-                const float amax = fmaxf(ctl->red_pair[par][0][et], ctl->red_pair[par][1][et]);
-                const float sc = __fdiv_rn(amax, 448.f);
-                ctl->col_scale[par][et] = sc;
-                if (half == 0 && et < it.rows)
-                    p.as_out[static_cast<size_t>(it.t0 + et) * ngo + it.wt] = sc;
-            }
-            epi_bar_sync();
-            if (has_cols && ok) {
-                const int f = it.wt * 128 + half * 64 + q * 16 + (lane & 15);
-                const int lim = it.rows - cbase;
-                uint8_t *dst = p.aq + static_cast<size_t>(it.t0 + cbase) * p.I + f;
+                // [4 i + 2 h + e]: fragment row fr + 8 h, column ch*CW + 8 i + 2 mq + e;
+                // ag from lanes 32q + 0..15, au from lanes 32q + 16..31
+                float ag[32], au[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    if (j < lim) {
-                        const float sc = ctl->col_scale[par][cbase + j];
-                        *dst = sc > 0.f ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(
-                                              __fdiv_rn(a[j], sc), __NV_SATFINITE, __NV_E4M3))
-                                        : static_cast<uint8_t>(0);
-                    }
-                    dst += p.I;
+                    ag[j] = 0.f;
+                    au[j] = 0.f;
                 }
-            }
-            }  // gate/up tile end
+                const uint32_t t_lo = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                      static_cast<uint32_t>(ch * CW);
+                const uint32_t t_hi = t_lo + (16u << 16);
+                bool ok = true;
+                int tslot = 0;
+                // Software pipeline: the load of the upper fragment is in flight
+                // while the lower one is promoted, and the lower fragment of K
+                // block kb + 1 while the upper one of kb is.
+                uint32_t vg[32], vu[32];
+                {
+                    const int buf = static_cast<int>(nblk % NBUF);
+                    const bool got = wait_bar(&ctl->tfull[buf], (nblk / NBUF) & 1u, ctl, p.status);
+                    if (!__all_sync(0xffffffffu, got)) ok = false;
+                    tc_fence_after();
+                    if (ok && has_cols) {
+                        tmem_ld_16x256b_x8(t_lo + buf * TN, vg);
+                        tmem_ld_wait(vg);
+                    }
+                }
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    if (kb % TBL == 0) {  // the next chunk of scales
+                        tslot = static_cast<int>(nchunk & 1u);
+                        const bool got = wait_bar(&ctl->tbl_full[tslot], (nchunk >> 1) & 1u, ctl, p.status);
+                        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                    }
+                    const int buf = static_cast<int>(nblk % NBUF);
+                    const float *sak = &ctl->sa[tslot][kb % TBL][ch * CW + mq * 16];
+                    const float2 w = ctl->sw[tslot][kb % TBL];
+                    if (has_cols) {
+                        tmem_ld_16x256b_x8(t_hi + buf * TN, vu);
+                        float sv[16];
+                        load_scales(sv, sak);
+                        promote(ag, vg, sv, w.x);
+                        tmem_ld_wait(vu);
+                    }
+                    // both fragments of this K block are in registers: its buffer is free
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(&ctl->tempty[buf], 0);  // the leader's barrier
+                    ++nblk;
+                    bool next = false;
+                    if (kb + 1 < nk) {
+                        const int nbuf = static_cast<int>(nblk % NBUF);
+                        const bool got = wait_bar(&ctl->tfull[nbuf], (nblk / NBUF) & 1u, ctl, p.status);
+                        if (!__all_sync(0xffffffffu, got)) ok = false;
+                        tc_fence_after();
+                        next = ok && has_cols;
+                        if (next) tmem_ld_16x256b_x8(t_lo + nbuf * TN, vg);
+                    }
+                    if (has_cols) {
+                        float sv[16];  // read again rather than held across the next load
+                        load_scales(sv, sak);
+                        promote(au, vu, sv, w.y);
+                    }
+                    if (kb % TBL == TBL - 1 || kb == nk - 1) {  // done with this chunk of scales
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ctl->tbl_empty[tslot]);
+                        ++nchunk;
+                    }
+                    if (next) tmem_ld_wait(vg);
+                }
+                // gate/up tile end: a = SiLU(gate) * up of fragment rows fr, fr + 8 (features
+                // 16 q + fr + 8 h of this CTA's 64), in place of ag
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float g = ag[j];
+                    ag[j] = __fdividef(g, 1.0f + __expf(-g)) * au[j];
+                }
+                // column maxima over the quarter's 16 features: the two rows of a
+                // thread, then a reduce-scatter butterfly over the 8 lanes of equal
+                // mq, which leaves lane l with columns ch*CW + 8 fr + 2 mq + {0, 1}
+                // (non-negative floats order like their bit patterns)
+                float m[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        m[2 * i + e] = fmaxf(fabsf(ag[4 * i + e]), fabsf(ag[4 * i + 2 + e]));
+                }
+#pragma unroll
+                for (int dist = 16, n = 16; dist >= 4; dist >>= 1, n >>= 1) {
+                    const bool upper = (lane & dist) != 0;
+#pragma unroll
+                    for (int i = 0; i < n / 2; ++i) {
+                        const float give = upper ? m[i] : m[i + n / 2];
+                        const float keep = upper ? m[i + n / 2] : m[i];
+                        m[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, dist));
+                    }
+                }
+                {
+                    const int cl = ch * CW + 8 * fr + 2 * mq;
+                    ctl->red_local[q][cl] = m[0];
+                    ctl->red_local[q][cl + 1] = m[1];
+                }
+                epi_bar_sync();
+                const int par = static_cast<int>(ntile & 1u);
+                if (et < TN) {
+                    const float cm = fmaxf(fmaxf(ctl->red_local[0][et], ctl->red_local[1][et]),
+                                           fmaxf(ctl->red_local[2][et], ctl->red_local[3][et]));
+                    float *slot = &ctl->red_pair[par][half][et];
+                    *slot = cm;
+                    st_cluster_f32(peer_addr(slot, half ^ 1), cm);
+                    mbar_arrive(&ctl->pair_red[par]);
+                    mbar_arrive_remote_release(&ctl->pair_red[par], half ^ 1);
+                }
+                if (!mbar_wait_cluster(&ctl->pair_red[par], (ntile >> 1) & 1u,
+                                       globaltimer_ns() + kWaitNs)) {
+                    set_status(p.status, kStatusTimeout);
+                    atomicExch(&ctl->abort, 1);
+                    ok = false;
+                }
+                const int ngo = p.I / kFp8Block;  // output groups per row
+                if (et < TN) {
+                    const float amax = fmaxf(ctl->red_pair[par][0][et], ctl->red_pair[par][1][et]);
+                    const float sc = __fdiv_rn(amax, 448.f);
+                    ctl->col_sr[par][et] = make_float2(sc, sc > 0.f ? __frcp_rn(sc) : 0.f);
+                    if (half == 0 && et < it.rows)
+                        p.as_out[static_cast<size_t>(it.t0 + et) * ngo + it.wt] = sc;
+                }
+                epi_bar_sync();
+                // codes through shared memory: [column][64 features of this CTA]
+                uint8_t *stg = ctl->stage;
+                if (has_cols && ok) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int c0 = ch * CW + 8 * i + 2 * mq;
+                        const float4 sr = *reinterpret_cast<const float4 *>(&ctl->col_sr[par][c0]);
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float sc = e ? sr.z : sr.x, rc = e ? sr.w : sr.y;
+                            uint8_t *row = stg + (c0 + e) * kPitchU8 + q * 16 + fr;
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                row[8 * h] = sc > 0.f ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(
+                                                            div_rn(ag[4 * i + 2 * h + e], sc, rc),
+                                                            __NV_SATFINITE, __NV_E4M3))
+                                                      : static_cast<uint8_t>(0);
+                        }
+                    }
+                }
+                epi_bar_sync();
+                if (ok) {
+                    // 4 chunks of 16 bytes per token row
+                    uint8_t *abase = p.aq + static_cast<size_t>(it.t0) * p.I + it.wt * 128 + half * 64;
+                    for (int x = et; x < it.rows * 4; x += kEpiThreads) {
+                        const int c = x >> 2, part = x & 3;
+                        const uint4 v = *reinterpret_cast<const uint4 *>(stg + c * kPitchU8 + part * 16);
+                        *reinterpret_cast<uint4 *>(abase + static_cast<size_t>(c) * p.I + part * 16) = v;
+                    }
+                }
+            }  // gate/up
         }
     }
 

@@ -55,6 +55,23 @@ void fp8_pair_free_maps(void *holder);
 int launch_fp8_pair_gate_up(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s);
 int launch_fp8_pair_down(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s);
 
+// a / b rounded to nearest (the IEEE quotient) from rb = RN(1/b) (__frcp_rn)
+// by Markstein's correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Develop.
+// 34(1), 1990): q0 = RN(a rb), r = a - q0 b formed inside a fused
+// multiply-add, q = RN(q0 + r rb). The result is the correctly rounded
+// quotient while nothing overflows or underflows; b outside [2^-100, 2^100]
+// takes the full division instead. Quotients that fall into the fp32
+// subnormal range may differ in the last place, which no e4m3 code can see
+// (every value below 2^-10 rounds to code 0). Tested against __fdiv_rn by
+// moe_selftest_fp8_divide.
+__device__ __forceinline__ float div_rn(float a, float b, float rb) {
+    if (!(b >= 0x1p-100f && b <= 0x1p100f)) return __fdiv_rn(a, b);
+    const float q0 = __fmul_rn(a, rb);
+    const float r = fmaf(-q0, b, a);
+    return fmaf(r, rb, q0);
+}
+
 // Grouped, quantised rows from the dispatch: codes [rows][d], scales [rows][d/128].
 int launch_dispatch_fp8(const DispatchParams &p, uint8_t *xq, float *xs, cudaStream_t s);
 

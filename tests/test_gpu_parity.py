@@ -530,3 +530,34 @@ def test_fp8_large_batch_deterministic_and_in_place():
     assert m.status() == 0
     assert torch.equal(a, b) and torch.equal(a, xi)
     m.close()
+
+
+def test_fp8_quantiser_division_is_the_ieee_quotient():
+    """The FP8 quantisers divide by a scale through its reciprocal and one
+    correction step; the quotient must equal the IEEE one bit for bit
+    wherever it is a normal float (the codes are e4m3 of it)."""
+    from sigmoid_bias_top_b200 import selftest_fp8_divide
+    g = torch.Generator().manual_seed(7)
+    n = 1 << 22
+    a = torch.randn(n, generator=g) * torch.exp2(torch.randint(-20, 21, (n,), generator=g).float())
+    # divisors as the quantisers meet them: amax / 448 over a wide range,
+    # plus significands with every bit set and exact powers of two
+    b = (torch.rand(n, generator=g) + 0.5) * torch.exp2(torch.randint(-40, 30, (n,), generator=g).float())
+    b[: n // 8] = torch.exp2(torch.randint(-40, 30, (n // 8,), generator=g).float())
+    ones = torch.tensor([float.fromhex("0x1.fffffep0")])
+    b[n // 8: n // 4] = ones * torch.exp2(torch.randint(-40, 30, (n // 8,), generator=g).float())
+    # numerators whose quotient lies next to a rounding midpoint
+    m = torch.randint(1 << 23, 1 << 24, (n // 8,), generator=g).double() + 0.5
+    a[n // 4: 3 * n // 8] = (m * b[n // 4: 3 * n // 8].double() * 2.0 ** -23).float()
+    a[:16] = 0.0
+    a[16:32] = -a[16:32]
+    b[32:48] = 2.0 ** -110      # outside the reciprocal's safe range:
+    b[48:64] = 2.0 ** 110       # the full division
+    b = b.to(DEV)
+    q, q_ref = selftest_fp8_divide(a.to(DEV), b)
+    torch.cuda.synchronize()
+    normal = q_ref.abs() >= 2.0 ** -126
+    assert torch.equal(q[normal].view(torch.int32), q_ref[normal].view(torch.int32))
+    assert torch.equal(q[q_ref == 0], q_ref[q_ref == 0])
+    # below the normal range both are tiny; e4m3 of either is code 0
+    assert (q[~normal & (q_ref != 0)].abs() < 2.0 ** -120).all()
