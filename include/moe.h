@@ -89,12 +89,16 @@ typedef struct moe_ctx moe_ctx;
  *   MOE_BF16: d % 64 == 0, d_ff % 64 == 0 (tensor-core tiles);
  *   MOE_FP8_BLOCK: d % 128 == 0, d_ff % 128 == 0 (whole scale blocks).
  * On success *out receives the context; on failure *out is set to NULL and
- * nothing stays allocated. Synchronous.
+ * nothing stays allocated. Synchronous. The workspace holds the grouped rows,
+ * the expert intermediates and outputs of max_tokens * top_k assignments;
+ * MOE_FP8_BLOCK layers add an fp32 [max_tokens * top_k][d_ff] buffer for the
+ * CTA-pair path (4 bytes per intermediate value; none with MOE_FP8_PAIR=0).
  * The kernels are chosen per forward from the batch size; two environment
  * variables, read here, force the choice between kernels that compute the
  * same result (for testing and tuning): MOE_TC_PAIR=0 (bf16 expert GEMMs
- * on single CTAs instead of the default CTA pairs) and MOE_ROUTE_TC=0|1 (SIMT or tensor-core
- * router for bf16 inputs). */
+ * on single CTAs instead of the default CTA pairs), MOE_ROUTE_TC=0|1 (SIMT or tensor-core
+ * router for bf16 inputs) and MOE_FP8_PAIR=0 (MOE_FP8_BLOCK batches of every
+ * size on the persistent FP8 kernel instead of the CTA-pair GEMMs). */
 int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
                const moe_weights *w, int max_tokens, moe_ctx **out);
 
@@ -146,8 +150,10 @@ int moe_profile(moe_ctx *h, int enable);
 int moe_kernel_times(moe_ctx *h, float *ms, int n);
 /* Name of kernel i of the last forward's launch sequence (static string), or
  * NULL: route, dispatch, gate_up, down, combine; or route, dispatch, experts,
- * combine when the batch was small enough for the fused expert kernel (and
- * always for MOE_FP8_BLOCK layers). */
+ * combine when the batch was small enough for the fused expert kernel (for
+ * MOE_FP8_BLOCK layers: the persistent FP8 kernel); or route, dispatch,
+ * gate_up, quantize, down, combine for MOE_FP8_BLOCK batches above that size
+ * (the CTA-pair FP8 GEMMs, SiLU(gate)*up quantised by its own kernel). */
 const char *moe_kernel_name(moe_ctx *h, int i);
 
 /* Number of kernel launches one forward makes for n_tokens tokens. */

@@ -28,7 +28,8 @@
 //     exactly one activation group of 128, so the group maximum is a max
 //     over the 128 TMEM lanes (a warp redux per column, then the four lane
 //     quadrants through shared memory, met at an mbarrier), s = amax / 448
-//     and the codes e4m3(a / s) (nearest-even, saturating) go to aq, s to as;
+//     and the codes e4m3(a / s) (the IEEE quotient, formed by div_rn;
+//     nearest-even, saturating) go to aq, s to as;
 //   down: y = the fp32 sum, rounded once to bf16.
 // Roles per CTA (320 threads): warp 0 lane 0 claims items and issues TMA
 // (and prefetches the item's block scales into L2); warp 1 owns TMEM (512
@@ -302,7 +303,9 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
             else promote<MAXT, false, NT, 1>(tq, buf, tg + row, tu + row, accg, accu);
         }
         tc_fence_before();
-        for (int k = 0; k < nkb; ++k) mbar_arrive(&ctl->tempty[(buf + k) % NBUF]);
+        __syncwarp();  // the whole warp's loads are done: one arrival per warp
+        if (lane == 0)
+            for (int k = 0; k < nkb; ++k) mbar_arrive(&ctl->tempty[(buf + k) % NBUF]);
         st.nblk += nkb;
         kb += nkb;
     }
@@ -344,11 +347,12 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
     if (!wait_bar(&ctl->red_bar[st.team][rb], (st.nred >> 1) & 1u, &ctl->abort, p.status))
         return false;
     ++st.nred;
-    float sl = 0.f;  // the scale of column lcol
+    float sl = 0.f, rl = 0.f;  // the scale of column lcol and RN(1 / scale)
     if (lserve) {
         const float amax = fmaxf(fmaxf(red[0][st.lcol], red[1][st.lcol]),
                                  fmaxf(red[2][st.lcol], red[3][st.lcol]));
         sl = __fdiv_rn(amax, 448.f);
+        rl = sl > 0.f ? __frcp_rn(sl) : 0.f;
     }
     if (st.q == 0 && lvalid) p.as[static_cast<size_t>(u.row0 + st.lcol) * ngi + u.tile] = sl;
     const int f = u.tile * WM + st.r;
@@ -357,10 +361,11 @@ __device__ __forceinline__ bool epi_unit(const Unit &u, Ctl<MAXT> *ctl, const Fp
 #pragma unroll
         for (int c = 0; c < CWW; ++c) {
             const float sc = __shfl_sync(0xffffffffu, sl, t * CWW + c);
+            const float rc = __shfl_sync(0xffffffffu, rl, t * CWW + c);
             const int col = t * TT + st.h2 * CWW + c;
             if (col < u.rows) {
                 const uint8_t code = sc > 0.f
-                    ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(accg[t * CWW + c], sc),
+                    ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(div_rn(accg[t * CWW + c], sc, rc),
                                                                  __NV_SATFINITE, __NV_E4M3))
                     : static_cast<uint8_t>(0);
                 p.aq[static_cast<size_t>(u.row0 + col) * p.I + f] = code;
@@ -412,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], Shape<MAXT>::TEAM_THREADS);  // the consuming team
+            mbar_init(&ctl->tempty[b], Shape<MAXT>::TEAM_THREADS / 32);  // the consuming team's warps
         }
         for (int r = 0; r < RING; ++r) {
             mbar_init(&ctl->ufull[r], 1);

@@ -9,8 +9,9 @@
 // verbraucht wie ein 2B-Modell", inferencekey.com, section "Für Engineers",
 // paragraph "Quantisierung": weights FP8 in static 128x128 blocks,
 // activations FP8 dynamic per group of 128):
-//   gate/up: aq, as = Q( silu(xq . Wg) * (xq . Wu) )  per group of 128 features
-//   down:    y      = bf16( aq . Wd )
+//   gate/up:  a32    = silu(xq . Wg) * (xq . Wu)        (fp32)
+//   quantise: aq, as = Q(a32)  per token and group of 128 features
+//   down:     y      = bf16( aq . Wd )
 // where every product over one 128-wide K block carries the weight block's
 // scale sw and the token group's scale sa.
 //
@@ -39,14 +40,14 @@
 // budget of 10 (the fullest of the four register-file quarters holds three
 // warps). In a gate/up tile the lower fragment holds gate and the upper one
 // up rows of the same features, so at the tile end each thread forms
-// SiLU(gate) * up for its 32 values in place; the group maximum over the
-// pair's 128 features per token is a reduce-scatter butterfly over the 8
-// lanes that share columns, then the four lane quarters through shared
-// memory, then the two CTAs through distributed shared memory (each writes
-// its maxima into both CTAs and arrives on both CTAs' barrier). s = amax / 448
-// and the codes e4m3(a / s) (the IEEE quotient, by a reciprocal and one
-// correction step: div_rn; nearest-even, saturating) are staged in shared
-// memory and written to aq as 16-byte row pieces, s to as.
+// SiLU(gate) * up for its 32 values and stores them in fp32 (each warp store
+// fills whole 32-byte sectors). A quantisation group of 128 features spans
+// both CTAs of a pair, so its maximum, s = amax / 448 and the codes
+// e4m3(a / s) (the IEEE quotient, by a reciprocal and one correction step:
+// div_rn; nearest-even, saturating) are left to a separate memory-bound
+// kernel (fp8_quantize_act_kernel): exchanging the maxima between the CTAs
+// and quantising inside the tile kept the epilogue from the next tile's
+// K blocks for longer than the whole quantisation pass takes.
 // All waits are bounded (1 s) and report MOE_ERR_DEVICE_TIMEOUT; the pair
 // meets at a cluster barrier before TMEM is freed. No load uses multicast.
 #include <cooperative_groups.h>
@@ -79,7 +80,6 @@ constexpr int kThreads = 64 + kEpiThreads + 32;
 constexpr int CW = TN / 2;               // token columns per epilogue warp
 constexpr int TBL = 16;                  // K blocks per chunk of a warp's factor table
 constexpr int kEpiBar = 1;               // named barrier of the epilogue threads
-constexpr int kPitchU8 = 64 + 16;        // staged gate/up codes: bytes per token row
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // shared::cluster address in the pair's even CTA
 
@@ -88,23 +88,17 @@ struct Ctl {
     uint64_t empty[STAGES];
     uint64_t tfull[NBUF];
     uint64_t tempty[NBUF];
-    uint64_t pair_red[2];       // gate/up: both CTAs' column maxima of a tile have arrived
     uint64_t tbl_full[2];       // a factor-table chunk is written
     uint64_t tbl_empty[2];      // every epilogue warp is done with it
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    float red_local[4][TN];     // per lane quarter: column maxima over its 16 features
-    float red_pair[2][2][TN];   // [tile parity][CTA][column]
-    alignas(16) float2 col_sr[2][TN];  // [tile parity][column]: (amax / 448, RN(1 / that))
     // two chunks of scales: per K block of the chunk, gate/up: the
     // activation scale sa of every token column in fragment order (frag_pos)
     // and the weight block scales sw of the gate and the up rows; down: the
     // factors sa * sw of the token columns in column order
     alignas(16) float sa[2][TBL][TN];
     float2 sw[2][TBL];
-    // a gate/up tile's codes on their way to global memory: [TN][kPitchU8] bytes
-    alignas(16) uint8_t stage[TN * kPitchU8];
 };
 
 // Position of token column c in a factor-table row: the epilogue thread with
@@ -216,44 +210,12 @@ __device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank) {
     return r;
 }
 
-// Arrival on the barrier at the same offset in CTA `rank`. The plain form
-// orders nothing beyond this thread's TMEM reads (fenced by the caller with
-// tcgen05.fence::before_thread_sync), which is all the TMEM buffer release
-// needs; the _release form also makes this thread's earlier shared-memory
-// writes to the peer (the column maxima) visible to its acquiring waiter.
+// Arrival on the barrier at the same offset in CTA `rank`. It orders nothing
+// beyond this thread's TMEM reads (fenced by the caller with
+// tcgen05.fence::before_thread_sync), which is all a TMEM buffer release needs.
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(peer_addr(bar, rank))
                  : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_remote_release(uint64_t *bar, uint32_t rank) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                     peer_addr(bar, rank))
-                 : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
-// Wait on a local barrier with cluster-scope acquire (remote arrivals release).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t dl) {
-    uint32_t ok = 0, it = 0;
-    while (true) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        if ((++it & 63u) == 0 && globaltimer_ns() > dl) return false;
-    }
-}
-
-__device__ __forceinline__ void epi_bar_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(kEpiBar), "n"(kEpiThreads) : "memory");
 }
 
 // The epilogue threads meet and learn whether any of them passed `v`.
@@ -335,7 +297,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&ctl->tempty[b], 2 * kEpiWarps);  // one per epilogue warp of both CTAs
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&ctl->pair_red[b], 2 * TN);  // TN local + TN remote
             mbar_init(&ctl->tbl_full[b], 1);
             mbar_init(&ctl->tbl_empty[b], kEpiWarps);
         }
@@ -523,7 +484,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int ch = ew >> 2;          // token columns ch*CW .. +CW-1
         const int mq = lane & 3;         // column pair of each 8 columns
         const int fr = lane >> 2;        // fragment rows fr and fr + 8
-        const int et = threadIdx.x - 64; // epilogue thread 0..255
         // The epilogue threads meet at named barriers inside every tile, so
         // they leave the tile loop together: the abort flag is agreed on at
         // the start of a tile, and a wait that times out inside a tile skips
@@ -689,93 +649,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     if (next) tmem_ld_wait(vg);
                 }
-                // gate/up tile end: a = SiLU(gate) * up of fragment rows fr, fr + 8 (features
-                // 16 q + fr + 8 h of this CTA's 64), in place of ag
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float g = ag[j];
-                    ag[j] = __fdividef(g, 1.0f + __expf(-g)) * au[j];
-                }
-                // column maxima over the quarter's 16 features: the two rows of a
-                // thread, then a reduce-scatter butterfly over the 8 lanes of equal
-                // mq, which leaves lane l with columns ch*CW + 8 fr + 2 mq + {0, 1}
-                // (non-negative floats order like their bit patterns)
-                float m[16];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-#pragma unroll
-                    for (int e = 0; e < 2; ++e)
-                        m[2 * i + e] = fmaxf(fabsf(ag[4 * i + e]), fabsf(ag[4 * i + 2 + e]));
-                }
-#pragma unroll
-                for (int dist = 16, n = 16; dist >= 4; dist >>= 1, n >>= 1) {
-                    const bool upper = (lane & dist) != 0;
-#pragma unroll
-                    for (int i = 0; i < n / 2; ++i) {
-                        const float give = upper ? m[i] : m[i + n / 2];
-                        const float keep = upper ? m[i + n / 2] : m[i];
-                        m[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, dist));
-                    }
-                }
-                {
-                    const int cl = ch * CW + 8 * fr + 2 * mq;
-                    ctl->red_local[q][cl] = m[0];
-                    ctl->red_local[q][cl + 1] = m[1];
-                }
-                epi_bar_sync();
-                const int par = static_cast<int>(ntile & 1u);
-                if (et < TN) {
-                    const float cm = fmaxf(fmaxf(ctl->red_local[0][et], ctl->red_local[1][et]),
-                                           fmaxf(ctl->red_local[2][et], ctl->red_local[3][et]));
-                    float *slot = &ctl->red_pair[par][half][et];
-                    *slot = cm;
-                    st_cluster_f32(peer_addr(slot, half ^ 1), cm);
-                    mbar_arrive(&ctl->pair_red[par]);
-                    mbar_arrive_remote_release(&ctl->pair_red[par], half ^ 1);
-                }
-                if (!mbar_wait_cluster(&ctl->pair_red[par], (ntile >> 1) & 1u,
-                                       globaltimer_ns() + kWaitNs)) {
-                    set_status(p.status, kStatusTimeout);
-                    atomicExch(&ctl->abort, 1);
-                    ok = false;
-                }
-                const int ngo = p.I / kFp8Block;  // output groups per row
-                if (et < TN) {
-                    const float amax = fmaxf(ctl->red_pair[par][0][et], ctl->red_pair[par][1][et]);
-                    const float sc = __fdiv_rn(amax, 448.f);
-                    ctl->col_sr[par][et] = make_float2(sc, sc > 0.f ? __frcp_rn(sc) : 0.f);
-                    if (half == 0 && et < it.rows)
-                        p.as_out[static_cast<size_t>(it.t0 + et) * ngo + it.wt] = sc;
-                }
-                epi_bar_sync();
-                // codes through shared memory: [column][64 features of this CTA]
-                uint8_t *stg = ctl->stage;
+                // gate/up tile end: a = SiLU(gate) * up of fragment rows fr, fr + 8
+                // (features 16 q + fr + 8 h of this CTA's 64) to a32 in fp32;
+                // a warp's store covers 8 consecutive features (one 32-byte
+                // sector) of 4 tokens
                 if (has_cols && ok) {
+                    float *abase = p.a32 + static_cast<size_t>(it.t0) * p.I + it.wt * 128 +
+                                   half * 64 + q * 16 + fr;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const int c0 = ch * CW + 8 * i + 2 * mq;
-                        const float4 sr = *reinterpret_cast<const float4 *>(&ctl->col_sr[par][c0]);
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
-                            const float sc = e ? sr.z : sr.x, rc = e ? sr.w : sr.y;
-                            uint8_t *row = stg + (c0 + e) * kPitchU8 + q * 16 + fr;
+                            const int c = ch * CW + 8 * i + 2 * mq + e;
+                            if (c < it.rows) {
+                                float *row = abase + static_cast<size_t>(c) * p.I;
 #pragma unroll
-                            for (int h = 0; h < 2; ++h)
-                                row[8 * h] = sc > 0.f ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(
-                                                            div_rn(ag[4 * i + 2 * h + e], sc, rc),
-                                                            __NV_SATFINITE, __NV_E4M3))
-                                                      : static_cast<uint8_t>(0);
+                                for (int h = 0; h < 2; ++h) {
+                                    const float g = ag[4 * i + 2 * h + e];
+                                    row[8 * h] = __fdividef(g, 1.0f + __expf(-g)) * au[4 * i + 2 * h + e];
+                                }
+                            }
                         }
-                    }
-                }
-                epi_bar_sync();
-                if (ok) {
-                    // 4 chunks of 16 bytes per token row
-                    uint8_t *abase = p.aq + static_cast<size_t>(it.t0) * p.I + it.wt * 128 + half * 64;
-                    for (int x = et; x < it.rows * 4; x += kEpiThreads) {
-                        const int c = x >> 2, part = x & 3;
-                        const uint4 v = *reinterpret_cast<const uint4 *>(stg + c * kPitchU8 + part * 16);
-                        *reinterpret_cast<uint4 *>(abase + static_cast<size_t>(c) * p.I + part * 16) = v;
                     }
                 }
             }  // gate/up
@@ -791,6 +685,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(TMEM_COLS)
                      : "memory");
+    }
+}
+
+// The e4m3 quantisation of SiLU(gate)*up per token and group of 128
+// features: a warp takes kQU groups of a row at a time (all loaded before any
+// is used), lane l holding features 4l..4l+3 of a group; amax = the group
+// maximum of |a|, s = amax / 448 and the codes e4m3(a / s) (both the IEEE
+// quotient, by div_rn; nearest-even, saturating), s to as.
+constexpr int kQU = 4;
+__global__ void __launch_bounds__(256) fp8_quantize_act_kernel(Fp8PairParams p) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int ngo = p.I / kFp8Block;
+    const int nch = (ngo + kQU - 1) / kQU;  // chunks of kQU groups per row
+    const int units = p.offsets[p.E] * nch;
+    const int nwarps = gridDim.x * (blockDim.x / 32);
+    const float r448 = __frcp_rn(448.f);
+    for (int u = (blockIdx.x * blockDim.x + threadIdx.x) / 32; u < units; u += nwarps) {
+        const int r = u / nch, g0 = (u - r * nch) * kQU;
+        const float *src = p.a32 + static_cast<size_t>(r) * p.I + 4 * lane;
+        uint8_t *dst = p.aq + static_cast<size_t>(r) * p.I + 4 * lane;
+        {
+            float4 v[kQU];
+#pragma unroll
+            for (int j = 0; j < kQU; ++j)
+                v[j] = g0 + j < ngo ? *reinterpret_cast<const float4 *>(src + (g0 + j) * kFp8Block)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < kQU; ++j) {
+                float m = fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w)));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (g0 + j >= ngo) continue;
+                const float sc = div_rn(m, 448.f, r448);
+                uint32_t code = 0;
+                if (sc > 0.f) {
+                    const float rc = __frcp_rn(sc);
+                    const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+                        make_float2(div_rn(v[j].x, sc, rc), div_rn(v[j].y, sc, rc)), __NV_SATFINITE, __NV_E4M3);
+                    const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                        make_float2(div_rn(v[j].z, sc, rc), div_rn(v[j].w, sc, rc)), __NV_SATFINITE, __NV_E4M3);
+                    code = lo | (hi << 16);
+                }
+                *reinterpret_cast<uint32_t *>(dst + (g0 + j) * kFp8Block) = code;
+                if (lane == 0) p.as_out[static_cast<size_t>(r) * ngo + g0 + j] = sc;
+            }
+        }
     }
 }
 
@@ -897,6 +839,11 @@ int launch_fp8_pair_gate_up(const void *holder, const Fp8PairParams &p, int n_sm
 
 int launch_fp8_pair_down(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s) {
     return launch<false>(static_cast<const Fp8PairMapsHolder *>(holder)->m, p, n_sm, s);
+}
+
+int launch_fp8_quantize_act(const Fp8PairParams &p, int n_sm, cudaStream_t s) {
+    if (p.I % kFp8Block != 0) return MOE_ERR_INVALID_ARG;
+    return launch_k(fp8_quantize_act_kernel, dim3(4 * n_sm), dim3(256), 0, s, p);
 }
 
 }  // namespace moe

@@ -48,6 +48,7 @@ struct moe_ctx {
     int fp8_pair_mode;   // -1 above the small-batch load, 0 never, 1 whenever not small
     uint8_t *xq, *aq;
     float *xs, *as;
+    float *a32;          // CTA-pair path: SiLU(gate)*up in fp32 [rows_cap][I] before quantisation
 
     void *ws;  // one allocation, carved below
     void *xp, *act, *y, *x_stage, *out_stage;
@@ -68,6 +69,7 @@ struct moe_ctx {
 
     int last_n;
     bool last_fused;  // the last forward used the fused small-batch expert kernel
+    bool last_fp8_pair;  // ... or the CTA-pair FP8 GEMMs with their quantiser between
 
     // profiling: a ring of event sets, one set (kEvPerFwd events) per forward
     bool profile;
@@ -80,6 +82,8 @@ struct moe_ctx {
 
 static const char *kKernelNames[] = {"route", "dispatch", "gate_up", "down", "combine"};
 static const char *kFusedKernelNames[] = {"route", "dispatch", "experts", "combine"};
+static const char *kFp8PairKernelNames[] = {"route", "dispatch", "gate_up", "quantize", "down",
+                                            "combine"};
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -208,6 +212,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
         (E + 1) * 4,                          // sched
         256,                                  // status
         3 * E * static_cast<size_t>(d) * 2,   // router_w3
+        (h->fp8 && h->fp8_pair_mode != 0) ? R * d_ff * 4 : 0,  // a32
     };
     const int nblocks = sizeof(sizes) / sizeof(sizes[0]);
     size_t total = 0, off[20];
@@ -238,6 +243,7 @@ extern "C" int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
     h->sched = reinterpret_cast<int32_t *>(b + off[16]);
     h->status = reinterpret_cast<int *>(b + off[17]);
     h->router_w3 = b + off[18];
+    h->a32 = reinterpret_cast<float *>(b + off[19]);
     if (h->fp8) {  // codes then scales, inside the (2-byte element) xp and act blocks
         h->xq = static_cast<uint8_t *>(h->xp);
         h->xs = reinterpret_cast<float *>(h->xq + R * d);
@@ -424,9 +430,11 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
         Fp8PairParams fp;
         fp.offsets = h->offsets; fp.mt_start = h->mt_start;
         fp.sgu = h->w.w_gate_up_scale; fp.sdn = h->w.w_down_scale;
-        fp.xs = h->xs; fp.as_in = h->as; fp.aq = h->aq; fp.as_out = h->as; fp.y = h->y;
-        fp.status = h->status; fp.E = h->E; fp.d = h->d; fp.I = h->I;
+        fp.xs = h->xs; fp.as_in = h->as; fp.a32 = h->a32; fp.aq = h->aq; fp.as_out = h->as;
+        fp.y = h->y; fp.status = h->status; fp.E = h->E; fp.d = h->d; fp.I = h->I;
         MOE_TRY(launch_fp8_pair_gate_up(h->fp8_pair_maps, fp, h->n_sm, s));
+        MOE_MARK();
+        MOE_TRY(launch_fp8_quantize_act(fp, h->n_sm, s));
         MOE_MARK();
         MOE_TRY(launch_fp8_pair_down(h->fp8_pair_maps, fp, h->n_sm, s));
         MOE_MARK();
@@ -480,6 +488,7 @@ static int forward_impl(moe_ctx *h, const void *x, void *out, int N, cudaStream_
     }
     h->last_n = N;
     h->last_fused = fused;
+    h->last_fp8_pair = fp8_pair;
     return MOE_OK;
 }
 
@@ -604,13 +613,14 @@ extern "C" int moe_kernel_times(moe_ctx *h, float *ms, int n) {
 extern "C" const char *moe_kernel_name(moe_ctx *h, int i) {
     if (!h) return nullptr;
     if (h->last_fused) return (i >= 0 && i < 4) ? kFusedKernelNames[i] : nullptr;
+    if (h->last_fp8_pair) return (i >= 0 && i < 6) ? kFp8PairKernelNames[i] : nullptr;
     return (i >= 0 && i < 5) ? kKernelNames[i] : nullptr;
 }
 
 extern "C" int moe_launches_per_forward(moe_ctx *h, int n_tokens) {
     if (!h) return MOE_ERR_INVALID_ARG;
     if (n_tokens <= 0) return 0;
-    return use_fused_experts(h, n_tokens) ? 4 : 5;
+    return use_fused_experts(h, n_tokens) ? 4 : use_fp8_pair(h, n_tokens) ? 6 : 5;
 }
 
 extern "C" int moe_selftest_timeout(moe_ctx *h, int timeout_us, void *stream) {

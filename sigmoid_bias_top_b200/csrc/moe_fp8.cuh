@@ -43,8 +43,9 @@ struct Fp8PairParams {
     const float *sdn;         // [E][d/128][I/128] block scales of w_down
     const float *xs;          // gate/up input: [rows][d/128] group scales of the grouped rows
     const float *as_in;       // down input: [rows][I/128] group scales of aq
-    uint8_t *aq;              // gate/up output: [rows][I] e4m3 codes of SiLU(gate)*up
-    float *as_out;            // gate/up output: [rows][I/128] their group scales
+    float *a32;               // gate/up output: [rows][I] fp32 SiLU(gate)*up
+    uint8_t *aq;              // quantiser output: [rows][I] e4m3 codes of a32
+    float *as_out;            // quantiser output: [rows][I/128] their group scales
     void *y;                  // down output: [rows][d] bf16
     int *status;
     int E, d, I;
@@ -54,6 +55,8 @@ int fp8_pair_build_maps(void **holder, const void *xq, const void *aq, const voi
 void fp8_pair_free_maps(void *holder);
 int launch_fp8_pair_gate_up(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s);
 int launch_fp8_pair_down(const void *holder, const Fp8PairParams &p, int n_sm, cudaStream_t s);
+// aq, as_out = the per-group-of-128 e4m3 quantisation of a32, rows offsets[E]
+int launch_fp8_quantize_act(const Fp8PairParams &p, int n_sm, cudaStream_t s);
 
 // a / b rounded to nearest (the IEEE quotient) from rb = RN(1/b) (__frcp_rn)
 // by Markstein's correction step (P. Markstein, "Computation of elementary

@@ -503,7 +503,7 @@ def test_fp8_pair_and_persistent_kernels_agree(shape):
     x = W.make_x(w, DEV)
     a = _fp8_layer_pair(w, layer, -1)
     b = _fp8_layer_pair(w, layer, 0)
-    assert a.launches_per_forward(w.n_tokens) == 5 and b.launches_per_forward(w.n_tokens) == 4
+    assert a.launches_per_forward(w.n_tokens) == 6 and b.launches_per_forward(w.n_tokens) == 4
     oa, ob = a(x), b(x)
     torch.cuda.synchronize()
     assert a.status() == 0 and b.status() == 0
@@ -521,8 +521,11 @@ def test_fp8_large_batch_deterministic_and_in_place():
     layer = W.make_layer(w, 0, DEV)
     x = W.make_x(w, DEV)
     m = MoeLayer(layer, w.top_k, w.eps, max_tokens=w.n_tokens)
-    assert m.launches_per_forward(w.n_tokens) == 5
+    assert m.launches_per_forward(w.n_tokens) == 6
+    m.profile(True)
     a = m(x)
+    assert list(m.kernel_times()) == ["route", "dispatch", "gate_up", "quantize", "down", "combine"]
+    m.profile(False)
     b = m(x)
     xi = x.clone()
     m(xi, out=xi)
