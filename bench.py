@@ -259,22 +259,39 @@ def measure(w, args, steps, world, rank, local, headline):
     outs = [torch.empty_like(xs[0]) for _ in range(2)]
     stream = torch.cuda.current_stream()
 
-    def step(i):
+    def step(i, st=None):
+        st = stream if st is None else st
         if w.n_layers > 1:  # chained blocks: h = x + MoE(RMSNorm(x))
             h = xs[i % len(xs)]
             for l, m in enumerate(mods):
                 dst = outs[l & 1]
-                m.forward(h, dst, stream)
+                m.forward(h, dst, st)
                 h = dst
         else:
             r = i % n_rot
-            mods[r].forward(xs[r % len(xs)], outs[i & 1], stream)
+            mods[r].forward(xs[r % len(xs)], outs[i & 1], st)
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
     for m in mods:
         assert m.status() == 0, m.status()
+    graph = None
+    if w.n_layers > 1:
+        # The stacked decode is timed as one CUDA graph holding all `steps`
+        # steps (every launch of the chained layers), replayed once per timed
+        # block: its thousands of small launches then cost no host time.
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            for i in range(steps):
+                step(i, gs)
+        stream.wait_stream(gs)
+        graph.replay()
+        torch.cuda.synchronize()
+        for m in mods:
+            assert m.status() == 0, m.status()
 
     # routing statistics of the timed batches (distinct active experts per layer)
     active = []
@@ -294,8 +311,11 @@ def measure(w, args, steps, world, rank, local, headline):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(steps):
-            step(i)
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(steps):
+                step(i)
         e1.record(stream)
         torch.cuda.synchronize()
         block_s.append(e0.elapsed_time(e1) / 1e3)
@@ -329,6 +349,8 @@ def measure(w, args, steps, world, rank, local, headline):
         "l2": (f"weights rotate over {n_rot} copies; each step streams one copy's active "
                "experts, >= 0.5 GB (> 126 MB L2)" if w.n_layers == 1
                else f"{w.n_layers} distinct layers, {w.n_layers * 1.21:.1f} GB per step (> L2)"),
+        "launch": ("one CUDA graph of the timed steps, replayed per block" if graph is not None
+                   else "eager launches through the C ABI"),
         "gpu_launches": mods[0].launches_per_forward(N) * steps * args.repeats
                         * (len(mods) if w.n_layers > 1 else 1),
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
