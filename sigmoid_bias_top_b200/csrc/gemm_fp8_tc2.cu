@@ -30,13 +30,13 @@
 // TMEM lane quarter, 64 token columns each) load it and add
 // partial * (sa[token][kb] * sw[kb]) into fp32 registers. The gate/up
 // epilogue loads 16x256b fragments, in which a thread holds 4 rows x 16 token
-// columns rather than 1 row x 64 columns, so it reads 16 activation scales
-// per K block (plus the two weight block scales) instead of 64 factors; the
-// down epilogue keeps one row per thread (32x32b) and reads the 64 factors
-// sa * sw, which lets it store 32 consecutive outputs of a token per warp
-// directly. An eleventh warp writes the scales of a chunk of 16 K blocks
-// ahead (two chunk buffers), in the order the fragments read them, issuing all
-// of a chunk's scale loads before using any; 11 warps keep the 168-register
+// columns rather than 1 row x 64 columns, so it reads 16 factors per K block
+// and fragment (sa * sw of the gate rows, then of the up rows) instead of 64;
+// the down epilogue keeps one row per thread (32x32b) and reads the 64
+// factors of its columns, which lets it store 32 consecutive outputs of a
+// token per warp directly. An eleventh warp forms the factors of a chunk of
+// 16 K blocks ahead (two chunk buffers), in the order the fragments read
+// them, issuing all of a chunk's scale loads before using any; 11 warps keep the 168-register
 // budget of 10 (the fullest of the four register-file quarters holds three
 // warps). In a gate/up tile the lower fragment holds gate and the upper one
 // up rows of the same features, so at the tile end each thread forms
@@ -93,12 +93,11 @@ struct Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    // two chunks of scales: per K block of the chunk, gate/up: the
-    // activation scale sa of every token column in fragment order (frag_pos)
-    // and the weight block scales sw of the gate and the up rows; down: the
-    // factors sa * sw of the token columns in column order
-    alignas(16) float sa[2][TBL][TN];
-    float2 sw[2][TBL];
+    // two chunks of promotion factors sa * sw, per K block of the chunk:
+    // gate/up: [0] with the gate rows' weight block scale, [1] with the up
+    // rows', each over the token columns in fragment order (frag_pos); down:
+    // [0] over the token columns in column order
+    alignas(16) float fac[2][TBL][2][TN];
 };
 
 // Position of token column c in a factor-table row: the epilogue thread with
@@ -139,15 +138,15 @@ __device__ __forceinline__ void load_scales(float (&sv)[16], const float *src) {
     }
 }
 
-// acc[4i + 2h + e] += v[4i + 2h + e] * sa[2i + e] * w, the factor rounded
-// to fp32 before the multiply-add
+// acc[4i + 2h + e] += v[4i + 2h + e] * f[2i + e] (f = sa * sw, formed in fp32
+// by the table warp)
 __device__ __forceinline__ void promote(float (&acc)[32], const uint32_t (&v)[32],
-                                        const float (&sv)[16], float w) {
+                                        const float (&sv)[16]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const float f = sv[2 * i + e] * w;
+            const float f = sv[2 * i + e];
             acc[4 * i + e] = fmaf(__uint_as_float(v[4 * i + e]), f, acc[4 * i + e]);
             acc[4 * i + 2 + e] = fmaf(__uint_as_float(v[4 * i + 2 + e]), f, acc[4 * i + 2 + e]);
         }
@@ -449,19 +448,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < TBL; ++j) sa[c][j] = (valid && j < n) ? __ldg(sa_row + j) : 0.f;
                 }
                 if constexpr (GATE_UP) {
-                    float *w2 = reinterpret_cast<float *>(&ctl->sw[slot][jj]);
-                    w2[lane < 16 ? 0 : 1] = wsc;
+                    int pos[4];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int pos = frag_pos(4 * lane + c);
+                    for (int c = 0; c < 4; ++c) pos[c] = frag_pos(4 * lane + c);
 #pragma unroll
-                        for (int j = 0; j < TBL; ++j) ctl->sa[slot][j][pos] = sa[c][j];
+                    for (int j = 0; j < TBL; ++j) {
+                        const float wg = __shfl_sync(0xffffffffu, wsc, j);
+                        const float wu = __shfl_sync(0xffffffffu, wsc, 16 + j);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            ctl->fac[slot][j][0][pos[c]] = sa[c][j] * wg;
+                            ctl->fac[slot][j][1][pos[c]] = sa[c][j] * wu;
+                        }
                     }
                 } else {
 #pragma unroll
                     for (int j = 0; j < TBL; ++j) {
                         const float w = __shfl_sync(0xffffffffu, wsc, j);
-                        *reinterpret_cast<float4 *>(&ctl->sa[slot][j][4 * lane]) =
+                        *reinterpret_cast<float4 *>(&ctl->fac[slot][j][0][4 * lane]) =
                             make_float4(sa[0][j] * w, sa[1][j] * w, sa[2][j] * w, sa[3][j] * w);
                     }
                 }
@@ -525,7 +529,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                     }
                     const int buf = static_cast<int>(nblk % NBUF);
-                    const float4 *f4 = reinterpret_cast<const float4 *>(&ctl->sa[tslot][kb % TBL][ch * CW]);
+                    const float4 *f4 = reinterpret_cast<const float4 *>(&ctl->fac[tslot][kb % TBL][0][ch * CW]);
                     if (has_cols) {
                         tmem_ld_32x32b_x32(t_lane + buf * TN + 32, v1);
 #pragma unroll
@@ -614,13 +618,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                     }
                     const int buf = static_cast<int>(nblk % NBUF);
-                    const float *sak = &ctl->sa[tslot][kb % TBL][ch * CW + mq * 16];
-                    const float2 w = ctl->sw[tslot][kb % TBL];
+                    const float *fgk = &ctl->fac[tslot][kb % TBL][0][ch * CW + mq * 16];
+                    const float *fuk = &ctl->fac[tslot][kb % TBL][1][ch * CW + mq * 16];
                     if (has_cols) {
                         tmem_ld_16x256b_x8(t_hi + buf * TN, vu);
                         float sv[16];
-                        load_scales(sv, sak);
-                        promote(ag, vg, sv, w.x);
+                        load_scales(sv, fgk);
+                        promote(ag, vg, sv);
                         tmem_ld_wait(vu);
                     }
                     // both fragments of this K block are in registers: its buffer is free
@@ -639,8 +643,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     if (has_cols) {
                         float sv[16];  // read again rather than held across the next load
-                        load_scales(sv, sak);
-                        promote(au, vu, sv, w.y);
+                        load_scales(sv, fuk);
+                        promote(au, vu, sv);
                     }
                     if (kb % TBL == TBL - 1 || kb == nk - 1) {  // done with this chunk of scales
                         __syncwarp();
