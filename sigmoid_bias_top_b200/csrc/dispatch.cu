@@ -80,13 +80,14 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float *scale) {
     for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float s = __fdiv_rn(m, 448.f);
+    const float s = div_rn(m, 448.f, __frcp_rn(448.f));  // the IEEE quotient m / 448
     uint32_t w[2] = {0u, 0u};
     if (s > 0.f) {
         const float rs = __frcp_rn(s);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {  // byte i of the 8 = value i
-            const uint32_t c = __nv_cvt_float_to_fp8(div_rn(v[i], s, rs), __NV_SATFINITE, __NV_E4M3);
+        for (int i = 0; i < 8; i += 2) {  // byte i of the 8 = value i (x of a pair in the low byte)
+            const uint32_t c = __nv_cvt_float2_to_fp8x2(
+                make_float2(div_rn(v[i], s, rs), div_rn(v[i + 1], s, rs)), __NV_SATFINITE, __NV_E4M3);
             w[i >> 2] |= c << (8 * (i & 3));
         }
     }
