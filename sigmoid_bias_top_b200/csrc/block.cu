@@ -39,6 +39,7 @@ constexpr size_t kPartialBytes = size_t(16) << 20;  // fp32 partial sums of spli
 // xn[r] = bf16(x[r] * rinv * gain), rinv = 1 / sqrt(mean(x[r]^2) + eps), one
 // warp per row (bf16 rows, d % 8 == 0). Block 0 also writes the one-group
 // tile plan of the GEMMs: loc = {0, N, 0, ceil(N / 256)}.
+template <int kNormU>
 __global__ void __launch_bounds__(kNormThreads)
     rmsnorm_rows_kernel(const __nv_bfloat16 *x, const float *gain, __nv_bfloat16 *xn,
                         int32_t *loc, int N, int d, float eps) {
@@ -56,34 +57,59 @@ __global__ void __launch_bounds__(kNormThreads)
     const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(r) * d);
     uint4 *dst = reinterpret_cast<uint4 *>(xn + static_cast<size_t>(r) * d);
     const int nv = d / 8;
+    // kNormU 16-byte vectors per lane are loaded before any is used (one
+    // memory round trip per 32 * kNormU vectors of the row instead of one per
+    // 32); each lane still adds its values in ascending column order
     float ss = 0.f;
-    for (int v = lane; v < nv; v += 32) {
-        const uint4 q = src[v];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    for (int base = 0; base < nv; base += 32 * kNormU) {
+        uint4 q[kNormU];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const float a = bf16_to_f32(w[h] & 0xFFFFu), b = bf16_to_f32(w[h] >> 16);
-            ss += a * a;
-            ss += b * b;
+        for (int u = 0; u < kNormU; ++u) {
+            const int v = base + u * 32 + lane;
+            q[u] = v < nv ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u) {
+            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float a = bf16_to_f32(w[h] & 0xFFFFu), b = bf16_to_f32(w[h] >> 16);
+                ss += a * a;
+                ss += b * b;
+            }
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rinv = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
-    for (int v = lane; v < nv; v += 32) {
-        const uint4 q = src[v];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-        const float4 g0 = *reinterpret_cast<const float4 *>(gain + v * 8);
-        const float4 g1 = *reinterpret_cast<const float4 *>(gain + v * 8 + 4);
-        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        uint32_t o[4];
+    for (int base = 0; base < nv; base += 32 * kNormU) {
+        uint4 q[kNormU];
+        float4 g[kNormU][2];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(bf16_to_f32(w[h] & 0xFFFFu) * rinv * gg[2 * h],
-                                                      bf16_to_f32(w[h] >> 16) * rinv * gg[2 * h + 1]);
-            o[h] = *reinterpret_cast<uint32_t *>(&b2);
+        for (int u = 0; u < kNormU; ++u) {
+            const int v = base + u * 32 + lane;
+            if (v < nv) {
+                q[u] = src[v];
+                g[u][0] = *reinterpret_cast<const float4 *>(gain + v * 8);
+                g[u][1] = *reinterpret_cast<const float4 *>(gain + v * 8 + 4);
+            }
         }
-        dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u) {
+            const int v = base + u * 32 + lane;
+            if (v >= nv) continue;
+            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+            const float gg[8] = {g[u][0].x, g[u][0].y, g[u][0].z, g[u][0].w,
+                                 g[u][1].x, g[u][1].y, g[u][1].z, g[u][1].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(bf16_to_f32(w[h] & 0xFFFFu) * rinv * gg[2 * h],
+                                                          bf16_to_f32(w[h] >> 16) * rinv * gg[2 * h + 1]);
+                o[h] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+            dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
 }
 
@@ -329,9 +355,13 @@ static cudaEvent_t *next_events(moe_block_ctx *h) {
     return p;
 }
 
+// Few rows: each warp keeps a whole 2048-wide row in flight (latency-bound:
+// 7.3 -> 5 us for 32 rows); many rows: one vector per lane at a time, which
+// keeps the occupancy that hides the latency there (8 in flight cost 13%).
 static int norm_launch(moe_block_ctx *h, const void *x, int N, cudaStream_t s) {
     const int blocks = (N + kNormThreads / 32 - 1) / (kNormThreads / 32);
-    return launch_k(rmsnorm_rows_kernel, dim3(blocks), dim3(kNormThreads), 0, s,
+    auto kern = N <= 512 ? rmsnorm_rows_kernel<8> : rmsnorm_rows_kernel<1>;
+    return launch_k(kern, dim3(blocks), dim3(kNormThreads), 0, s,
                     static_cast<const __nv_bfloat16 *>(x), h->gain, h->xn, h->loc, N, h->d,
                     h->eps);
 }
