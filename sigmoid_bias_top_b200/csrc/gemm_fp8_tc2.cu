@@ -35,10 +35,10 @@
 // the down epilogue keeps one row per thread (32x32b) and reads the 64
 // factors of its columns, which lets it store 32 consecutive outputs of a
 // token per warp directly. An eleventh warp forms the factors of a chunk of
-// 16 K blocks ahead (two chunk buffers), in the order the fragments read
-// them, issuing all of a chunk's scale loads before using any; 11 warps keep the 168-register
-// budget of 10 (the fullest of the four register-file quarters holds three
-// warps). In a gate/up tile the lower fragment holds gate and the upper one
+// 16 K blocks ahead (two chunk buffers), in the order the epilogue reads
+// them, issuing all of a chunk's scale loads before using any; 11 warps keep
+// the 168-register budget of 10 (the fullest of the four register-file
+// quarters holds three warps). In a gate/up tile the lower fragment holds gate and the upper one
 // up rows of the same features, so at the tile end each thread forms
 // SiLU(gate) * up for its 32 values and stores them in fp32 (each warp store
 // fills whole 32-byte sectors). A quantisation group of 128 features spans
@@ -78,7 +78,7 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kTblWarp = 2 + kEpiWarps;  // builds the tiles' factor tables
 constexpr int kThreads = 64 + kEpiThreads + 32;
 constexpr int CW = TN / 2;               // token columns per epilogue warp
-constexpr int TBL = 16;                  // K blocks per chunk of a warp's factor table
+constexpr int TBL = 16;                  // K blocks per chunk of the factor tables
 constexpr int kEpiBar = 1;               // named barrier of the epilogue threads
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // shared::cluster address in the pair's even CTA
@@ -477,21 +477,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
         // ---------------- epilogue (warps 2..9, both CTAs) ----------------
         // Warp (q, ch) owns TMEM lane quarter q and token columns ch*CW..+CW-1.
-        // It reads them as two 16x256b fragments: lanes 32q..+15 (gate rows of
-        // the quarter's 16 features, or down rows 32q..+15) and 32q+16..+31
-        // (the up rows of the same features, or down rows 32q+16..+31), so a
-        // thread holds, for fragment rows fr and fr + 8, 16 token columns
-        // ch*CW + 8 i + 2 mq + e of both: 16 activation scales per K block
-        // instead of one per column and register.
+        // gate/up reads them as two 16x256b fragments: lanes 32q..+15 (gate
+        // rows of the quarter's 16 features) and 32q+16..+31 (the up rows of
+        // the same features), so a thread holds, for fragment rows fr and
+        // fr + 8, 16 token columns ch*CW + 8 i + 2 mq + e of both: 16 factors
+        // per K block and fragment instead of one per column. down reads one
+        // row per thread (32x32b: lane 32q + lane, 64 columns).
         const int ew = warp - 2;
         const int q = warp & 3;          // TMEM lane quarter
         const int ch = ew >> 2;          // token columns ch*CW .. +CW-1
         const int mq = lane & 3;         // column pair of each 8 columns
         const int fr = lane >> 2;        // fragment rows fr and fr + 8
-        // The epilogue threads meet at named barriers inside every tile, so
-        // they leave the tile loop together: the abort flag is agreed on at
-        // the start of a tile, and a wait that times out inside a tile skips
-        // the rest of its work but not its meeting points.
+        // The epilogue threads agree at the start of every tile whether to
+        // stop (the abort flag), so they leave the tile loop together; a wait
+        // that times out inside a tile skips the rest of its work.
         uint32_t nblk = 0, ntile = 0, nchunk = 0;
         for (int item = pair; item < total; item += npairs, ++ntile) {
             if (epi_bar_or(aborted(ctl))) break;
