@@ -112,8 +112,10 @@ int moe_create(int d, int n_experts, int d_ff, int top_k, float eps,
 int moe_forward(moe_ctx *h, const void *x, void *out, int n_tokens, void *stream);
 
 /* Same as moe_forward for HOST buffers: copies x_host into device staging,
- * runs the forward and copies the result back into out_host, then waits for
- * the stream. Pinned host memory gives asynchronous copies; pageable works. */
+ * runs the forward and brings the result into out_host, then waits for the
+ * stream. With pinned out_host (device-mapped) the last kernel stores the
+ * rows into it directly; other memory gets a copy from device staging.
+ * Pinned x_host gives an asynchronous copy; pageable works. */
 int moe_forward_host(moe_ctx *h, const void *x_host, void *out_host, int n_tokens,
                      void *stream);
 

@@ -518,11 +518,24 @@ extern "C" int moe_forward_host(moe_ctx *h, const void *x_host, void *out_host, 
     if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = static_cast<size_t>(n_tokens) * h->d * h->elem;
+    // Pinned (page-locked) host memory is mapped into the device's address
+    // space: the last kernel then stores the rows there itself, and no copy
+    // back (with its own start-up) follows. Other host memory goes through
+    // the device staging buffer.
+    void *out_dev = nullptr;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, out_host) == cudaSuccess) {
+        if (attr.type == cudaMemoryTypeHost && attr.devicePointer && aligned16(attr.devicePointer))
+            out_dev = attr.devicePointer;
+    } else {
+        cudaGetLastError();  // pageable memory unknown to CUDA: not an error here
+    }
     if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return MOE_ERR_CUDA;
-    rc = forward_impl(h, h->x_stage, h->out_stage, n_tokens, s);
+    rc = forward_impl(h, h->x_stage, out_dev ? out_dev : h->out_stage, n_tokens, s);
     if (rc != MOE_OK) return rc;
-    if (cudaMemcpyAsync(out_host, h->out_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    if (!out_dev &&
+        cudaMemcpyAsync(out_host, h->out_stage, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     return cudaStreamSynchronize(s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -162,8 +162,15 @@ def test_deterministic_in_place_and_host_path():
     assert torch.equal(xi, a)
     xh = x.cpu().pin_memory()
     oh = torch.empty_like(xh).pin_memory()
-    m.forward_host(xh, oh)
+    m.forward_host(xh, oh)  # pinned: the last kernel stores into it
     assert torch.equal(oh, a.cpu())
+    op = torch.empty_like(x.cpu())
+    m.forward_host(xh, op)  # pageable: a copy from device staging
+    assert torch.equal(op, a.cpu())
+    big = torch.empty(xh.numel() + 4, dtype=xh.dtype).pin_memory()
+    om = big[4:].view_as(xh)  # pinned but 8 bytes off a 16-byte boundary: staging
+    m.forward_host(xh, om)
+    assert torch.equal(om, a.cpu())
     assert m.status() == 0
 
 
