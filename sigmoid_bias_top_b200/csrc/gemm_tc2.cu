@@ -40,6 +40,10 @@
 // up (kEpiSiluMul), a plain product g * v of paired rows (kEpiMul), a plain
 // store (kEpiPlain), the store plus a residual (kEpiResid), or the u stream
 // times the depthwise causal width-3 convolution of a stored a (kEpiConv).
+// The last two read an input of the output's shape; they move it and the
+// output in 16-byte rows through a 4 KB shared-memory tile per epilogue warp
+// (32 KB in all, beside the 192 KB of stages), so a chunk costs one memory
+// round trip instead of one per 16 scalar loads.
 #include <cooperative_groups.h>
 
 #include "moe_internal.cuh"
@@ -335,6 +339,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int q = warp & 3;            // TMEM lane quarter of this warp
         const int c_first = ((warp - 2) >> 2) * 64;  // its 64-column chunks, every kEpiWarps/4-th
         __nv_bfloat16 *c = static_cast<__nv_bfloat16 *>(p.c);
+        // the warp's 64 x 32 bf16 staging tile (kEpiResid, kEpiConv), after the expert tables
+        __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(
+                                   (reinterpret_cast<uintptr_t>(offs + E + 1) + 15) & ~static_cast<uintptr_t>(15)) +
+                               (warp - 2) * 64 * 32;
         int tile = 0;
         for (int item = pair; item < total && !aborted(ctl); item += npairs, ++tile) {
             const int buf = tile & 1;
@@ -379,7 +387,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 64; ++j)
                         if (j < lim) prow[static_cast<size_t>(c0 + j) * NOUT] = __uint_as_float(v[j >> 5][j & 31]);
                 }
-            } else if (GATE_UP) {
+            } else if constexpr (GATE_UP) {
                 // lanes 0..15: gate of features f, lanes 16..31: up of the same f
                 const bool is_gate = lane < 16;
                 const int f = it.wt * 128 + half * 64 + q * 16 + (lane & 15);
@@ -408,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-            } else {
+            } else if constexpr (MODE == kEpiPlain) {
                 const int n = it.wt * 2 * WM + half * WM + q * 32 + lane;
 #pragma unroll 1
                 for (int c0 = c_first; c0 < it.N; c0 += 64 * (kEpiWarps / 4)) {
@@ -418,73 +426,128 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tmem_ld_wait();
                     if (n < NOUT) {
                         const int lim = nvalid - c0;
-                        const size_t r0 = static_cast<size_t>(it.t0 + c0);
-                        __nv_bfloat16 *dst = c + r0 * NOUT + n;
-                        if constexpr (MODE == kEpiPlain) {
+                        __nv_bfloat16 *dst = c + static_cast<size_t>(it.t0 + c0) * NOUT + n;
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) {
+                            if (j < lim) *dst = __float2bfloat16_rn(__uint_as_float(v[j >> 5][j & 31]));
+                            dst += NOUT;
+                        }
+                    }
+                }
+            } else {
+                // kEpiResid: out = x + acc; kEpiConv: y = u * (k0 a_t + k1 a_{t-1} + k2 a_{t-2})
+                // per sequence. A warp's chunk is 64 token rows of its 32 channels
+                // n0..n0+31 (64 contiguous bytes per row). The rows of x or a come
+                // in by 16-byte loads, 8 per lane, issued before the TMEM loads
+                // (one memory round trip per chunk), and are staged in the warp's
+                // 4 KB of shared memory [row][32]; each thread then walks its own
+                // channel's column, overwriting every input with its output, and
+                // the chunk leaves by 16-byte stores from the same lanes and
+                // addresses as the loads. Each lane thus stores exactly the
+                // elements it loaded, so out may be x.
+                const int n0 = it.wt * 2 * WM + half * WM + q * 32;
+                const int n = n0 + lane;
+                const bool nval = n < NOUT;
+                const int vcol = n0 + (lane & 3) * 8;  // first channel of this lane's 16-byte column
+                const bool vval = vcol < NOUT;         // NOUT % 8 == 0: all 8 channels or none
+                const __nv_bfloat16 *src =
+                    static_cast<const __nv_bfloat16 *>(MODE == kEpiResid ? p.resid : p.aux);
+                __nv_bfloat16 *col = stage + lane;
+                float k0 = 0.f, k1 = 0.f, k2 = 0.f;
+                if (MODE == kEpiConv && nval) {
+                    k0 = p.conv[n * 3];
+                    k1 = p.conv[n * 3 + 1];
+                    k2 = p.conv[n * 3 + 2];
+                }
+#pragma unroll 1
+                for (int c0 = c_first; c0 < it.N; c0 += 64 * (kEpiWarps / 4)) {
+                    const int lim = nvalid - c0;
+                    const size_t r0 = static_cast<size_t>(it.t0 + c0);
+                    uint4 in[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int row = (lane >> 2) + 8 * i;
+                        in[i] = make_uint4(0u, 0u, 0u, 0u);
+                        if (vval && row < lim)
+                            in[i] = *reinterpret_cast<const uint4 *>(src + (r0 + row) * NOUT + vcol);
+                    }
+                    // kEpiConv: the two a values before the chunk, from a (same
+                    // sequence) or the sequence's carried state
+                    const int T = p.seq_len;
+                    int b = 0, t = 0;
+                    float am1 = 0.f, am2 = 0.f;
+                    auto hist = [&](int seq, int slot) {  // a of position slot - 2 of seq
+                        return p.state_in ? p.state_in[(static_cast<size_t>(seq) * 2 + slot) * NOUT + n] : 0.f;
+                    };
+                    if (MODE == kEpiConv && nval && lim > 0) {
+                        b = (it.t0 + c0) / T;  // rows < 2^30
+                        t = it.t0 + c0 - b * T;
+                        am1 = t >= 1 ? __bfloat162float(src[(r0 - 1) * NOUT + n]) : hist(b, 1);
+                        am2 = t >= 2 ? __bfloat162float(src[(r0 - 2) * NOUT + n])
+                                     : t == 1 ? hist(b, 1) : hist(b, 0);
+                    }
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(t_lane + c0, v[0]);
+                    tmem_ld_32x32b_x32(t_lane + c0 + 32, v[1]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<uint4 *>(stage + ((lane >> 2) + 8 * i) * 32 + (lane & 3) * 8) = in[i];
+                    __syncwarp();
+                    // every row of the stage is valid to read (rows past lim hold
+                    // zeros and are not stored), so the common paths run without a
+                    // branch per row and the shared-memory loads go out 32 at a time
+                    if (nval) {
+                        if (MODE == kEpiResid || t + min(lim, 64) <= T) {
+                            // kEpiConv: no sequence starts after the chunk's first row
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                float xin[32];
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) xin[j] = __bfloat162float(col[(h * 32 + j) * 32]);
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) {
+                                    const float acc = __uint_as_float(v[h][j]);
+                                    if constexpr (MODE == kEpiResid) {
+                                        col[(h * 32 + j) * 32] = __float2bfloat16_rn(xin[j] + acc);
+                                    } else {
+                                        const float cv = fmaf(k2, am2, fmaf(k1, am1, k0 * xin[j]));
+                                        col[(h * 32 + j) * 32] = __float2bfloat16_rn(acc * cv);
+                                        am2 = am1;
+                                        am1 = xin[j];
+                                    }
+                                }
+                            }
+                        } else {
+                            // kEpiConv across sequence starts: the window restarts
+                            // from the carried state of each new sequence
 #pragma unroll
                             for (int j = 0; j < 64; ++j) {
-                                if (j < lim) *dst = __float2bfloat16_rn(__uint_as_float(v[j >> 5][j & 31]));
-                                dst += NOUT;
-                            }
-                        } else if constexpr (MODE == kEpiResid) {
-                            // out = x + acc. out may be x, so a store may not move
-                            // ahead of the load of its own element: the loads of 16
-                            // rows are issued together, then their 16 stores (each
-                            // thread reads and writes only its own elements).
-                            const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(p.resid) +
-                                                      r0 * NOUT + n;
-#pragma unroll
-                            for (int j0 = 0; j0 < 64; j0 += 16) {
-                                float xv[16];
-#pragma unroll
-                                for (int j = 0; j < 16; ++j)
-                                    xv[j] = j0 + j < lim ? __bfloat162float(xr[static_cast<size_t>(j0 + j) * NOUT]) : 0.f;
-#pragma unroll
-                                for (int j = 0; j < 16; ++j)
-                                    if (j0 + j < lim)
-                                        dst[static_cast<size_t>(j0 + j) * NOUT] = __float2bfloat16_rn(
-                                            xv[j] + __uint_as_float(v[(j0 + j) >> 5][(j0 + j) & 31]));
-                            }
-                        } else {  // kEpiConv: y = u * (k0 a_t + k1 a_{t-1} + k2 a_{t-2}) per sequence
-                            // this thread's rows r0 .. r0+63 of channel n: a rolling
-                            // window over a, the two values before the chunk from a
-                            // (same sequence) or the sequence's carried state, the
-                            // chunk's own a loaded 16 rows at a time
-                            const __nv_bfloat16 *a = static_cast<const __nv_bfloat16 *>(p.aux) + n;
-                            const float k0 = p.conv[n * 3], k1 = p.conv[n * 3 + 1], k2 = p.conv[n * 3 + 2];
-                            const int T = p.seq_len;
-                            int b = static_cast<int>(r0 / T);
-                            int t = static_cast<int>(r0 - static_cast<size_t>(b) * T);
-                            auto hist = [&](int seq, int slot) {  // a of position slot - 2 of seq
-                                return p.state_in ? p.state_in[(static_cast<size_t>(seq) * 2 + slot) * NOUT + n] : 0.f;
-                            };
-                            float am1 = t >= 1 ? __bfloat162float(a[(r0 - 1) * NOUT]) : hist(b, 1);
-                            float am2 = t >= 2 ? __bfloat162float(a[(r0 - 2) * NOUT])
-                                               : t == 1 ? hist(b, 1) : hist(b, 0);
-#pragma unroll
-                            for (int j0 = 0; j0 < 64; j0 += 16) {
-                                float av[16];
-#pragma unroll
-                                for (int j = 0; j < 16; ++j)
-                                    av[j] = j0 + j < lim ? __bfloat162float(a[(r0 + j0 + j) * NOUT]) : 0.f;
-#pragma unroll
-                                for (int j = 0; j < 16; ++j) {
-                                    if (j0 + j < lim) {
-                                        if (t == 0) {  // a new sequence starts at this row
-                                            am1 = hist(b, 1);
-                                            am2 = hist(b, 0);
-                                        }
-                                        const float cv = fmaf(k2, am2, fmaf(k1, am1, k0 * av[j]));
-                                        dst[static_cast<size_t>(j0 + j) * NOUT] = __float2bfloat16_rn(
-                                            __uint_as_float(v[(j0 + j) >> 5][(j0 + j) & 31]) * cv);
-                                        am2 = am1;
-                                        am1 = av[j];
-                                        if (++t == T) { t = 0; ++b; }
+                                if (j < lim) {
+                                    const float acc = __uint_as_float(v[j >> 5][j & 31]);
+                                    const float xin = __bfloat162float(col[j * 32]);
+                                    if (t == 0) {  // a new sequence starts at this row
+                                        am1 = hist(b, 1);
+                                        am2 = hist(b, 0);
                                     }
+                                    const float cv = fmaf(k2, am2, fmaf(k1, am1, k0 * xin));
+                                    col[j * 32] = __float2bfloat16_rn(acc * cv);
+                                    am2 = am1;
+                                    am1 = xin;
+                                    if (++t == T) { t = 0; ++b; }
                                 }
                             }
                         }
                     }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int row = (lane >> 2) + 8 * i;
+                        if (vval && row < lim)
+                            *reinterpret_cast<uint4 *>(c + (r0 + row) * NOUT + vcol) =
+                                *reinterpret_cast<const uint4 *>(stage + row * 32 + (lane & 3) * 8);
+                    }
+                    __syncwarp();  // the stores' reads of the stage precede the next chunk's writes
                 }
             }
             tc_fence_before();
@@ -505,8 +568,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
 }
 
-size_t smem_bytes(int E) {
-    return 1024 + STAGES * STAGE_BYTES + sizeof(Ctl) + 2 * (E + 1) * sizeof(int32_t);
+constexpr size_t kStageBytes = 16 + kEpiWarps * 64 * 32 * 2;  // staging tiles + alignment
+
+size_t smem_bytes(int E, bool staged) {
+    return 1024 + STAGES * STAGE_BYTES + sizeof(Ctl) + 2 * (E + 1) * sizeof(int32_t) +
+           (staged ? kStageBytes : 0);
 }
 
 // CTA pairs that can be resident at once (an SM without a partner in its GPC
@@ -528,7 +594,7 @@ template <int MODE>
 int launch(const CUtensorMap &w, const CUtensorMap &t, const GroupedParams &p, int n_sm,
            cudaStream_t s) {
     auto kern = grouped_tc2_kernel<MODE>;
-    const size_t smem = smem_bytes(p.E);
+    const size_t smem = smem_bytes(p.E, MODE == kEpiResid || MODE == kEpiConv);
     if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_CUDA;
     static int pairs = 0;  // per kernel, for the device model of the process
     if (pairs == 0) pairs = resident_pairs(reinterpret_cast<const void *>(kern), smem, n_sm);

@@ -88,7 +88,9 @@ struct GroupedParams {
     int *status;
     int E, d, I, k;
     int rows_cap;             // allocated grouped rows (act, y)
-    // epilogue inputs of the dense and short-convolution blocks (CTA-pair kernel)
+    // epilogue inputs of the dense and short-convolution blocks (CTA-pair kernel);
+    // kEpiResid / kEpiConv move c, resid and aux in 16-byte pieces: d % 8 == 0
+    // and all three 16-byte aligned
     const void *resid;        // kEpiResid: [rows][d] added to the product
     const void *aux;          // kEpiConv: a [rows][d] (bf16), convolved along each sequence
     const float *conv;        // kEpiConv: taps [d][3] by lag
