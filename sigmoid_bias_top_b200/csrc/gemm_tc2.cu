@@ -20,8 +20,9 @@
 //     c rows are split into ceil(c/256) tiles of equal size rounded up to 16,
 //     so at most 15 padded columns per tile are computed, where 256-row tiles
 //     of the untransposed product would pad up to 255 rows per expert.
-// Per CTA a stage is 16 KB of weights and a 128-row box of tokens (16 KB, of
-// which the MMA reads N/2 rows), 6 stages.
+// Per CTA a stage is K = 128: two 64-wide boxes of weights (2 x 16 KB) and two
+// 128-row boxes of tokens (2 x 16 KB, of which the MMA reads N/2 rows), so
+// one barrier handshake covers eight MMAs; 3 stages.
 // Both CTAs' TMA loads complete on the leader's full barrier (the leader
 // expects the pair's bytes); the leader's single MMA thread issues the
 // cta_group::2 MMAs and its commits arrive on both CTAs' barriers
@@ -55,13 +56,18 @@ namespace {
 
 constexpr int WM = 128;       // weight rows per CTA (MMA M = 256 per pair)
 constexpr int TN = 256;       // most tokens per tile (MMA N)
-constexpr int BK = 64;
+constexpr int SUBK = 64;                          // K of one 128-byte-swizzled box
+constexpr int KSUB = 2;                           // boxes per operand and stage
+constexpr int BK = SUBK * KSUB;                   // K per stage
+static_assert(BK == kTcPairBK, "K per stage");
 constexpr int UK = 16;
-constexpr int STAGES = 6;
-constexpr int A_BYTES = WM * BK * 2;              // 16 KB
+constexpr int STAGES = 3;
 constexpr int B_ROWS = TN / 2;                    // token rows per CTA
-constexpr int B_BYTES = B_ROWS * BK * 2;          // one 128-row box (rows past N/2 unused)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB
+constexpr int A_SUB = WM * SUBK * 2;              // 16 KB
+constexpr int B_SUB = B_ROWS * SUBK * 2;          // one 128-row box (rows past N/2 unused)
+constexpr int A_BYTES = A_SUB * KSUB;
+constexpr int B_BYTES = B_SUB * KSUB;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 64 KB
 constexpr int TMEM_COLS = 2 * TN;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -274,12 +280,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (!wait_bar(&ctl->empty[s], ph ^ 1u, ctl, p.status)) { ok = false; break; }
                     uint8_t *sa = smem + s * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
-                    if (leader) mbar_arrive_expect_tx(&ctl->full[s], 2 * STAGE_BYTES);
-                    if (GATE_UP)
-                        tma_load_4d_pair(sa, &tmW, kb * BK, wc, &ctl->full[s]);
-                    else
-                        tma_load_2d_pair(sa, &tmW, kb * BK, wc, &ctl->full[s]);
-                    tma_load_2d_pair(sb, &tmT, kb * BK, trow, &ctl->full[s]);
+                    // boxes that start inside K (the last stage of a K that is
+                    // not a multiple of BK may hold one)
+                    const int nsub = min(KSUB, (K - kb * BK + SUBK - 1) / SUBK);
+                    if (leader) mbar_arrive_expect_tx(&ctl->full[s], 2 * nsub * (A_SUB + B_SUB));
+                    for (int j = 0; j < nsub; ++j) {
+                        const int x = kb * BK + j * SUBK;
+                        if (GATE_UP)
+                            tma_load_4d_pair(sa + j * A_SUB, &tmW, x, wc, &ctl->full[s]);
+                        else
+                            tma_load_2d_pair(sa + j * A_SUB, &tmW, x, wc, &ctl->full[s]);
+                        tma_load_2d_pair(sb + j * B_SUB, &tmT, x, trow, &ctl->full[s]);
+                    }
                     issued[s] = true;
                     issued_parity[s] = ph;
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -314,11 +326,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
                     const uint32_t b0 = a0 + A_BYTES;
+                    const int nsub = min(KSUB, (K - kb * BK + SUBK - 1) / SUBK);
 #pragma unroll
-                    for (int kk = 0; kk < BK / UK; ++kk)
-                        umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + kk * UK * 2),
-                                       sw128_kmajor_desc(b0 + kk * UK * 2), idesc,
-                                       (kb != kb0 || kk != 0) ? 1u : 0u);
+                    for (int j = 0; j < KSUB; ++j) {
+                        if (j < nsub) {
+#pragma unroll
+                            for (int kk = 0; kk < SUBK / UK; ++kk)
+                                umma_bf16_pair(d_tmem, sw128_kmajor_desc(a0 + j * A_SUB + kk * UK * 2),
+                                               sw128_kmajor_desc(b0 + j * B_SUB + kk * UK * 2), idesc,
+                                               (kb != kb0 || j != 0 || kk != 0) ? 1u : 0u);
+                        }
+                    }
                     any = true;
                     umma_commit_pair(&ctl->empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }

@@ -98,7 +98,7 @@ struct GroupedParams {
     int seq_len;              // kEpiConv: positions per sequence (rows are sequence-major)
     int wt_fastest;           // CTA-pair kernel: weight tiles vary fastest within an expert
     // split-K (CTA-pair kernel, kEpiPartial / kEpiPartialPaired): every tile
-    // in ksplit K slices of ceil(nk / ksplit) 64-wide blocks, none empty (the
+    // in ksplit K slices of ceil(nk / ksplit) kTcPairBK-wide blocks, none empty (the
     // caller picks ksplit so); slice ks writes fp32 sums to
     // partial[ks][row][width], row < partial_rows, width = NOUT (plain) or
     // 2 NOUT (paired: the first block's rows, then the partner rows)
@@ -115,7 +115,7 @@ constexpr int kEpiConv = 3;     // u * depthwise causal conv of a         (2-D w
 constexpr int kEpiResid = 4;    // residual + product                     (2-D weight map)
 constexpr int kEpiPartialPaired = 5;  // paired rows, fp32 partial sums of a K slice (4-D)
 constexpr int kEpiPartial = 6;        // fp32 partial sums of a K slice         (2-D weight map)
-constexpr int kTcPairBK = 64;         // K per stage of the CTA-pair kernel
+constexpr int kTcPairBK = 128;        // K per stage of the CTA-pair kernel
 
 struct DecodeParams {
     // the fused small-batch expert kernel (gate/up and down in one launch)
