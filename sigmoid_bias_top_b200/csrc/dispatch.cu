@@ -83,11 +83,19 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float *scale) {
     const float s = div_rn(m, 448.f, __frcp_rn(448.f));  // the IEEE quotient m / 448
     uint32_t w[2] = {0u, 0u};
     if (s > 0.f) {
-        const float rs = __frcp_rn(s);
+        // the half-warp's divisor is tested once for its 8 quotients per lane
+        float q[8];
+        if (div_rn_step_ok(s)) {
+            const float rs = __frcp_rn(s);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) q[i] = div_rn_step(v[i], s, rs);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(v[i], s);
+        }
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {  // byte i of the 8 = value i (x of a pair in the low byte)
-            const uint32_t c = __nv_cvt_float2_to_fp8x2(
-                make_float2(div_rn(v[i], s, rs), div_rn(v[i + 1], s, rs)), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(q[i], q[i + 1]), __NV_SATFINITE, __NV_E4M3);
             w[i >> 2] |= c << (8 * (i & 3));
         }
     }

@@ -725,11 +725,18 @@ __global__ void __launch_bounds__(256) fp8_quantize_act_kernel(Fp8PairParams p) 
                 const float sc = div_rn(m, 448.f, r448);
                 uint32_t code = 0;
                 if (sc > 0.f) {
-                    const float rc = __frcp_rn(sc);
-                    const uint32_t lo = __nv_cvt_float2_to_fp8x2(
-                        make_float2(div_rn(v[j].x, sc, rc), div_rn(v[j].y, sc, rc)), __NV_SATFINITE, __NV_E4M3);
-                    const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-                        make_float2(div_rn(v[j].z, sc, rc), div_rn(v[j].w, sc, rc)), __NV_SATFINITE, __NV_E4M3);
+                    // the group's divisor is tested once for its quotients
+                    float4 q;
+                    if (div_rn_step_ok(sc)) {
+                        const float rc = __frcp_rn(sc);
+                        q = make_float4(div_rn_step(v[j].x, sc, rc), div_rn_step(v[j].y, sc, rc),
+                                        div_rn_step(v[j].z, sc, rc), div_rn_step(v[j].w, sc, rc));
+                    } else {
+                        q = make_float4(__fdiv_rn(v[j].x, sc), __fdiv_rn(v[j].y, sc),
+                                        __fdiv_rn(v[j].z, sc), __fdiv_rn(v[j].w, sc));
+                    }
+                    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(q.x, q.y), __NV_SATFINITE, __NV_E4M3);
+                    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(q.z, q.w), __NV_SATFINITE, __NV_E4M3);
                     code = lo | (hi << 16);
                 }
                 *reinterpret_cast<uint32_t *>(dst + (g0 + j) * kFp8Block) = code;

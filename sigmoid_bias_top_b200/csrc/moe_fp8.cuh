@@ -67,12 +67,17 @@ int launch_fp8_quantize_act(const Fp8PairParams &p, int n_sm, cudaStream_t s);
 // takes the full division instead. Quotients that fall into the fp32
 // subnormal range may differ in the last place, which no e4m3 code can see
 // (every value below 2^-10 rounds to code 0). Tested against __fdiv_rn by
-// moe_selftest_fp8_divide.
-__device__ __forceinline__ float div_rn(float a, float b, float rb) {
-    if (!(b >= 0x1p-100f && b <= 0x1p100f)) return __fdiv_rn(a, b);
+// moe_selftest_fp8_divide. A caller with one divisor for many quotients tests
+// the range once (div_rn_step_ok) and takes div_rn_step or __fdiv_rn for all.
+__device__ __forceinline__ bool div_rn_step_ok(float b) { return b >= 0x1p-100f && b <= 0x1p100f; }
+__device__ __forceinline__ float div_rn_step(float a, float b, float rb) {
     const float q0 = __fmul_rn(a, rb);
     const float r = fmaf(-q0, b, a);
     return fmaf(r, rb, q0);
+}
+__device__ __forceinline__ float div_rn(float a, float b, float rb) {
+    if (!div_rn_step_ok(b)) return __fdiv_rn(a, b);
+    return div_rn_step(a, b, rb);
 }
 
 // Grouped, quantised rows from the dispatch: codes [rows][d], scales [rows][d/128].
