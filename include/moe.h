@@ -263,7 +263,8 @@ int moe_ep_destroy(moe_ep_ctx *h);
 
 /* Test hook of the FP8 quantisers' division: for n operand pairs (device
  * arrays), q[i] = a[i] / b[i] as the quantisers form it (a reciprocal and
- * one correction step) and q_ref[i] = the IEEE quotient; the two are equal
+ * one correction step, in paired fp32 operations where b[i] is in the step's
+ * range) and q_ref[i] = the IEEE quotient; the two are equal
  * bit for bit wherever the quotient is a normal float. Asynchronous on
  * stream. */
 int moe_selftest_fp8_divide(const float *a, const float *b, float *q, float *q_ref, int n,

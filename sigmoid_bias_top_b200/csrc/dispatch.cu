@@ -88,7 +88,11 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float *scale) {
         if (div_rn_step_ok(s)) {
             const float rs = __frcp_rn(s);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) q[i] = div_rn_step(v[i], s, rs);
+            for (int i = 0; i < 8; i += 2) {
+                const float2 qq = div_rn_step2(make_float2(v[i], v[i + 1]), s, rs);
+                q[i] = qq.x;
+                q[i + 1] = qq.y;
+            }
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(v[i], s);
@@ -251,11 +255,16 @@ __global__ void __launch_bounds__(kThreads, 4)
                     const float4 g1 = *reinterpret_cast<const float4 *>(g + 4);
                     const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
                     const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+                    // (x r) g per value, two values per paired multiply
                     float xnv[8];
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        xnv[2 * h] = bf16_to_f32(w[h] & 0xFFFFu) * r * gg[2 * h];
-                        xnv[2 * h + 1] = bf16_to_f32(w[h] >> 16) * r * gg[2 * h + 1];
+                        const float2 xr = __fmul2_rn(
+                            make_float2(bf16_to_f32(w[h] & 0xFFFFu), bf16_to_f32(w[h] >> 16)),
+                            make_float2(r, r));
+                        const float2 o = __fmul2_rn(xr, make_float2(gg[2 * h], gg[2 * h + 1]));
+                        xnv[2 * h] = o.x;
+                        xnv[2 * h + 1] = o.y;
                     }
                     float sc;
                     const uint2 codes = quant8(xnv, &sc);  // every lane takes part

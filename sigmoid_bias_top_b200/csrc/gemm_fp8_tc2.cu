@@ -729,8 +729,9 @@ __global__ void __launch_bounds__(256) fp8_quantize_act_kernel(Fp8PairParams p) 
                     float4 q;
                     if (div_rn_step_ok(sc)) {
                         const float rc = __frcp_rn(sc);
-                        q = make_float4(div_rn_step(v[j].x, sc, rc), div_rn_step(v[j].y, sc, rc),
-                                        div_rn_step(v[j].z, sc, rc), div_rn_step(v[j].w, sc, rc));
+                        const float2 qa = div_rn_step2(make_float2(v[j].x, v[j].y), sc, rc);
+                        const float2 qb = div_rn_step2(make_float2(v[j].z, v[j].w), sc, rc);
+                        q = make_float4(qa.x, qa.y, qb.x, qb.y);
                     } else {
                         q = make_float4(__fdiv_rn(v[j].x, sc), __fdiv_rn(v[j].y, sc),
                                         __fdiv_rn(v[j].z, sc), __fdiv_rn(v[j].w, sc));

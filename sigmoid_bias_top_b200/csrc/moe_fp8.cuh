@@ -79,6 +79,15 @@ __device__ __forceinline__ float div_rn(float a, float b, float rb) {
     if (!div_rn_step_ok(b)) return __fdiv_rn(a, b);
     return div_rn_step(a, b, rb);
 }
+// div_rn_step of two numerators over one divisor, in paired fp32 operations
+// (each component rounded as the scalar one; a - q0 b as fma(q0, -b, a), the
+// same exact product).
+__device__ __forceinline__ float2 div_rn_step2(float2 a, float b, float rb) {
+    const float2 rb2 = make_float2(rb, rb);
+    const float2 q0 = __fmul2_rn(a, rb2);
+    const float2 r = __ffma2_rn(q0, make_float2(-b, -b), a);
+    return __ffma2_rn(r, rb2, q0);
+}
 
 // Grouped, quantised rows from the dispatch: codes [rows][d], scales [rows][d/128].
 int launch_dispatch_fp8(const DispatchParams &p, uint8_t *xq, float *xs, cudaStream_t s);
