@@ -171,6 +171,25 @@ def test_deterministic_in_place_and_host_path():
     om = big[4:].view_as(xh)  # pinned but 8 bytes off a 16-byte boundary: staging
     m.forward_host(xh, om)
     assert torch.equal(om, a.cpu())
+    # pinned in and out: a captured graph, replayed while the buffers and the
+    # batch size stay; it reads the buffers' current contents
+    x2 = W.make_x(w, DEV, seed=w.seed + 1)
+    a2 = m(x2)
+    torch.cuda.synchronize()
+    for xin, ref in ((x, a), (x2, a2), (x, a)):
+        xh.copy_(xin.cpu())
+        oh.zero_()
+        m.forward_host(xh, oh)
+        assert torch.equal(oh, ref.cpu())
+    # another batch size into the same buffers: a new capture, then the old size again
+    h16 = xh[:16]
+    o16 = oh[:16]
+    ref16 = m(x[:16].contiguous())
+    torch.cuda.synchronize()
+    m.forward_host(h16, o16)
+    assert torch.equal(o16, ref16.cpu())
+    m.forward_host(xh, oh)
+    assert torch.equal(oh, a.cpu())
     assert m.status() == 0
 
 
